@@ -1,0 +1,212 @@
+/*
+ * w4a16.h -- C ABI of the W4A16 pack + matmul library (libw4a16.so, sm_100a).
+ *
+ * Block-scaled 4-bit weight-only linear layers: pack BF16 weight matrices to
+ * NVFP4 or ROCmFP4, then multiply BF16 activations by the packed weights.
+ *
+ * Sources (web pages on the subject):
+ *   [EdgeRock]  "EdgeRock-4B-NVFP4" model card, intro: the W4A16 NVFP4 format --
+ *               E2M1 4-bit weights, one FP8 E4M3 scale per 16 values and one
+ *               FP32 global scale per matrix; activations stay BF16.
+ *   [Nanbeige]  "Nanbeige4.2-3B-NVFP4A16" card, Creation: data-free
+ *               round-to-nearest quantisation, group 16; Serving: the fused
+ *               W4A16 kernel is the batch-1 decode path.
+ *   [rocmwhy]   "rocmwhy" ROCmFP4 research page, sections 01-03 and the format
+ *               table: Codebook10 levels 0,+-1,+-2,+-3,+-4,+-6,+-8,+-10; Dual
+ *               blocks (32 weights, two unsigned E4M3 half scales, 18 bytes,
+ *               4.50 bits/weight) and FAST blocks (one scale, 17 bytes, 4.25
+ *               bits/weight); scales chosen by exhaustive search over the
+ *               finite UE4M3 candidates scored by reconstruction error.
+ *
+ * Conventions shared by every entry point
+ *   - Matrices are "K-major": logical weight W is K x N (y = x . W) and is
+ *     stored as rows n = 0..N-1 of K contiguous elements, like the weight of a
+ *     torch Linear layer.  x is M x K row-major BF16, y is M x N row-major.
+ *   - Every pointer argument is caller-owned DEVICE memory (cudaMalloc or
+ *     equivalent) unless stated otherwise.  The library never allocates; the
+ *     scratch an operation needs is passed in as `workspace` (size from the
+ *     matching *_workspace_bytes query).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     asynchronous on it: arguments are validated on the host first and an
+ *     error is returned before anything is launched; a launch failure returns
+ *     W4_ERR_CUDA.  Device-side conditions (non-finite input, a bounded wait
+ *     that expired) are reported through `d_status` where the call has one,
+ *     and always through the sticky word read by w4_device_error().
+ *   - Device pointers must be 16-byte aligned (W4_ERR_ALIGN otherwise).
+ */
+#ifndef W4A16_H
+#define W4A16_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    W4_OK = 0,
+    W4_ERR_ARG = 1,          /* bad size, null pointer, bad enum */
+    W4_ERR_ALIGN = 2,        /* a pointer is not 16-byte aligned */
+    W4_ERR_UNSUPPORTED = 3,  /* valid request this build does not implement */
+    W4_ERR_CUDA = 4,         /* a CUDA call or launch failed */
+    W4_ERR_NONFINITE = 5,    /* NaN or Inf in a matrix given to a packer */
+    W4_ERR_TIMEOUT = 6,      /* a bounded device-side wait expired */
+    W4_ERR_WORKSPACE = 7     /* workspace missing or smaller than required */
+} w4_status;
+
+typedef enum {
+    W4_FMT_NVFP4 = 1,         /* [EdgeRock] E2M1 + E4M3 per 16 + FP32 global */
+    W4_FMT_ROCMFP4_DUAL = 2,  /* [rocmwhy] 18-byte blocks, two half scales   */
+    W4_FMT_ROCMFP4_FAST = 3   /* [rocmwhy] 17-byte blocks, one scale         */
+} w4_format;
+
+typedef enum {
+    W4_SCALE_ABSMAX = 0,  /* NVFP4 round-to-nearest abs-max recipe */
+    W4_SCALE_MSE = 1      /* exhaustive finite-scale error search */
+} w4_scale_search;
+
+/*
+ * A packed weight matrix (all pointers device memory, owned by the caller).
+ *   NVFP4:   codes  = [N][K/2] bytes; element k of row n sits in byte k/2, the
+ *                     even element in the low nibble.  Nibble = E2M1 code (bit 3
+ *                     sign, bits 2..1 exponent with bias 1, bit 0 mantissa).
+ *            scales = [N][K/16] E4M3FN bytes (one per 16 consecutive k).
+ *            global_scale = one float.  w_hat = e2m1 * scale * global.
+ *   ROCmFP4: codes  = [N][K/32] blocks of 18 (Dual) or 17 (FAST) bytes, blocks
+ *                     contiguous along K.  Dual block: byte 0 = scale of
+ *                     elements 0..15, byte 1 = scale of 16..31; FAST block:
+ *                     byte 0 = scale of all 32.  Then 16 code bytes, byte j =
+ *                     code[j] | code[j+16] << 4.  Code = Codebook10 nibble (bit
+ *                     3 sign, bits 2..0 index into 0,1,2,3,4,6,8,10).  Scale =
+ *                     unsigned E4M3 byte 0x00..0x7E.  w_hat = level * scale.
+ *            scales = NULL, global_scale = NULL.
+ */
+typedef struct {
+    int fmt;                     /* w4_format */
+    int K;                       /* reduction length (input features) */
+    int N;                       /* output features */
+    const uint8_t *codes;
+    const uint8_t *scales;
+    const float *global_scale;
+} w4_weights;
+
+/* ---------------------------------------------------------------- packers -- */
+
+/*
+ * pack_nvfp4 -- quantise a BF16 matrix to NVFP4 ([EdgeRock] intro; the
+ * round-to-nearest recipe of [Nanbeige] Creation):
+ *   global g = absmax(W) / (6 * 448)                      (binary32)
+ *   block scale s = E4M3(absmax(block) / 6 / g)           (two binary32 divisions,
+ *                                                          round to nearest even,
+ *                                                          saturate at 448)
+ *   code = E2M1(x / (s * g))                              (binary32, nearest even,
+ *                                                          saturate at 6, sign kept)
+ * g == 0, or a block whose s * g is 0, gives all-zero scales and codes.
+ *   W            [N][K] BF16, K % 16 == 0, K >= 16, N >= 1.
+ *   block        must be 16.
+ *   scale_search W4_SCALE_ABSMAX (W4_SCALE_MSE returns W4_ERR_UNSUPPORTED).
+ *   codes        out [N][K/2];  scales out [N][K/16];  global_scale out float.
+ *   workspace    >= pack_nvfp4_workspace_bytes() bytes of device scratch.
+ *   d_status     optional device int: set to W4_OK at the start of the call,
+ *                W4_ERR_NONFINITE if W holds NaN/Inf (outputs then undefined).
+ */
+w4_status pack_nvfp4(const void *W, int K, int N, int block, int scale_search,
+                     uint8_t *codes, uint8_t *scales, float *global_scale,
+                     void *workspace, size_t workspace_bytes, int *d_status,
+                     void *stream);
+size_t pack_nvfp4_workspace_bytes(void);
+
+/*
+ * pack_rocmfp4 -- quantise a BF16 matrix to ROCmFP4 Dual or FAST ([rocmwhy]
+ * sections 01-03).  For each scale group (16-weight half for Dual, the whole
+ * 32-weight block for FAST) every finite UE4M3 code u = 0x00..0x7E is tried:
+ * each weight takes the nearest Codebook10 level at scale dec(u) (ties to the
+ * even level index), and the group error E(u) = sum fma(d, d, E) over the
+ * weights in k order, d = x - level * dec(u), binary32.  The smallest E wins,
+ * ties to the smaller code.
+ *   W        [N][K] BF16, K % 32 == 0.
+ *   block    must be 32.  fmt = W4_FMT_ROCMFP4_DUAL or W4_FMT_ROCMFP4_FAST.
+ *   importance must be NULL (weighted error returns W4_ERR_UNSUPPORTED).
+ *   blocks   out [N][K/32][18 | 17] (layout as in w4_weights).
+ *   d_status optional, as for pack_nvfp4.
+ */
+w4_status pack_rocmfp4(const void *W, int K, int N, int block, int fmt,
+                       const float *importance, uint8_t *blocks, int *d_status,
+                       void *stream);
+
+/* ---------------------------------------------------------------- matmul --- */
+
+/*
+ * w4a16_gemv -- y[M][N] = x[M][K] . w_hat, fused dequantise-and-multiply for
+ * decode-sized M ([Nanbeige] Serving: the W4A16 kernel a decode step spends its
+ * weight bandwidth on).  Products and sums are binary32; the NVFP4 global scale
+ * is applied once per output.  The result is deterministic (fixed summation
+ * order for a given shape).
+ *   w        packed weights (any format); K % 32 == 0.
+ *   x        [M][K] BF16, 1 <= M <= 16.
+ *   y        out [M][N] float.
+ *   workspace>= w4a16_workspace_bytes(w, M) bytes (may be 0 -> NULL allowed).
+ */
+w4_status w4a16_gemv(const w4_weights *w, const void *x, int M, float *y,
+                     void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * w4a16_gemv_ex -- w4a16_gemv with launch flags.  W4_LAUNCH_PDL launches the
+ * kernel with programmatic dependent launch: it may start streaming weights
+ * while the previous kernel on the stream is still running, and reads x only
+ * after that kernel has completed.  Use inside a captured CUDA graph of
+ * back-to-back layers.
+ */
+#define W4_LAUNCH_PDL 1u
+w4_status w4a16_gemv_ex(const w4_weights *w, const void *x, int M, float *y,
+                        void *workspace, size_t workspace_bytes, unsigned flags,
+                        void *stream);
+
+/*
+ * w4a16_gemm -- y = x . w_hat for prefill-sized M: NVFP4 tiles are dequantised
+ * to BF16 in shared memory (e2m1 * scale, exact in BF16) and multiplied on the
+ * tensor cores with binary32 accumulation; the epilogue multiplies by the
+ * global scale and writes binary32 and/or BF16 (round to nearest even).
+ *   w        NVFP4 weights, K % 128 == 0.
+ *   x        [M][K] BF16, M >= 1.
+ *   y_f32    out [M][N] float, or NULL;  y_bf16 out [M][N] BF16, or NULL
+ *            (at least one of the two).
+ */
+w4_status w4a16_gemm(const w4_weights *w, const void *x, int M, float *y_f32,
+                     void *y_bf16, void *workspace, size_t workspace_bytes,
+                     void *stream);
+
+/* Scratch bytes w4a16_gemv / w4a16_gemm need for this shape (0 if none). */
+size_t w4a16_workspace_bytes(const w4_weights *w, int M);
+
+/* ------------------------------------------------------------- utilities --- */
+
+/*
+ * w4_encode_scalars -- the binary32 -> E4M3 (saturating, nearest even) and
+ * binary32 -> E2M1 (saturating, nearest even, sign kept) conversions the packers
+ * use, applied elementwise: e4m3[i] = E4M3(v[i]), e2m1[i] = E2M1(v[i]) (low
+ * nibble).  For checking conversions; v, e4m3, e2m1 are device arrays of n.
+ */
+w4_status w4_encode_scalars(const float *v, size_t n, uint8_t *e4m3, uint8_t *e2m1,
+                            void *stream);
+
+/*
+ * w4_device_error -- read (and, if clear != 0, reset) the library's sticky
+ * device error word on the current device: 0, or the w4_status of the first
+ * device-side failure (W4_ERR_TIMEOUT, W4_ERR_NONFINITE) since the last reset.
+ * Synchronises the device.
+ */
+w4_status w4_device_error(int *out, int clear);
+
+/* Human-readable name of a status code. */
+const char *w4_status_string(int status);
+
+/* Library version string. */
+const char *w4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A16_H */

@@ -58,6 +58,8 @@ def lib():
         L.orc_dequant_rocmfp4.argtypes = [P, I, I, I, I, P]
         L.orc_matmul.argtypes = [P, I, I, P, I, P, P]
         L.orc_set_threads.argtypes = [I]
+        L.orc_e4m3_encode_array.argtypes = [P, ctypes.c_longlong, P]
+        L.orc_e2m1_encode_array.argtypes = [P, ctypes.c_longlong, P]
         _lib = L
     return _lib
 
@@ -109,6 +111,20 @@ def e4m3_encode(v: float) -> int:
 
 def cb10_index(a: float, s: float) -> int:
     return lib().orc_cb10_index(a, s)
+
+
+def e4m3_encode_array(v) -> np.ndarray:
+    v = np.ascontiguousarray(v, np.float32)
+    out = np.zeros(v.shape, np.uint8)
+    lib().orc_e4m3_encode_array(_p(v), v.size, _p(out))
+    return out
+
+
+def e2m1_encode_array(v) -> np.ndarray:
+    v = np.ascontiguousarray(v, np.float32)
+    out = np.zeros(v.shape, np.uint8)
+    lib().orc_e2m1_encode_array(_p(v), v.size, _p(out))
+    return out
 
 
 # --- packers ------------------------------------------------------------------

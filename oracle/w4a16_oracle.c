@@ -386,3 +386,18 @@ void orc_set_threads(int n)
     (void)n;
 #endif
 }
+
+/* Elementwise encoders over arrays (for checking other implementations). */
+void orc_e4m3_encode_array(const float *v, long long n, uint8_t *out)
+{
+    #pragma omp parallel for schedule(static)
+    for (long long i = 0; i < n; i++)
+        out[i] = (uint8_t)orc_e4m3_encode(v[i]);
+}
+
+void orc_e2m1_encode_array(const float *v, long long n, uint8_t *out)
+{
+    #pragma omp parallel for schedule(static)
+    for (long long i = 0; i < n; i++)
+        out[i] = (uint8_t)orc_e2m1_encode(v[i]);
+}

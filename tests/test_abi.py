@@ -1,0 +1,65 @@
+"""The C-ABI library loads without a GPU and exports every entry point that
+include/w4a16.h declares; host-side argument checks answer before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import w4a16_matmul_pack_b200 as W4
+from w4a16_matmul_pack_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return W4.lib()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "w4a16.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*([a-z_0-9]+)\s*\(", text, re.M)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert {"pack_nvfp4", "pack_rocmfp4", "w4a16_gemv", "w4a16_gemm"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for s in range(8):
+        assert lib.w4_status_string(s).decode().startswith("W4_")
+    assert b"sm_100a" in lib.w4_version()
+
+
+def test_host_validation_without_gpu(lib):
+    P = ctypes.c_void_p
+    # null matrix / bad block size / bad format: rejected before any CUDA call
+    assert lib.pack_nvfp4(None, 64, 4, 16, 0, P(16), P(16), P(16), P(16), 16, None, None) == 1
+    assert lib.pack_nvfp4(P(16), 64, 4, 32, 0, P(16), P(16), P(16), P(16), 16, None, None) == 1
+    assert lib.pack_nvfp4(P(16), 64, 4, 16, 1, P(16), P(16), P(16), P(16), 16, None, None) == 3
+    assert lib.pack_nvfp4(P(16), 64, 4, 16, 0, P(16), P(16), P(16), P(16), 4, None, None) == 7
+    assert lib.pack_nvfp4(P(17), 64, 4, 16, 0, P(16), P(16), P(16), P(16), 16, None, None) == 2
+    assert lib.pack_rocmfp4(P(16), 48, 4, 32, 2, None, P(16), None, None) == 1
+    assert lib.pack_rocmfp4(P(16), 64, 4, 32, 9, None, P(16), None, None) == 1
+    assert lib.pack_rocmfp4(P(16), 64, 4, 32, 2, P(16), P(16), None, None) == 3
+    w = W4._Weights(1, 256, 8, 16, 16, 16)
+    assert lib.w4a16_gemv(ctypes.byref(w), P(16), 17, P(16), None, 0, None) == 1
+    assert lib.w4a16_gemv(ctypes.byref(w), P(16), 0, P(16), None, 0, None) == 1
+    assert lib.w4a16_gemv(ctypes.byref(w), P(24), 1, P(16), None, 0, None) == 2
+    bad = W4._Weights(7, 256, 8, 16, 16, 16)
+    assert lib.w4a16_gemv(ctypes.byref(bad), P(16), 1, P(16), None, 0, None) == 1
+    assert lib.w4a16_gemm(ctypes.byref(w), P(16), 4, None, None, None, 0, None) == 1
+
+
+def test_python_binding_refuses_cpu_tensors():
+    with pytest.raises(ValueError):
+        W4.pack_nvfp4(torch.zeros(4, 64, dtype=torch.bfloat16))
+    with pytest.raises(ValueError):
+        W4.pack_rocmfp4(torch.zeros(4, 64, dtype=torch.bfloat16), "dual")

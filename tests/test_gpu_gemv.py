@@ -1,0 +1,141 @@
+"""CUDA GEMV vs the oracle's binary64 matmul: |y - y_ref| <= 1e-3 * sum|x w_hat|.
+
+The packed weights given to the GPU are the oracle's own packing, so these
+tests check the matmul alone."""
+import os
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import w4a16_inputs as I
+import w4a16_matmul_pack_b200 as W4
+from gpu_util import assert_within_tolerance, np_of
+
+pytestmark = pytest.mark.gpu
+
+
+def nvfp4_packed(W):
+    c, s, g = O.pack_nvfp4(W)
+    pw = W4.PackedWeights(W4.FMT_NVFP4, W.shape[1], W.shape[0], torch.from_numpy(c).cuda(),
+                          torch.from_numpy(s).cuda(), torch.tensor([g], dtype=torch.float32).cuda())
+    return pw, O.dequant_nvfp4(c, s, g)
+
+
+def rocm_packed(W, fmt):
+    b = O.pack_rocmfp4(W, fmt)
+    return W4.PackedWeights(fmt, W.shape[1], W.shape[0], torch.from_numpy(b).cuda()), O.dequant_rocmfp4(b, fmt)
+
+
+def run_and_check(pw, w_hat, x, flags=0):
+    y = W4.w4a16_gemv(pw, x.cuda(), flags=flags)
+    yr, ar = O.matmul(x, w_hat)
+    assert_within_tolerance(np_of(y), yr, ar)
+    return y
+
+
+def test_nvfp4_small_case():
+    W, x = I.nvfp4_small()
+    pw, wh = nvfp4_packed(W)
+    run_and_check(pw, wh, x)
+
+
+@pytest.mark.parametrize("idx", range(5))
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_nvfp4_sweep(idx, M):
+    K, N = I.SWEEP_SHAPES[idx]
+    pw, wh = nvfp4_packed(I.sweep_weights(K, N, idx))
+    run_and_check(pw, wh, I.sweep_x(M, K, idx))
+
+
+@pytest.mark.parametrize("M", [2, 3, 5, 7, 8, 12])
+def test_nvfp4_other_m(M):
+    pw, wh = nvfp4_packed(I.sweep_weights(9728, 2560, 4))
+    run_and_check(pw, wh, I.sweep_x(M, 9728, 4))
+
+
+@pytest.mark.parametrize("N,K", [(1, 256), (7, 512), (333, 2560), (149, 1024), (2, 9728), (1000, 256)])
+@pytest.mark.parametrize("M", [1, 3, 16])
+def test_nvfp4_ragged(N, K, M):
+    pw, wh = nvfp4_packed(I.matrix("student_t4", N, K, N + K, 0.02, 1e-3))
+    run_and_check(pw, wh, I.activations(M, K, 9 + M))
+
+
+@pytest.mark.parametrize("fmt", [W4.FMT_ROCMFP4_DUAL, W4.FMT_ROCMFP4_FAST])
+@pytest.mark.parametrize("M", [1, 8])
+def test_rocm_laplace(fmt, M):
+    W = I.rocm_weights()[:1536].contiguous()
+    pw, wh = rocm_packed(W, fmt)
+    run_and_check(pw, wh, I.rocm_x(M))
+
+
+@pytest.mark.parametrize("fmt", [W4.FMT_ROCMFP4_DUAL, W4.FMT_ROCMFP4_FAST])
+@pytest.mark.parametrize("N,K,M", [(1, 512, 1), (77, 1024, 2), (5, 9728, 16), (300, 2560, 4)])
+def test_rocm_ragged(fmt, N, K, M):
+    pw, wh = rocm_packed(I.matrix("laplace", N, K, N * 3 + K, 0.015, 1e-3), fmt)
+    run_and_check(pw, wh, I.activations(M, K, 40 + M))
+
+
+def test_outlier_activations_and_zero_weights():
+    K, N = 2560, 512
+    W = I.sweep_weights(K, N, 1)[:N].clone()
+    W[:5] = 0
+    pw, wh = nvfp4_packed(W.contiguous())
+    x = I.activations(4, K, 3, outlier_cols=16, outlier_mult=30.0)
+    y = run_and_check(pw, wh, x)
+    assert torch.all(y[:, :5] == 0)
+
+
+def test_deterministic_and_pdl_flag_and_graph():
+    pw, wh = nvfp4_packed(I.sweep_weights(2560, 9728, 3))
+    x = I.sweep_x(1, 2560, 3).cuda()
+    y1 = W4.w4a16_gemv(pw, x)
+    y2 = W4.w4a16_gemv(pw, x)
+    y3 = W4.w4a16_gemv(pw, x, flags=W4.LAUNCH_PDL)
+    assert torch.equal(y1, y2) and torch.equal(y1, y3)
+    out = torch.empty_like(y1)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        W4.w4a16_gemv(pw, x, out=out, flags=W4.LAUNCH_PDL)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(3):
+            W4.w4a16_gemv(pw, x, out=out, flags=W4.LAUNCH_PDL)
+    out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, y1)
+    assert W4.w4_device_error(clear=True) == 0
+
+
+def test_unsupported_k_is_reported():
+    pw, _ = nvfp4_packed(I.matrix("normal", 4, 288, 1, 0.02))
+    with pytest.raises(W4.W4Error) as e:
+        W4.w4a16_gemv(pw, I.activations(1, 288, 1).cuda())
+    assert e.value.status == 3
+
+
+def test_save_reload_in_fresh_process(tmp_path):
+    """Pack on the GPU, write the bytes, reload them in a new process: the GEMV
+    output there is bit-identical (fresh-process reload check)."""
+    W = I.sweep_weights(2560, 1024, 1)
+    x = I.sweep_x(1, 2560, 1)
+    pw = W4.pack_nvfp4(W.cuda())
+    y = W4.w4a16_gemv(pw, x.cuda())
+    path = tmp_path / "packed.pt"
+    torch.save({"codes": pw.codes.cpu(), "scales": pw.scales.cpu(), "g": pw.global_scale.cpu(), "x": x,
+                "y": y.cpu()}, path)
+    code = (
+        "import torch, w4a16_matmul_pack_b200 as W4\n"
+        f"d = torch.load({str(path)!r})\n"
+        "pw = W4.PackedWeights(W4.FMT_NVFP4, 2560, 1024, d['codes'].cuda(), d['scales'].cuda(), d['g'].cuda())\n"
+        "y = W4.w4a16_gemv(pw, d['x'].cuda()).cpu()\n"
+        "assert torch.equal(y, d['y']), (y - d['y']).abs().max()\n"
+    )
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    subprocess.run([sys.executable, "-c", code], check=True, cwd=root,
+                   env={**os.environ, "PYTHONPATH": root})

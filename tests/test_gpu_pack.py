@@ -1,0 +1,100 @@
+"""CUDA packers vs the oracle: packed bytes, scales and global scale bit-exact."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import w4a16_inputs as I
+import w4a16_matmul_pack_b200 as W4
+from gpu_util import np_of
+
+pytestmark = pytest.mark.gpu
+
+
+def check_nvfp4(W):
+    pw = W4.pack_nvfp4(W.cuda())
+    c, s, g = O.pack_nvfp4(W)
+    torch.cuda.synchronize()
+    assert np.float32(pw.global_scale.item()).tobytes() == np.float32(g).tobytes()
+    assert np.array_equal(np_of(pw.scales), s)
+    gc = np_of(pw.codes)
+    bad = np.argwhere(gc != c)
+    assert bad.size == 0, f"{len(bad)} code bytes differ, first {bad[:4].tolist()}"
+
+
+def test_nvfp4_small_case():
+    W, _ = I.nvfp4_small()
+    check_nvfp4(W)
+
+
+@pytest.mark.parametrize("idx", range(5))
+def test_nvfp4_sweep_shapes(idx):
+    K, N = I.SWEEP_SHAPES[idx]
+    check_nvfp4(I.sweep_weights(K, N, idx))
+
+
+@pytest.mark.parametrize("N,K", [(1, 16), (3, 48), (7, 272), (1, 2560), (333, 160)])
+def test_nvfp4_ragged_and_minimum(N, K):
+    check_nvfp4(I.matrix("student_t4", N, K, 77 + N, 0.02, 1e-2))
+
+
+def test_nvfp4_zero_and_tiny():
+    check_nvfp4(torch.zeros(5, 64, dtype=torch.bfloat16))
+    W = torch.zeros(4, 64, dtype=torch.float64)
+    W[0, :16] = 2.0 ** -130          # bf16 subnormals
+    W[1, 3] = -(2.0 ** -133)
+    W[2, 20] = 1.0
+    W[3, 40:56] = torch.linspace(-1e-3, 1e-3, 16, dtype=torch.float64)
+    check_nvfp4(I.bf16_rne(W))
+    check_nvfp4(I.bf16_rne(W * 2.0 ** -100))   # global scale underflows to subnormal / zero
+
+
+def test_nvfp4_nonfinite_sets_status():
+    W = I.matrix("normal", 4, 64, 5, 0.02).cuda()
+    W[2, 7] = float("nan")
+    st = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    W4.w4_device_error(clear=True)
+    W4.pack_nvfp4(W, d_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 5
+    assert W4.w4_device_error(clear=True) == 5
+    st.fill_(-1)
+    W4.pack_nvfp4(I.matrix("normal", 4, 64, 5, 0.02).cuda(), d_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+
+
+def check_rocm(W, fmt):
+    code = W4.FMT_ROCMFP4_DUAL if fmt == "dual" else W4.FMT_ROCMFP4_FAST
+    pw = W4.pack_rocmfp4(W.cuda(), fmt)
+    ref = O.pack_rocmfp4(W, code)
+    got = np_of(pw.codes)
+    bad = np.argwhere(got != ref)
+    assert bad.size == 0, f"{len(bad)} bytes differ, first {bad[:4].tolist()}"
+
+
+@pytest.mark.parametrize("fmt", ["dual", "fast"])
+def test_rocm_laplace_matrix(fmt):
+    W = I.rocm_weights()
+    rows = torch.cat([torch.arange(0, 192), torch.arange(4800, 4864), torch.arange(9728 - 64, 9728)])
+    check_rocm(W[rows].contiguous(), fmt)
+
+
+@pytest.mark.parametrize("fmt", ["dual", "fast"])
+@pytest.mark.parametrize("N,K", [(1, 32), (5, 96), (3, 2560)])
+def test_rocm_ragged(fmt, N, K):
+    check_rocm(I.matrix("laplace", N, K, 11 * N + K, 0.015, 1e-2), fmt)
+
+
+@pytest.mark.parametrize("fmt", ["dual", "fast"])
+def test_rocm_degenerate(fmt):
+    W = torch.zeros(3, 64, dtype=torch.float64)
+    W[1, 5] = 10.6
+    W[1, 6:21] = 1.0
+    W[2, :] = 2.0 ** -130
+    check_rocm(I.bf16_rne(W), fmt)
+    check_rocm(torch.zeros(2, 64, dtype=torch.bfloat16), fmt)
+
+
+def test_full_laplace_matrix_dual():
+    check_rocm(I.rocm_weights(), "dual")

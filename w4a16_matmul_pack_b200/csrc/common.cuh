@@ -1,0 +1,155 @@
+// common.cuh -- device helpers for the sm_100a kernels: format conversions,
+// mbarrier / bulk-copy PTX wrappers, bounded waits, programmatic dependent
+// launch.  Single translation unit: included once from w4a16.cu.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "../../include/w4a16.h"
+
+namespace w4 {
+
+// Sticky device error word (w4_status of the first device-side failure).
+__device__ int g_device_error;
+
+// A wait on an mbarrier that takes longer than this is treated as a failure:
+// the kernel records W4_ERR_TIMEOUT and returns instead of spinning forever.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+
+__device__ __forceinline__ void record_error(int status) {
+    atomicCAS(&g_device_error, 0, status);
+}
+
+// ------------------------------------------------------------------ formats --
+
+// Two E2M1 codes in the low byte of `byte` (element 0 in the low nibble) ->
+// f16x2 with element 0 in the low half.  Exact (E2M1 values are f16 values).
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+        : "=r"(r) : "r"(byte));
+    return r;
+}
+
+// E4M3FN byte (low 8 bits) -> float.  Exact.
+__device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
+    uint32_t r;
+    uint16_t b = (uint16_t)(byte & 0xFF);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(b));
+    return __half2float(__ushort_as_half((unsigned short)(r & 0xFFFF)));
+}
+
+// float -> E4M3FN byte: round to nearest even, saturate to +-448, NaN -> 0x7F.
+__device__ __forceinline__ uint32_t f32_to_e4m3(float v) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(v));
+    return r & 0xFF;
+}
+
+// Two floats -> byte of two E2M1 codes (v0 in the low nibble): round to nearest
+// even, saturate to +-6.  The sign bit of each code is the sign bit of its input
+// (so -0 and negatives that round to zero give 0x8).
+__device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float v0, float v1) {
+    uint16_t r;
+    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u16.u8 %0, t;\n\t}"
+        : "=h"(r) : "f"(v1), "f"(v0));
+    uint32_t s = ((__float_as_uint(v0) >> 28) & 0x8u) | ((__float_as_uint(v1) >> 24) & 0x80u);
+    return ((uint32_t)r & 0x77u) | s;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+// ------------------------------------------------------------ async copies --
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                 ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for phase `parity` of an mbarrier, for at most kWaitLimitNs.  `abort`
+// is a CTA-shared flag: once any wait of the CTA has expired every later wait
+// returns false at once, so all threads run to the end of the kernel (and
+// through its barriers) instead of spinning.  Returns false on expiry/abort and
+// records W4_ERR_TIMEOUT.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = global_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort) return false;
+        if (global_ns() - t0 > kWaitLimitNs) {
+            *abort = 1;
+            record_error(W4_ERR_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+// Global -> shared bulk copy (no multicast), completion counted in bytes on `bar`.
+// dst, src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
+                                         uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+        "[%0], [%1], %2, [%3], %4;"
+        ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+
+// L2 policy: streamed-once data (packed weights) is evicted first.
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// Programmatic dependent launch.  Both are no-ops when the kernel was not
+// launched with the programmatic-serialization attribute.
+__device__ __forceinline__ void pdl_wait_prior_grid() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_allow_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;");
+}
+
+__device__ __forceinline__ void named_barrier_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+}  // namespace w4

@@ -1,0 +1,215 @@
+// pack.cuh -- NVFP4 and ROCmFP4 packers (sm_100a, CUDA cores).
+//
+// NVFP4 ("EdgeRock-4B-NVFP4" card, intro; round-to-nearest recipe of the
+// "Nanbeige4.2-3B-NVFP4A16" card, Creation):
+//   global g = absmax / (6 * 448); block scale s = E4M3(absmax_block / 6 / g);
+//   code = E2M1(x / (s * g)).  Two launches: an abs-max reduction into the
+//   workspace, then one thread per 16-element block.
+// ROCmFP4 ("rocmwhy" page, sections 01-03): for each scale group every finite
+//   UE4M3 code is scored by its binary32 reconstruction error with nearest
+//   Codebook10 levels; one warp per 32-weight block, lanes split the 127
+//   candidates, a lexicographic (error, code) shuffle reduction picks the
+//   winner (ties to the smaller code).
+#pragma once
+
+#include "common.cuh"
+
+namespace w4 {
+
+// ---------------------------------------------------------------- NVFP4 ----
+
+// ws[0]: max over |W| as bf16 magnitude bits (monotone in the value for finite
+// inputs); ws[1]: non-zero if any element is NaN or Inf.
+__global__ void __launch_bounds__(256) nvfp4_absmax_kernel(const uint4 *__restrict__ W, long long n8,
+                                                           unsigned *__restrict__ ws) {
+    unsigned m = 0, bad = 0;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8;
+         i += (long long)gridDim.x * blockDim.x) {
+        uint4 v = __ldg(W + i);
+        const unsigned w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            unsigned lo = w[j] & 0x7FFFu, hi = (w[j] >> 16) & 0x7FFFu;
+            bad |= (lo >= 0x7F80u) | (hi >= 0x7F80u);
+            m = max(m, max(lo, hi));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        bad |= __shfl_xor_sync(0xFFFFFFFFu, bad, o);
+    }
+    __shared__ unsigned sm[8], sb[8];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) {
+        sm[warp] = m;
+        sb[warp] = bad;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int i = 1; i < (int)(blockDim.x >> 5); i++) {
+            m = max(m, sm[i]);
+            bad |= sb[i];
+        }
+        if (m) atomicMax(ws, m);
+        if (bad) atomicOr(ws + 1, 1u);
+    }
+}
+
+// One thread per 16-element block; block b covers W[16b .. 16b+15] (rows are
+// K-contiguous and K % 16 == 0, so blocks never straddle rows).
+__global__ void __launch_bounds__(256) nvfp4_encode_kernel(const uint4 *__restrict__ W, long long nblocks,
+                                                           const unsigned *__restrict__ ws,
+                                                           uint2 *__restrict__ codes,
+                                                           uint8_t *__restrict__ scales,
+                                                           float *__restrict__ global_scale,
+                                                           int *__restrict__ d_status) {
+    const float amax = __uint_as_float(ws[0] << 16);
+    const float g = __fdiv_rn(amax, 2688.0f);  // absmax / (6 * 448)
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        *global_scale = g;
+        if (ws[1]) {
+            if (d_status) *d_status = W4_ERR_NONFINITE;
+            record_error(W4_ERR_NONFINITE);
+        }
+    }
+    for (long long b = blockIdx.x * (long long)blockDim.x + threadIdx.x; b < nblocks;
+         b += (long long)gridDim.x * blockDim.x) {
+        const uint4 v0 = __ldg(W + 2 * b), v1 = __ldg(W + 2 * b + 1);
+        const unsigned w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        float x[16];
+        float bamax = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            x[2 * j] = bf16_lo(w[j]);
+            x[2 * j + 1] = bf16_hi(w[j]);
+            bamax = fmaxf(bamax, fmaxf(fabsf(x[2 * j]), fabsf(x[2 * j + 1])));
+        }
+        uint32_t s = 0;
+        if (g != 0.0f) s = f32_to_e4m3(__fdiv_rn(__fdiv_rn(bamax, 6.0f), g));
+        const float d = __fmul_rn(e4m3_to_f32(s), g);
+        uint32_t c[2] = {0u, 0u};
+        if (d != 0.0f) {
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                const uint32_t byte = f32x2_to_e2m1x2(__fdiv_rn(x[2 * j], d), __fdiv_rn(x[2 * j + 1], d));
+                c[j >> 2] |= byte << (8 * (j & 3));
+            }
+        }
+        codes[b] = make_uint2(c[0], c[1]);
+        scales[b] = (uint8_t)s;
+    }
+}
+
+// -------------------------------------------------------------- ROCmFP4 ----
+
+// Binary32 reconstruction error of n weights (xs, in k order) at scale s with
+// nearest Codebook10 levels.  Level = nearest of s*{0,1,2,3,4,6,8,10}; the
+// midpoints s*{.5,1.5,2.5,3.5,5,7,9} are exact in binary32, and a tie goes to
+// the even level index, i.e. ">=" at the midpoints that lead to an even index
+// (1.5, 3.5, 7) and ">" at the others.
+template <int n>
+__device__ __forceinline__ float rocm_error(const float (&xs)[n], float s) {
+    const float t0 = s * 0.5f, t1 = s * 1.5f, t2 = s * 2.5f, t3 = s * 3.5f;
+    const float t4 = s * 5.0f, t5 = s * 7.0f, t6 = s * 9.0f;
+    float E = 0.0f;
+#pragma unroll
+    for (int i = 0; i < n; i++) {
+        const float a = fabsf(xs[i]);
+        float L = (a > t0 ? 1.0f : 0.0f) + (a >= t1 ? 1.0f : 0.0f) + (a > t2 ? 1.0f : 0.0f) +
+                  (a >= t3 ? 1.0f : 0.0f);
+        L += 2.0f * ((a > t4 ? 1.0f : 0.0f) + (a >= t5 ? 1.0f : 0.0f) + (a > t6 ? 1.0f : 0.0f));
+        const float d = __fsub_rn(a, __fmul_rn(s, L));
+        E = __fmaf_rn(d, d, E);
+    }
+    return E;
+}
+
+// Codebook10 code (bit 3 sign, bits 2..0 level index) of x at scale s.
+__device__ __forceinline__ uint32_t rocm_code(float x, float s) {
+    if (s == 0.0f) return 0u;
+    const float a = fabsf(x);
+    const uint32_t idx = (a > s * 0.5f) + (a >= s * 1.5f) + (a > s * 2.5f) + (a >= s * 3.5f) +
+                         (a > s * 5.0f) + (a >= s * 7.0f) + (a > s * 9.0f);
+    if (idx == 0) return 0u;
+    return idx | ((__float_as_uint(x) >> 28) & 8u);
+}
+
+// Lexicographic (error, code) minimum across `width` lanes (xor shuffles).
+__device__ __forceinline__ void argmin_lanes(float &E, uint32_t &u, int width) {
+    for (int o = width >> 1; o; o >>= 1) {
+        const float Eo = __shfl_xor_sync(0xFFFFFFFFu, E, o);
+        const uint32_t uo = __shfl_xor_sync(0xFFFFFFFFu, u, o);
+        if (Eo < E || (Eo == E && uo < u)) {
+            E = Eo;
+            u = uo;
+        }
+    }
+}
+
+// DUAL: lanes 0..15 search the scale of elements 0..15 (8 candidates each),
+// lanes 16..31 the scale of 16..31.  FAST: all 32 lanes search one scale (4
+// candidates each).  Lane l ends holding the winning scale of element l.
+template <bool DUAL>
+__global__ void __launch_bounds__(256) rocm_pack_kernel(const uint16_t *__restrict__ W, long long nblk,
+                                                        uint8_t *__restrict__ out,
+                                                        int *__restrict__ d_status) {
+    constexpr int BB = DUAL ? 18 : 17;
+    constexpr int NG = DUAL ? 16 : 32;  // weights per scale group
+    const int lane = threadIdx.x & 31;
+    const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+    for (long long blk = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5; blk < nblk; blk += warps) {
+        const uint32_t bits = __ldg(W + blk * 32 + lane);
+        const float xl = __uint_as_float(bits << 16);
+        if ((bits & 0x7F80u) == 0x7F80u) {
+            if (d_status) atomicExch(d_status, W4_ERR_NONFINITE);
+            record_error(W4_ERR_NONFINITE);
+        }
+        const int base = DUAL ? (lane & 16) : 0;
+        float xs[NG];
+#pragma unroll
+        for (int i = 0; i < NG; i++) xs[i] = __shfl_sync(0xFFFFFFFFu, xl, base + i);
+
+        float bestE = 0.0f;
+        uint32_t bestU = 0xFFu;
+        const int sub = DUAL ? (lane & 15) : lane;
+#pragma unroll 1
+        for (int t = 0; t < (DUAL ? 8 : 4); t++) {
+            const uint32_t u = (uint32_t)(sub + t * NG);
+            if (u > 0x7Eu) break;
+            const float E = rocm_error<NG>(xs, e4m3_to_f32(u));
+            if (bestU == 0xFFu || E < bestE) {
+                bestE = E;
+                bestU = u;
+            }
+        }
+        argmin_lanes(bestE, bestU, NG);
+
+        const uint32_t code = rocm_code(xl, e4m3_to_f32(bestU));
+        const uint32_t hi = __shfl_down_sync(0xFFFFFFFFu, code, 16);
+        uint8_t *o = out + blk * BB;
+        if (DUAL) {
+            const uint32_t u1 = __shfl_sync(0xFFFFFFFFu, bestU, 16);
+            if (lane == 0) {
+                o[0] = (uint8_t)bestU;
+                o[1] = (uint8_t)u1;
+            }
+        } else if (lane == 0) {
+            o[0] = (uint8_t)bestU;
+        }
+        if (lane < 16) o[(DUAL ? 2 : 1) + lane] = (uint8_t)(code | (hi << 4));
+    }
+}
+
+// Elementwise conversion check kernel (the packers' encoders on raw floats).
+__global__ void encode_scalars_kernel(const float *__restrict__ v, long long n, uint8_t *__restrict__ e4,
+                                      uint8_t *__restrict__ e2) {
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+         i += (long long)gridDim.x * blockDim.x) {
+        const float x = v[i];
+        if (e4) e4[i] = (uint8_t)f32_to_e4m3(x);
+        if (e2) e2[i] = (uint8_t)(f32x2_to_e2m1x2(x, 0.0f) & 0xFu);
+    }
+}
+
+}  // namespace w4

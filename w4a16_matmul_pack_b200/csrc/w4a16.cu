@@ -1,0 +1,313 @@
+// w4a16.cu -- the C ABI of libw4a16.so (declared in include/w4a16.h): host-side
+// validation, launch configuration and launches of the sm_100a kernels.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+#include "pack.cuh"
+#include "gemv.cuh"
+#include "gemm.cuh"
+
+using namespace w4;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    int sms = 0;
+    int smem_optin = 0;
+};
+
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+w4_status device_info(DeviceInfo &out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return W4_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceInfo &d = g_dev[dev];
+    if (d.sms == 0) {
+        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) {
+            d.sms = 0;
+            return W4_ERR_CUDA;
+        }
+    }
+    out = d;
+    return W4_OK;
+}
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline w4_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
+inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// ------------------------------------------------------------------ GEMV ----
+
+constexpr size_t kXBudget = 64 * 1024;      // shared bytes for the x slice
+constexpr int kTileTarget = 24 * 1024;      // bytes per pipeline stage
+
+inline int gemv_rows_per_task(int M) { return M <= 2 ? 4 : (M <= 4 ? 2 : 1); }
+
+// Alignment unit of K for the bulk-copy path: row pieces must start on 16 bytes.
+inline int k_unit(int fmt) { return fmt == W4_FMT_ROCMFP4_FAST ? 512 : 256; }
+
+struct GemvPlan {
+    int S = 1, kc = 0, TR = 0, P = 0, NS = 0, tile_bytes = 0, grid = 0;
+    size_t smem = 0;
+    size_t ws_bytes = 0;
+};
+
+int piece_bytes(int fmt, int kc) {
+    if (fmt == W4_FMT_NVFP4) return kc / 2 + kc / 16;
+    return (kc / 32) * (fmt == W4_FMT_ROCMFP4_DUAL ? 18 : 17);
+}
+
+w4_status plan_gemv(int fmt, int K, int N, int M, bool pdl, GemvPlan &p) {
+    DeviceInfo d;
+    if (device_info(d) != W4_OK) return W4_ERR_CUDA;
+    const int unit = k_unit(fmt);
+    // split-K slices so that x[M][kc] fits the x budget
+    const int units = K / unit;
+    int per = (int)std::max<size_t>(1, kXBudget / ((size_t)2 * M * unit));
+    per = std::min(per, units);
+    p.kc = per * unit;
+    p.S = (units + per - 1) / per;
+    const int R = gemv_rows_per_task(M);
+    const int rowB = piece_bytes(fmt, p.kc);
+    int TR = R;
+    while (TR * 2 <= 8 * R && TR * 2 * rowB <= kTileTarget) TR *= 2;
+    p.TR = TR;
+    p.P = 8 * R / TR;
+    p.tile_bytes = (TR * rowB + 127) & ~127;
+    const size_t xs = ((size_t)M * p.kc * 2 + 127) & ~(size_t)127;
+    const size_t red = (size_t)2 * TR * p.P * M * 4 + 16;  // + abort flag
+    const size_t budget = std::min<size_t>(pdl ? 110 * 1024 : 200 * 1024, (size_t)d.smem_optin);
+    int NS = 8;
+    while (NS > 2 && xs + (size_t)NS * p.tile_bytes + red + 16 * NS > budget) NS--;
+    p.NS = NS;
+    p.smem = xs + (size_t)NS * p.tile_bytes + red + 16 * NS;
+    if (p.smem > (size_t)d.smem_optin) return W4_ERR_UNSUPPORTED;
+    p.grid = std::min(d.sms, N);
+    p.ws_bytes = p.S > 1 ? (size_t)p.S * M * N * sizeof(float) : 0;
+    return W4_OK;
+}
+
+template <int FMT, int M>
+w4_status launch_gemv_m(const w4_weights *w, const void *x, float *y, void *ws, const GemvPlan &p, bool pdl,
+                        cudaStream_t st) {
+    constexpr int R = M <= 2 ? 4 : (M <= 4 ? 2 : 1);
+    auto kern = gemv_kernel<FMT, M, R>;
+    static size_t configured = 0;  // largest dynamic smem size set so far for this instantiation
+    if (p.smem > configured) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem) != cudaSuccess)
+            return W4_ERR_CUDA;
+        configured = p.smem;
+    }
+    GemvArgs a;
+    a.codes = w->codes;
+    a.scales = w->scales;
+    a.gscale = w->global_scale;
+    a.x = reinterpret_cast<const uint16_t *>(x);
+    a.y = y;
+    a.partial = reinterpret_cast<float *>(ws);
+    a.K = w->K;
+    a.N = w->N;
+    a.kc = p.kc;
+    a.TR = p.TR;
+    a.P = p.P;
+    a.NS = p.NS;
+    a.tile_bytes = p.tile_bytes;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.grid, p.S, 1);
+    cfg.blockDim = dim3(kGemvThreads, 1, 1);
+    cfg.dynamicSmemBytes = p.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return W4_ERR_CUDA;
+    if (p.S > 1) {
+        const int MN = M * w->N;
+        gemv_finalize_kernel<<<std::min((MN + 255) / 256, 1024), 256, 0, st>>>(
+            a.partial, p.S, MN, FMT == W4_FMT_NVFP4 ? w->global_scale : nullptr, y);
+    }
+    return launch_status();
+}
+
+template <int FMT>
+w4_status launch_gemv_fmt(const w4_weights *w, const void *x, int M, float *y, void *ws, const GemvPlan &p,
+                          bool pdl, cudaStream_t st) {
+    switch (M) {
+#define W4_CASE(m) \
+    case m: return launch_gemv_m<FMT, m>(w, x, y, ws, p, pdl, st);
+        W4_CASE(1) W4_CASE(2) W4_CASE(3) W4_CASE(4) W4_CASE(5) W4_CASE(6) W4_CASE(7) W4_CASE(8)
+        W4_CASE(9) W4_CASE(10) W4_CASE(11) W4_CASE(12) W4_CASE(13) W4_CASE(14) W4_CASE(15) W4_CASE(16)
+#undef W4_CASE
+    }
+    return W4_ERR_ARG;
+}
+
+w4_status check_weights(const w4_weights *w) {
+    if (!w || !w->codes || w->K <= 0 || w->N <= 0) return W4_ERR_ARG;
+    if (w->fmt == W4_FMT_NVFP4) {
+        if (!w->scales || !w->global_scale || w->K % 16) return W4_ERR_ARG;
+        if (!aligned16(w->codes) || !aligned16(w->scales) || (reinterpret_cast<uintptr_t>(w->global_scale) & 3))
+            return W4_ERR_ALIGN;
+    } else if (w->fmt == W4_FMT_ROCMFP4_DUAL || w->fmt == W4_FMT_ROCMFP4_FAST) {
+        if (w->K % 32) return W4_ERR_ARG;
+        if (!aligned16(w->codes)) return W4_ERR_ALIGN;
+    } else {
+        return W4_ERR_ARG;
+    }
+    return W4_OK;
+}
+
+}  // namespace
+
+// ======================================================================== ABI
+
+extern "C" {
+
+size_t pack_nvfp4_workspace_bytes(void) { return 16; }
+
+w4_status pack_nvfp4(const void *W, int K, int N, int block, int scale_search, uint8_t *codes, uint8_t *scales,
+                     float *global_scale, void *workspace, size_t workspace_bytes, int *d_status, void *stream) {
+    if (!W || !codes || !scales || !global_scale || K < 16 || N < 1 || K % 16 || block != 16) return W4_ERR_ARG;
+    if (scale_search == W4_SCALE_MSE) return W4_ERR_UNSUPPORTED;
+    if (scale_search != W4_SCALE_ABSMAX) return W4_ERR_ARG;
+    if (!workspace || workspace_bytes < pack_nvfp4_workspace_bytes()) return W4_ERR_WORKSPACE;
+    if (!aligned16(W) || !aligned16(codes) || !aligned16(scales) || !aligned16(workspace) ||
+        (reinterpret_cast<uintptr_t>(global_scale) & 3) || (reinterpret_cast<uintptr_t>(d_status) & 3))
+        return W4_ERR_ALIGN;
+    DeviceInfo d;
+    if (device_info(d) != W4_OK) return W4_ERR_CUDA;
+    cudaStream_t st = as_stream(stream);
+    const long long total = (long long)K * N;
+    if (cudaMemsetAsync(workspace, 0, 8, st) != cudaSuccess) return W4_ERR_CUDA;
+    if (d_status && cudaMemsetAsync(d_status, 0, sizeof(int), st) != cudaSuccess) return W4_ERR_CUDA;
+    const long long n8 = total / 8;
+    const int g1 = (int)std::min<long long>((n8 + 255) / 256, (long long)d.sms * 8);
+    nvfp4_absmax_kernel<<<g1, 256, 0, st>>>(reinterpret_cast<const uint4 *>(W), n8,
+                                             reinterpret_cast<unsigned *>(workspace));
+    const long long nb = total / 16;
+    const int g2 = (int)std::min<long long>((nb + 255) / 256, (long long)d.sms * 16);
+    nvfp4_encode_kernel<<<g2, 256, 0, st>>>(reinterpret_cast<const uint4 *>(W), nb,
+                                             reinterpret_cast<const unsigned *>(workspace),
+                                             reinterpret_cast<uint2 *>(codes), scales, global_scale, d_status);
+    return launch_status();
+}
+
+w4_status pack_rocmfp4(const void *W, int K, int N, int block, int fmt, const float *importance, uint8_t *blocks,
+                       int *d_status, void *stream) {
+    if (!W || !blocks || K < 32 || N < 1 || K % 32 || block != 32) return W4_ERR_ARG;
+    if (fmt != W4_FMT_ROCMFP4_DUAL && fmt != W4_FMT_ROCMFP4_FAST) return W4_ERR_ARG;
+    if (importance) return W4_ERR_UNSUPPORTED;
+    if (!aligned16(W) || !aligned16(blocks) || (reinterpret_cast<uintptr_t>(d_status) & 3)) return W4_ERR_ALIGN;
+    DeviceInfo d;
+    if (device_info(d) != W4_OK) return W4_ERR_CUDA;
+    cudaStream_t st = as_stream(stream);
+    if (d_status && cudaMemsetAsync(d_status, 0, sizeof(int), st) != cudaSuccess) return W4_ERR_CUDA;
+    const long long nblk = (long long)K * N / 32;
+    const int grid = (int)std::min<long long>((nblk + 7) / 8, (long long)d.sms * 16);
+    if (fmt == W4_FMT_ROCMFP4_DUAL)
+        rocm_pack_kernel<true><<<grid, 256, 0, st>>>(reinterpret_cast<const uint16_t *>(W), nblk, blocks, d_status);
+    else
+        rocm_pack_kernel<false><<<grid, 256, 0, st>>>(reinterpret_cast<const uint16_t *>(W), nblk, blocks, d_status);
+    return launch_status();
+}
+
+size_t w4a16_workspace_bytes(const w4_weights *w, int M) {
+    if (check_weights(w) != W4_OK || M < 1) return 0;
+    if (M <= 16) {
+        if (w->K % k_unit(w->fmt)) return 0;
+        GemvPlan p;
+        if (plan_gemv(w->fmt, w->K, w->N, M, false, p) != W4_OK) return 0;
+        GemvPlan q;
+        if (plan_gemv(w->fmt, w->K, w->N, M, true, q) != W4_OK) return p.ws_bytes;
+        return std::max(p.ws_bytes, q.ws_bytes);
+    }
+    return gemm_workspace_bytes(w, M);
+}
+
+w4_status w4a16_gemv_ex(const w4_weights *w, const void *x, int M, float *y, void *workspace,
+                        size_t workspace_bytes, unsigned flags, void *stream) {
+    w4_status s = check_weights(w);
+    if (s != W4_OK) return s;
+    if (!x || !y || M < 1 || M > 16 || (flags & ~W4_LAUNCH_PDL)) return W4_ERR_ARG;
+    if (!aligned16(x) || !aligned16(y) || (workspace && !aligned16(workspace))) return W4_ERR_ALIGN;
+    if (w->K % k_unit(w->fmt)) return W4_ERR_UNSUPPORTED;
+    const bool pdl = (flags & W4_LAUNCH_PDL) != 0;
+    GemvPlan p;
+    if ((s = plan_gemv(w->fmt, w->K, w->N, M, pdl, p)) != W4_OK) return s;
+    if (p.ws_bytes && (!workspace || workspace_bytes < p.ws_bytes)) return W4_ERR_WORKSPACE;
+    cudaStream_t st = as_stream(stream);
+    switch (w->fmt) {
+    case W4_FMT_NVFP4: return launch_gemv_fmt<W4_FMT_NVFP4>(w, x, M, y, workspace, p, pdl, st);
+    case W4_FMT_ROCMFP4_DUAL: return launch_gemv_fmt<W4_FMT_ROCMFP4_DUAL>(w, x, M, y, workspace, p, pdl, st);
+    case W4_FMT_ROCMFP4_FAST: return launch_gemv_fmt<W4_FMT_ROCMFP4_FAST>(w, x, M, y, workspace, p, pdl, st);
+    }
+    return W4_ERR_ARG;
+}
+
+w4_status w4a16_gemv(const w4_weights *w, const void *x, int M, float *y, void *workspace, size_t workspace_bytes,
+                     void *stream) {
+    return w4a16_gemv_ex(w, x, M, y, workspace, workspace_bytes, 0u, stream);
+}
+
+w4_status w4a16_gemm(const w4_weights *w, const void *x, int M, float *y_f32, void *y_bf16, void *workspace,
+                     size_t workspace_bytes, void *stream) {
+    w4_status s = check_weights(w);
+    if (s != W4_OK) return s;
+    if (!x || M < 1 || (!y_f32 && !y_bf16)) return W4_ERR_ARG;
+    if (!aligned16(x) || (y_f32 && !aligned16(y_f32)) || (y_bf16 && !aligned16(y_bf16))) return W4_ERR_ALIGN;
+    return gemm_launch(w, x, M, y_f32, y_bf16, workspace, workspace_bytes, as_stream(stream));
+}
+
+w4_status w4_encode_scalars(const float *v, size_t n, uint8_t *e4m3, uint8_t *e2m1, void *stream) {
+    if (!v || (!e4m3 && !e2m1)) return W4_ERR_ARG;
+    if (n == 0) return W4_OK;
+    DeviceInfo d;
+    if (device_info(d) != W4_OK) return W4_ERR_CUDA;
+    const int grid = (int)std::min<long long>(((long long)n + 255) / 256, (long long)d.sms * 16);
+    encode_scalars_kernel<<<grid, 256, 0, as_stream(stream)>>>(v, (long long)n, e4m3, e2m1);
+    return launch_status();
+}
+
+w4_status w4_device_error(int *out, int clear) {
+    if (!out) return W4_ERR_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return W4_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(out, g_device_error, sizeof(int)) != cudaSuccess) return W4_ERR_CUDA;
+    if (clear) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return W4_ERR_CUDA;
+    }
+    return W4_OK;
+}
+
+const char *w4_status_string(int status) {
+    switch (status) {
+    case W4_OK: return "W4_OK";
+    case W4_ERR_ARG: return "W4_ERR_ARG: invalid argument";
+    case W4_ERR_ALIGN: return "W4_ERR_ALIGN: pointer not 16-byte aligned";
+    case W4_ERR_UNSUPPORTED: return "W4_ERR_UNSUPPORTED: shape or option not supported";
+    case W4_ERR_CUDA: return "W4_ERR_CUDA: CUDA call or launch failed";
+    case W4_ERR_NONFINITE: return "W4_ERR_NONFINITE: NaN or Inf in the input matrix";
+    case W4_ERR_TIMEOUT: return "W4_ERR_TIMEOUT: device-side wait expired";
+    case W4_ERR_WORKSPACE: return "W4_ERR_WORKSPACE: workspace missing or too small";
+    }
+    return "unknown w4_status";
+}
+
+const char *w4_version(void) { return "w4a16 0.1.0 (sm_100a)"; }
+
+}  // extern "C"
