@@ -1,0 +1,83 @@
+"""CUDA tcgen05 GEMM vs the oracle's binary64 matmul.
+
+float32 output: |y - y_ref| <= 1e-3 * sum|x w_hat|.  BF16 output: the same
+bound plus half a BF16 unit in the last place of y_ref (the rounding of the
+result itself)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import w4a16_inputs as I
+import w4a16_matmul_pack_b200 as W4
+from gpu_util import assert_within_tolerance, np_of
+
+pytestmark = pytest.mark.gpu
+
+
+def packed(W):
+    c, s, g = O.pack_nvfp4(W)
+    pw = W4.PackedWeights(W4.FMT_NVFP4, W.shape[1], W.shape[0], torch.from_numpy(c).cuda(),
+                          torch.from_numpy(s).cuda(), torch.tensor([g], dtype=torch.float32).cuda())
+    return pw, (c, s, g)
+
+
+def half_ulp_bf16(v):
+    a = np.abs(v)
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -133)))
+    return np.where(a > 0, 2.0 ** (e - 8), 2.0 ** -134)
+
+
+def check(pw, cs, x, rows=None):
+    c, s, g = cs
+    y32, y16 = W4.w4a16_gemm(pw, x.cuda())
+    torch.cuda.synchronize()
+    y32, y16 = np_of(y32), np_of(y16.float())
+    N = pw.N
+    rows = np.arange(N) if rows is None else np.asarray(rows)
+    wh = np.concatenate([O.dequant_nvfp4(c, s, g, int(r), 1) for r in rows])
+    yr, ar = O.matmul(x, wh)
+    assert_within_tolerance(y32[:, rows], yr, ar)
+    err16 = np.abs(y16[:, rows] - yr)
+    bound16 = 1e-3 * ar + half_ulp_bf16(yr)
+    assert np.all(err16 <= bound16), float((err16 - bound16).max())
+
+
+def test_prefill_full_size_sampled_rows():
+    W, x = I.prefill()
+    pw, cs = packed(W)
+    rng = np.random.default_rng(0)
+    rows = np.unique(np.concatenate([np.arange(0, 130), np.arange(9600, 9728), rng.integers(0, 9728, 64)]))
+    check(pw, cs, x, rows)
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 128, 64), (300, 200, 128), (1, 77, 640), (16, 1000, 2560),
+                                   (513, 384, 1024), (2048, 256, 256)])
+def test_ragged_shapes(M, N, K):
+    W = I.matrix("student_t4", N, K, M + N + K, 0.02, 1e-3)
+    x = I.activations(M, K, 7, outlier_cols=min(16, K // 8))
+    pw, cs = packed(W)
+    check(pw, cs, x)
+
+
+def test_repeatable():
+    W = I.matrix("student_t4", 512, 1024, 3, 0.02, 1e-3)
+    x = I.activations(512, 1024, 4).cuda()
+    pw, _ = packed(W)
+    a = W4.w4a16_gemm(pw, x)[0].clone()
+    b = W4.w4a16_gemm(pw, x)[0]
+    assert torch.equal(a, b)
+    assert W4.w4_device_error(clear=True) == 0
+
+
+def test_unsupported_inputs():
+    W = I.matrix("normal", 64, 96, 1, 0.02)
+    pw, _ = packed(W)
+    with pytest.raises(W4.W4Error) as e:
+        W4.w4a16_gemm(pw, I.activations(4, 96, 1).cuda())
+    assert e.value.status == 3
+    b = O.pack_rocmfp4(I.matrix("laplace", 64, 128, 2, 0.015), O.FMT_DUAL)
+    pr = W4.PackedWeights(W4.FMT_ROCMFP4_DUAL, 128, 64, torch.from_numpy(b).cuda())
+    with pytest.raises(W4.W4Error) as e:
+        W4.w4a16_gemm(pr, I.activations(4, 128, 1).cuda())
+    assert e.value.status == 3

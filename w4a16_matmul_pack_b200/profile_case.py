@@ -1,0 +1,64 @@
+"""Run one operation of the library on one shape a few times (for profilers).
+
+    python -m w4a16_matmul_pack_b200.profile_case gemv --fmt nvfp4 --K 2560 --N 9728 --M 1 --reps 3
+    python -m w4a16_matmul_pack_b200.profile_case gemm --M 2048 --K 2560 --N 9728 --reps 2
+    python -m w4a16_matmul_pack_b200.profile_case pack --fmt dual --K 2560 --N 9728
+
+Inputs are the seeded synthetic matrices (Student-t weights, N(0,1) x; Laplace
+weights for ROCmFP4).  Exits non-zero on any library or CUDA error.
+"""
+from __future__ import annotations
+
+import argparse
+import os
+import sys
+
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import w4a16_inputs as I  # noqa: E402
+import w4a16_matmul_pack_b200 as W4  # noqa: E402
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("op", choices=["gemv", "gemm", "pack"])
+    ap.add_argument("--fmt", default="nvfp4", choices=["nvfp4", "dual", "fast"])
+    ap.add_argument("--M", type=int, default=1)
+    ap.add_argument("--K", type=int, default=2560)
+    ap.add_argument("--N", type=int, default=9728)
+    ap.add_argument("--reps", type=int, default=3)
+    a = ap.parse_args()
+    torch.cuda.set_device(0)
+    if a.fmt == "nvfp4":
+        W = I.matrix("student_t4", a.N, a.K, 7, 0.02, 1e-4, 20.0, device="cuda")
+    else:
+        W = I.matrix("laplace", a.N, a.K, 7, 0.015, 1e-4, 20.0, device="cuda")
+    x = I.activations(a.M, a.K, 8, device="cuda")
+    if a.op == "pack":
+        for _ in range(a.reps):
+            if a.fmt == "nvfp4":
+                W4.pack_nvfp4(W)
+            else:
+                W4.pack_rocmfp4(W, a.fmt)
+    else:
+        pw = W4.pack_nvfp4(W) if a.fmt == "nvfp4" else W4.pack_rocmfp4(W, a.fmt)
+        torch.cuda.synchronize()
+        for _ in range(a.reps):
+            if a.op == "gemv":
+                W4.w4a16_gemv(pw, x)
+            else:
+                W4.w4a16_gemm(pw, x)
+    torch.cuda.synchronize()
+    err = W4.w4_device_error(clear=True)
+    if err:
+        print(f"device error word: {err}")
+        sys.exit(1)
+    print("ok")
+
+
+if __name__ == "__main__":
+    main()
