@@ -180,6 +180,28 @@ w4_status w4a16_gemm(const w4_weights *w, const void *x, int M, float *y_f32,
 /* Scratch bytes w4a16_gemv / w4a16_gemm need for this shape (0 if none). */
 size_t w4a16_workspace_bytes(const w4_weights *w, int M);
 
+/*
+ * w4a16_gemv_noalloc -- w4a16_gemv for callers that cannot allocate device
+ * memory (for example a plugin whose host framework owns every device
+ * allocation, or an embedded runtime with a fixed memory budget): the same
+ * computation, but the split-K scratch comes from a device array built into
+ * the library instead of a caller-provided workspace.  The pages have no
+ * counterpart to this entry point; it only changes where scratch lives.
+ *   w, x, M, y, stream  as for w4a16_gemv (x, y and the packed weights are still
+ *                       caller-owned device memory).
+ *   Returns W4_ERR_WORKSPACE, before launching anything, when the shape needs
+ *   more than W4_NOALLOC_SCRATCH_BYTES of scratch (w4a16_workspace_bytes).
+ * The array (W4_NOALLOC_SCRATCH_BYTES) is held by every GPU that loads the
+ * library until the process exits.  The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress, with that device current) and
+ * caches it; make that first call before any stream capture.  All calls on a
+ * device share the array: calls whose work overlaps on the GPU race and must
+ * be serialised by the caller.  Every scratch value a call reads is written
+ * earlier in the same call, so no clearing is needed between calls.
+ */
+#define W4_NOALLOC_SCRATCH_BYTES (8u << 20)
+w4_status w4a16_gemv_noalloc(const w4_weights *w, const void *x, int M, float *y, void *stream);
+
 /* ------------------------------------------------------------- utilities --- */
 
 /*

@@ -12,6 +12,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 SRC_DIR = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libw4a16.so")
 MAIN = os.path.join(SRC_DIR, "w4a16.cu")
+UNITS = [MAIN, os.path.join(SRC_DIR, "noalloc.cu")]
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-lineinfo",
@@ -41,7 +42,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB
     nvcc = os.environ.get("NVCC", "nvcc")
     tmp = LIB + f".{os.getpid()}.tmp"
-    cmd = [nvcc, *NVCC_FLAGS, MAIN, "-o", tmp]
+    cmd = [nvcc, *NVCC_FLAGS, *UNITS, "-o", tmp]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), flush=True)
