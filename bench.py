@@ -127,13 +127,20 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(world, v: float) -> float:
+def max_over_ranks(world, v: float, device="cuda") -> float:
+    """The largest of each rank's v (device timings are combined as the slowest rank's)."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_value(world: int, step_bytes: float, ms_total: float, steps: int) -> float:
+    """Whole-job GB/s of `world` replicas that each process step_bytes per step,
+    over the slowest rank's time for `steps` steps."""
+    return world * step_bytes / (ms_total / steps) / 1e6
 
 
 # ------------------------------------------------------------------ workloads (GPU)
@@ -187,6 +194,53 @@ def per_shape(W4, mats, reps=40):
         g = capture(run)
         ms = time_graphs([g], reps, 5) / ROTATE
         out[f"{m['K']}x{m['N']}"] = {"us": round(ms * 1e3, 3), "GB/s": round(m["bytes"] / ms / 1e6, 1)}
+    return out
+
+
+def sweep_m_bench(W4, I, mats, pk):
+    """The decode sweep at M = 4 and 16 (same packed copies, PDL graph per step)."""
+    out = {}
+    for M in (4, 16):
+        xs = [I.sweep_x(M, m["K"], idx, device="cuda") for idx, m in enumerate(mats)]
+        ys = [torch.empty(M, m["N"], dtype=torch.float32, device="cuda") for m in mats]
+        ws = torch.empty(max(W4.w4a16_workspace_bytes(m["copies"][0], M) for m in mats) + 16,
+                         dtype=torch.uint8, device="cuda")
+
+        def step(r):
+            def run():
+                for m, x, y in zip(mats, xs, ys):
+                    W4.w4a16_gemv(m["copies"][r], x, out=y, workspace=ws, flags=W4.LAUNCH_PDL)
+            return run
+        graphs = [capture(step(r)) for r in range(ROTATE)]
+        ms = time_graphs(graphs, 60, 6)
+        nb = sum(m["bytes"] for m in mats)
+        out[f"M{M}"] = {"GB/s": round(nb / ms / 1e6, 1), "frac": round(nb / ms / 1e6 / pk["hbm_gbs"], 4),
+                        "us_per_step": round(ms * 1e3, 2)}
+        del graphs
+    return out
+
+
+def rocm_gemv_bench(W4, I, pk):
+    """ROCmFP4 GEMV on the 2560x9728 Laplace matrix, Dual and FAST, M = 1 and 8."""
+    out = {}
+    L = I.rocm_weights(device="cuda")
+    for fmt in ("dual", "fast"):
+        base = W4.pack_rocmfp4(L, fmt)
+        copies = [base] + [W4.PackedWeights(base.fmt, base.K, base.N, base.codes.clone()) for _ in range(ROTATE - 1)]
+        nb = base.nbytes
+        for M in (1, 8):
+            x = I.rocm_x(M, device="cuda")
+            y = torch.empty(M, base.N, dtype=torch.float32, device="cuda")
+            ws = torch.empty(W4.w4a16_workspace_bytes(base, M) + 16, dtype=torch.uint8, device="cuda")
+
+            def run():
+                for c in copies:
+                    W4.w4a16_gemv(c, x, out=y, workspace=ws)
+            g = capture(run)
+            ms = time_graphs([g], 20, 3) / ROTATE
+            out[f"{fmt}_M{M}"] = {"us": round(ms * 1e3, 2), "GB/s": round(nb / ms / 1e6, 1),
+                                  "frac": round(nb / ms / 1e6 / pk["hbm_gbs"], 4), "bytes": nb}
+        del copies
     return out
 
 
@@ -339,7 +393,7 @@ def run_ours(args, world, rank, local):
     ck = clocks.stop()
     ms_total = max_over_ranks(world, a.elapsed_time(b))
     ms_step = ms_total / args.steps
-    value = world * step_bytes / ms_step / 1e6  # GB/s over all ranks
+    value = replica_value(world, step_bytes, ms_total, args.steps)  # GB/s over all ranks
     launches = 5 * args.steps
 
     # per-launch duration of the dominant kernel (the M=1 GEMV; every launch in the step)
@@ -382,11 +436,14 @@ def run_ours(args, world, rank, local):
     extras = {}
     if not args.no_extras:
         extras["per_shape_isolated"] = per_shape(W4, mats)
+        extras["sweep_skinny"] = sweep_m_bench(W4, I, mats, pk)
         del graphs, mats
         torch.cuda.empty_cache()
         extras["gemm"] = gemm_bench(W4, I, pk)
         torch.cuda.empty_cache()
         extras["packers"] = pack_bench(W4, I)
+        torch.cuda.empty_cache()
+        extras["rocm_gemv"] = rocm_gemv_bench(W4, I, pk)
         torch.cuda.empty_cache()
         extras["stream"] = stream_bench(W4, I)
     err = W4.w4_device_error(clear=True)

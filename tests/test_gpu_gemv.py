@@ -139,3 +139,23 @@ def test_save_reload_in_fresh_process(tmp_path):
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     subprocess.run([sys.executable, "-c", code], check=True, cwd=root,
                    env={**os.environ, "PYTHONPATH": root})
+
+
+@pytest.mark.parametrize("case", ["scaled_up", "scaled_down", "wide_range", "subnormal"])
+@pytest.mark.parametrize("M", [1, 3, 12])
+def test_activation_range_cases(case, M):
+    """x far from 1 (the tensor-core path rescales x by a power of two) and x whose
+    dynamic range no single power of two maps into f16 (the binary32 path)."""
+    K, N = 2560, 512
+    pw, wh = nvfp4_packed(I.sweep_weights(K, N, 1)[:N].contiguous())
+    x = I.activations(M, K, 17 + M).double()
+    if case == "scaled_up":
+        x *= 2.0 ** 100
+    elif case == "scaled_down":
+        x *= 2.0 ** -100
+    elif case == "wide_range":
+        x[:, :8] *= 2.0 ** 40
+        x[:, 8:16] *= 2.0 ** -40
+    else:
+        x[:, ::3] = 2.0 ** -130
+    run_and_check(pw, wh, I.bf16_rne(x))

@@ -25,8 +25,6 @@
 // of the next.  Every mbarrier wait is bounded (common.cuh: mbar_wait).
 #pragma once
 
-#include <cuda.h>
-
 #include "common.cuh"
 
 namespace w4 {
@@ -44,6 +42,9 @@ constexpr int kEpiThreads = 128;
 constexpr uint32_t X_STAGE_BYTES = BN * BK * 2;   // 32 KB
 constexpr uint32_t A_STAGE_BYTES = BM * BK * 2;   // 16 KB
 constexpr uint32_t TMEM_COLS = 512;               // two 256-column fp32 accumulators
+constexpr int WK = 256;                           // k per packed-weight stage (4 k-steps)
+constexpr int WSTAGES = 2;
+constexpr uint32_t W_STAGE_BYTES = BM * WK / 2;   // 16 KB of codes (128 rows x 128 bytes)
 
 // Instruction descriptor, kind::f16: D = F32 (bit 4), A = BF16 (bits 7-9),
 // B = BF16 (bits 10-12), both K-major, N >> 3 at bit 17, M >> 4 at bit 24.
@@ -53,6 +54,8 @@ constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >
 struct SharedStorage {
     uint8_t x[STAGES][X_STAGE_BYTES];   // 1024-byte aligned (swizzle atoms)
     uint8_t a[STAGES][A_STAGE_BYTES];
+    uint8_t w[WSTAGES][W_STAGE_BYTES];  // packed codes, 128-byte swizzle
+    uint64_t w_full[WSTAGES], w_empty[WSTAGES];
     uint64_t x_full[STAGES], x_empty[STAGES];
     uint64_t a_full[STAGES], a_empty[STAGES];
     uint64_t acc_full[2], acc_empty[2];
@@ -85,14 +88,6 @@ __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                  ::"r"(smem_addr(bar)) : "memory");
-}
-
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int c0, int c1, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
-        "[%0], [%1, {%2, %3}], [%4];"
-        ::"r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_addr(bar))
-        : "memory");
 }
 
 #define W4_TMEM_LD32(taddr, v)                                                                              \
@@ -131,7 +126,8 @@ struct Params {
     int tiles_m, tiles_n;
 };
 
-__global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
+__global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ CUtensorMap xmap,
+                                                            const __grid_constant__ CUtensorMap cmap, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     SharedStorage &sh = *reinterpret_cast<SharedStorage *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -145,12 +141,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         for (int i = 0; i < STAGES; i++) {
             mbar_init(&sh.x_full[i], 1);
             mbar_init(&sh.x_empty[i], 1);
-            mbar_init(&sh.a_full[i], kDequantThreads);
+            mbar_init(&sh.a_full[i], kDequantThreads / 32);   // one arrival per dequant warp
             mbar_init(&sh.a_empty[i], 1);
+        }
+        for (int i = 0; i < WSTAGES; i++) {
+            mbar_init(&sh.w_full[i], 1);
+            mbar_init(&sh.w_empty[i], kDequantThreads / 32);
         }
         for (int i = 0; i < 2; i++) {
             mbar_init(&sh.acc_full[i], 1);
-            mbar_init(&sh.acc_empty[i], kEpiThreads);
+            mbar_init(&sh.acc_empty[i], kEpiThreads / 32);
         }
         fence_mbar_init();
     }
@@ -167,10 +167,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     if (warp == 0) {
         // ---------------------------- x producer (TMA) ----------------------------
         if (lane == 0) {
-            int it = 0;
+            int it = 0, wit = 0;
             for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
                 const int m0 = (t % p.tiles_m) * BN;
+                const int n0 = (t / p.tiles_m) * BM;
                 for (int kt = 0; kt < KT; kt++, it++) {
+                    if (kt % (WK / BK) == 0) {   // packed codes of the next 256 k
+                        const int ws = wit % WSTAGES;
+                        if (wit >= WSTAGES) mbar_wait(&sh.w_empty[ws], ((wit / WSTAGES) - 1) & 1, abort);
+                        if (*abort) break;
+                        mbar_arrive_expect_tx(&sh.w_full[ws], W_STAGE_BYTES);
+                        tma_load_2d(sh.w[ws], &cmap, kt * (BK / 2), n0, &sh.w_full[ws]);
+                        wit++;
+                    }
                     const int s = it % STAGES;
                     if (it >= STAGES) mbar_wait(&sh.x_empty[s], ((it / STAGES) - 1) & 1, abort);
                     if (*abort) break;
@@ -234,46 +243,60 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                 }
             }
             tc_fence_before();
-            mbar_arrive(&sh.acc_empty[b]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.acc_empty[b]);
         }
     } else {
         // ------------------------------- dequantise -------------------------------
+        // thread (row r, half h): 32 codes of row r per k-step from the swizzled
+        // codes stage (conflict-free: 8 consecutive rows read 8 distinct 16-byte
+        // chunks), 2 scales from a register ring filled one codes stage ahead.
         const int dt = threadIdx.x - 6 * 32;    // 0..255
         const int r = dt & (BM - 1), h = dt >> 7;
-        int it = 0;
+        constexpr int KQ = WK / BK;             // k-steps per codes stage
+        int it = 0, wit = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
             const int n = (t / p.tiles_m) * BM + r;
             const bool valid = n < p.N;
-            const uint8_t *crow = p.codes + (size_t)(valid ? n : 0) * (p.K / 2) + h * 16;
-            const uint8_t *srow = p.scales + (size_t)(valid ? n : 0) * (p.K / 16) + h * 2;
-            uint4 cw = make_uint4(0, 0, 0, 0);
-            uint32_t sw = 0;
-            if (valid) {
-                cw = __ldg(reinterpret_cast<const uint4 *>(crow));
-                sw = __ldg(reinterpret_cast<const uint16_t *>(srow));
-            }
-            for (int kt = 0; kt < KT; kt++, it++) {
-                const int s = it % STAGES;
-                uint4 cn = make_uint4(0, 0, 0, 0);
-                uint32_t sn = 0;
-                if (valid && kt + 1 < KT) {   // prefetch the next stage's codes
-                    cn = __ldg(reinterpret_cast<const uint4 *>(crow + (kt + 1) * (BK / 2)));
-                    sn = __ldg(reinterpret_cast<const uint16_t *>(srow + (kt + 1) * (BK / 16)));
-                }
-                if (it >= STAGES) mbar_wait(&sh.a_empty[s], ((it / STAGES) - 1) & 1, abort);
-                const float s0 = e4m3_to_f32(sw & 0xFFu), s1 = e4m3_to_f32(sw >> 8);
-                uint8_t *arow = sh.a[s] + r * 128;
-                const uint32_t cws[4] = {cw.x, cw.y, cw.z, cw.w};
+            const uint8_t *srow = p.scales + (size_t)(valid ? n : 0) * (p.K / 16);
+            uint32_t sc[KQ], sn[KQ];
 #pragma unroll
-                for (int cc = 0; cc < 4; cc++) {
-                    const uint4 o = valid ? dequant8(cws[cc], cc < 2 ? s0 : s1) : make_uint4(0, 0, 0, 0);
-                    const int chunk = (h * 4 + cc) ^ (r & 7);
-                    *reinterpret_cast<uint4 *>(arow + chunk * 16) = o;
+            for (int q = 0; q < KQ; q++) sc[q] = (valid && q < KT) ? __ldg(reinterpret_cast<const uint32_t *>(srow) + q) : 0u;
+            for (int kw = 0; kw < KT; kw += KQ, wit++) {
+                const int ws = wit % WSTAGES;
+#pragma unroll
+                for (int q = 0; q < KQ; q++)   // prefetch the next stage's scales
+                    sn[q] = (valid && kw + KQ + q < KT) ? __ldg(reinterpret_cast<const uint32_t *>(srow) + kw + KQ + q) : 0u;
+                mbar_wait(&sh.w_full[ws], (wit / WSTAGES) & 1, abort);
+                const uint8_t *wrow = sh.w[ws] + r * 128;
+#pragma unroll
+                for (int q = 0; q < KQ; q++) {
+                    if (kw + q < KT) {
+                        const int s = it % STAGES;
+                        if (it >= STAGES) mbar_wait(&sh.a_empty[s], ((it / STAGES) - 1) & 1, abort);
+                        const uint4 cw = *reinterpret_cast<const uint4 *>(wrow + (((q * 2 + h) ^ (r & 7)) * 16));
+                        const uint32_t sw = sc[q] >> (16 * h);
+                        const float s0 = e4m3_to_f32(sw & 0xFFu), s1 = e4m3_to_f32((sw >> 8) & 0xFFu);
+                        uint8_t *arow = sh.a[s] + r * 128;
+                        const uint32_t cws[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+                        for (int cc = 0; cc < 4; cc++) {
+                            const uint4 o = valid ? dequant8(cws[cc], cc < 2 ? s0 : s1) : make_uint4(0, 0, 0, 0);
+                            const int chunk = (h * 4 + cc) ^ (r & 7);
+                            *reinterpret_cast<uint4 *>(arow + chunk * 16) = o;
+                        }
+                        // each thread makes its stores visible to the tensor core's
+                        // (async) proxy; the warp then arrives once
+                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&sh.a_full[s]);
+                        it++;
+                    }
                 }
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                mbar_arrive(&sh.a_full[s]);
-                cw = cn;
-                sw = sn;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sh.w_empty[ws]);
+#pragma unroll
+                for (int q = 0; q < KQ; q++) sc[q] = sn[q];
             }
         }
     }
@@ -289,23 +312,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
 }  // namespace gemm
 
 // ---------------------------------------------------------------- host side --
-
-typedef CUresult (*PFN_encodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                    const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
-                                    CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
-                                    CUtensorMapFloatOOBfill);
-
-inline PFN_encodeTiled get_encode_tiled() {
-    static PFN_encodeTiled fn = nullptr;
-    if (!fn) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_encodeTiled>(p);
-    }
-    return fn;
-}
 
 inline size_t gemm_workspace_bytes(const w4_weights *, int) { return 0; }
 
@@ -325,6 +331,14 @@ inline w4_status gemm_launch(const w4_weights *w, const void *x, int M, float *y
     const cuuint32_t box[2] = {BK, BN};
     const cuuint32_t estr[2] = {1, 1};
     if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return W4_ERR_CUDA;
+    CUtensorMap cmap;
+    const cuuint64_t cdims[2] = {(cuuint64_t)K / 2, (cuuint64_t)N};
+    const cuuint64_t cstrides[1] = {(cuuint64_t)K / 2};
+    const cuuint32_t cbox[2] = {WK / 2, BM};
+    if (enc(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(w->codes), cdims, cstrides, cbox, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return W4_ERR_CUDA;
@@ -350,7 +364,7 @@ inline w4_status gemm_launch(const w4_weights *w, const void *x, int M, float *y
     p.tiles_m = (M + BN - 1) / BN;
     p.tiles_n = (N + BM - 1) / BM;
     const int ntiles = p.tiles_m * p.tiles_n;
-    gemm_kernel<<<std::min(ntiles, sms), kThreads, smem, st>>>(map, p);
+    gemm_kernel<<<std::min(ntiles, sms), kThreads, smem, st>>>(map, cmap, p);
     return cudaGetLastError() == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
 

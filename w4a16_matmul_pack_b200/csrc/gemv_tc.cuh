@@ -1,0 +1,412 @@
+// gemv_tc.cuh -- NVFP4 decode GEMV (M = 1..16) with the products on the tensor
+// cores (sm_100a, mma.sync.m16n8k16, f16 inputs, binary32 accumulation).
+//
+// y[m][n] = g * sum_k x[m][k] * e2m1[n][k] * scale[n][k/16]   ("EdgeRock-4B-NVFP4"
+// card, intro; the fused W4A16 decode kernel of the "Nanbeige4.2-3B-NVFP4A16"
+// card, Serving).  The kernel is bound by HBM: every packed byte is read once.
+//
+// Decode on the CUDA cores would cost ~6 lane instructions per weight, above the
+// ~4 the SMs can issue per weight at 75% of HBM bandwidth.  Here a lane decodes
+// two E2M1 codes with one cvt (E2M1 -> f16x2, exact) and applies the block scale
+// with one HMUL2 (e2m1 * E4M3 has at most 6 significant bits and lies in
+// [2^-10, 2688]: exact in f16); the MMA does the multiply-add.  x is converted
+// once per CTA to f16 as x * 2^-sigma (sigma from the largest |x|), exact when
+// every x fits f16's range; a CTA that finds an x it cannot convert exactly runs
+// a binary32 CUDA-core loop on the same staged tiles instead.
+//
+// Data movement: bulk copies only reach full HBM bandwidth when each copy is
+// large (>= 16 KB; small copies are limited by a per-copy cost), so a stage is
+// one 2-D TMA box of codes (16 rows x KP/2 bytes, the codes viewed as 8-byte
+// elements) and one box of scales (16 rows x KP/16 bytes), in an NS-deep
+// mbarrier ring filled by one producer thread.  Rows are contiguous in shared
+// memory.
+//
+// MMA operand mapping.  In an m16n8k16 a lane (g = lane/4, t = lane%4) holds A
+// rows g and g+8 at two k-pairs and B column g at the same k-pairs.  Any
+// permutation of k applied to both operands leaves the product unchanged, so
+// within a 128-k super-chunk lane t owns k = 32t..32t+31: one 16-byte load per
+// row gives the codes of 8 MMAs (two scale groups: 2t and 2t+1), and x is
+// stored permuted (the 8 x of MMAs 2j, 2j+1 of lane t at offset 32j + 8t) so
+// that the B loads of the four lanes of a row are one contiguous 64-byte run.
+// Consumer warp w takes a contiguous 1/8 of each stage's super-chunks; the MMA
+// accumulators persist over the k-pieces of a row tile and the 8 warps' partial
+// sums are added in a fixed order at its end.
+#pragma once
+
+#include "gemv.cuh"
+
+namespace w4 {
+
+struct GemvTcArgs {
+    const uint8_t *codes;
+    const uint8_t *scales;
+    const float *gscale;
+    const uint16_t *x;   // [M][K] bf16
+    float *y;            // [M][N]
+    float *partial;      // [S][M][N] when gridDim.y > 1
+    int K, N;
+    int kc;              // slice length (split-K over blockIdx.y)
+    int KP;              // k per stage (multiple of 256, <= 4096)
+    int NS;              // stages
+    int xstride;         // halves per x row in shared memory (kc + 32)
+    int tile_bytes;      // bytes of one stage: 16 * (KP/2 + KP/16), rounded up
+    int rows_mode;       // 0: balanced rows per CTA; 1: whole 16-row tiles per CTA
+    int tiles_per_cta;   // rows_mode 1
+    int box_min_rows;    // a partial tile with at least this many rows uses the TMA box
+    int red_tiles;       // tiles whose partial sums fit the reduction buffer at once (>= ntiles:
+                         // one barrier per CTA; else 2 and a barrier per tile)
+    int pdl;             // launched with programmatic dependent launch: prefetch weights before x
+};
+
+// v * 2^e for |e| <= 252 as two exact multiplies (each factor a normal power of two).
+__device__ __forceinline__ float mul_pow2(float v, int e) {
+    const int h = e / 2, h2 = e - h;
+    return (v * __int_as_float((127 + h) << 23)) * __int_as_float((127 + h2) << 23);
+}
+
+constexpr int kTcRows = 16;                    // rows per tile (one MMA M)
+constexpr int kTcWarps = 8;                    // consumer warps, each a contiguous share of a tile's k
+constexpr int kTcParts = kTcWarps;
+constexpr int kTcThreads = (kTcWarps + 1) * 32; // + one producer warp
+constexpr int kTcFbRows = kTcRows / kTcWarps;  // rows per warp on the binary32 path
+
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Two E4M3 bytes (low 16 bits) -> f16x2 (low byte -> low half).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
+    uint32_t r;
+    const uint16_t b = (uint16_t)(two & 0xFFFFu);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(b));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
+    const __half2 r = __hmul2(*reinterpret_cast<const __half2 *>(&a), *reinterpret_cast<const __half2 *>(&b));
+    return *reinterpret_cast<const uint32_t *>(&r);
+}
+
+// 16 code bytes of one row (32 k) times their two group scales -> 16 f16x2
+// values (h[i] = elements 2i, 2i+1 of the lane's 32 k).
+__device__ __forceinline__ void decode_row32(uint4 c, uint32_t s2, uint32_t (&h)[16]) {
+    const uint32_t sc = e4m3x2_to_f16x2(s2);        // (s_lo, s_hi)
+    const uint32_t slo = __byte_perm(sc, 0, 0x1010); // (s_lo, s_lo)
+    const uint32_t shi = __byte_perm(sc, 0, 0x3232); // (s_hi, s_hi)
+    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+    for (int i = 0; i < 16; i++) h[i] = hmul2_u32(e2m1x2_to_f16x2(w[i >> 2] >> (8 * (i & 3))), i < 8 ? slo : shi);
+}
+
+// Sum a tile's parts in a fixed order and store (per-tile reduction mode).
+__device__ __forceinline__ void reduce_tile(const GemvTcArgs &a, const float *rb, long long rt, int rows, int nparts,
+                                            float gs, int yexp, int slice, int M) {
+    for (int i = threadIdx.x; i < rows * M; i += kTcWarps * 32) {
+        const int row = i / M, m = i % M;
+        float s = 0.0f;
+        for (int q = 0; q < nparts; q++) s += rb[(q * kTcRows + row) * M + m];
+        const long long n = rt + row;
+        if (gridDim.y == 1)
+            a.y[(size_t)m * a.N + n] = gs * mul_pow2(s, yexp);
+        else
+            a.partial[((size_t)slice * M + m) * a.N + n] = mul_pow2(s, yexp);
+    }
+}
+
+template <int M>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    gemv_nvfp4_tc_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant__ CUtensorMap smap,
+                         const GemvTcArgs a) {
+    constexpr int NT = (M + 7) / 8;   // n-tiles of 8 tokens
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int K = a.K, N = a.N, kc = a.kc, KP = a.KP, NS = a.NS, XS = a.xstride;
+    const int slice = blockIdx.y, k0 = slice * kc, kcs = min(kc, K - k0);
+    const int npieces = (kcs + KP - 1) / KP;
+    const int CS = KP / 2, SS = KP / 16;   // row strides of a stage (bytes)
+
+    uint16_t *xs = reinterpret_cast<uint16_t *>(smem);                              // [M][XS]
+    uint8_t *stages = smem + (((size_t)M * XS * 2 + 127) & ~(size_t)127);          // NS x tile_bytes
+    float *red = reinterpret_cast<float *>(stages + (size_t)NS * a.tile_bytes);    // [red_tiles][P][16][M]
+    uint64_t *full = reinterpret_cast<uint64_t *>(red + (size_t)a.red_tiles * kTcParts * kTcRows * M);
+    uint64_t *empty = full + NS;
+    uint64_t *xfull = empty + NS;
+    int *flags = reinterpret_cast<int *>(xfull + 1);   // [0] abort, [1] inexact x, [2..] per-warp max
+    volatile int *abort = flags;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    long long r0, r1;
+    if (a.rows_mode == 0) {
+        r0 = (long long)blockIdx.x * N / gridDim.x;
+        r1 = (long long)(blockIdx.x + 1) * N / gridDim.x;
+    } else {
+        r0 = (long long)blockIdx.x * a.tiles_per_cta * kTcRows;
+        r1 = min((long long)N, r0 + (long long)a.tiles_per_cta * kTcRows);
+    }
+    const int ntiles = (int)((r1 - r0 + kTcRows - 1) / kTcRows);
+    const int nstages = ntiles * npieces;
+
+    if (threadIdx.x == 0) {
+        flags[0] = 0;
+        flags[1] = 0;
+        for (int i = 0; i < NS; i++) {
+            mbar_init(full + i, 1);
+            mbar_init(empty + i, kTcWarps);
+        }
+        mbar_init(xfull, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    pdl_allow_dependents();
+    const float gs = __ldg(a.gscale);   // weights do not depend on earlier kernels
+
+    if (warp == kTcWarps) {
+        // ------------------------------ producer ------------------------------
+        if (lane == 0) {
+            const uint64_t pol = policy_evict_first();
+            // x depends on the previous kernel: copy it after the dependency wait.  Under
+            // programmatic launch the first NS weight stages go out before that wait.
+            const int before = a.pdl ? min(NS, nstages) : 0;
+            for (int t = 0; t < nstages + 1; t++) {
+                if (t == before) {
+                    pdl_wait_prior_grid();
+                    mbar_arrive_expect_tx(xfull, (uint32_t)(M * kcs * 2));
+                    for (int m = 0; m < M; m++)
+                        bulk_g2s(xs + (size_t)m * XS, a.x + (size_t)m * K + k0, (uint32_t)(kcs * 2), xfull, pol);
+                    continue;
+                }
+                const int tt = t > before ? t - 1 : t;   // weight stage index
+                const int st = tt % NS;
+                if (tt >= NS && !mbar_wait(empty + st, ((tt / NS) - 1) & 1, abort)) break;
+                const long long rt = r0 + (long long)(tt / npieces) * kTcRows;
+                const int rows = (int)min((long long)kTcRows, r1 - rt);
+                const int kpos = k0 + (tt % npieces) * KP;
+                const int kps = min(KP, k0 + kcs - kpos);
+                uint8_t *dst = stages + (size_t)st * a.tile_bytes;
+                uint8_t *dsts = dst + kTcRows * CS;
+                if (rows == kTcRows || rows >= a.box_min_rows) {
+                    // two boxes of 16 rows x KP (k beyond K and rows beyond N are zero-filled)
+                    mbar_arrive_expect_tx(full + st, (uint32_t)(kTcRows * (CS + SS)));
+                    tma_load_2d(dst, &cmap, kpos / 16, (int)rt, full + st);
+                    tma_load_2d(dsts, &smap, kpos / 16, (int)rt, full + st);
+                } else {
+                    // a short tail: row-piece copies of exactly the bytes needed
+                    mbar_arrive_expect_tx(full + st, (uint32_t)(rows * (kps / 2 + kps / 16)));
+                    for (int i = 0; i < rows; i++) {
+                        bulk_g2s(dst + i * CS, a.codes + (rt + i) * (K / 2) + kpos / 2, (uint32_t)(kps / 2),
+                                 full + st, pol);
+                        bulk_g2s(dsts + i * SS, a.scales + (rt + i) * (K / 16) + kpos / 16, (uint32_t)(kps / 16),
+                                 full + st, pol);
+                    }
+                }
+            }
+        }
+        return;
+    }
+
+    // -------------------------------- consumers --------------------------------
+    pdl_wait_prior_grid();   // y may be read by the previous kernel
+    mbar_wait(xfull, 0, abort);
+    // largest |x| of the slice
+    uint32_t mx = 0;
+    {
+        const int nvec = kcs / 8;
+        for (int i = threadIdx.x; i < M * nvec; i += kTcWarps * 32) {
+            const int m = i / nvec, v = i % nvec;
+            const uint4 val = *reinterpret_cast<const uint4 *>(xs + (size_t)m * XS + v * 8);
+            const uint32_t w4v[4] = {val.x, val.y, val.z, val.w};
+#pragma unroll
+            for (int j = 0; j < 4; j++) mx = max(mx, max(w4v[j] & 0x7FFFu, (w4v[j] >> 16) & 0x7FFFu));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+    if (lane == 0) flags[2 + warp] = (int)mx;
+    named_barrier_sync(1, kTcWarps * 32);
+    for (int i = 0; i < kTcWarps; i++) mx = max(mx, (uint32_t)flags[2 + i]);
+    // x' = x * 2^-sigma puts the largest |x| in [2^14, 2^15)
+    const int emax = (int)((mx >> 7) & 0xFFu);
+    const int sigma = (mx == 0) ? 0 : max(emax, 1) - 127 - 14;
+    // Convert in place to f16 and permute each 128-k super-chunk: the 8 values
+    // k = 32t + 8j .. +7 go to offset 32j + 8t.  A warp owns whole super-chunks
+    // (lane l converts vector l % 16 of super-chunk 2i + l / 16), so __syncwarp
+    // orders its loads before its stores.  Exactness: scale back and compare.
+    {
+        const int nsc = kcs / 128, total = M * nsc;
+        bool bad = mx >= 0x7F80u;   // NaN / Inf: binary32 path
+        for (int base = 2 * warp; base < total; base += 2 * kTcWarps) {
+            const int sc = base + (lane >> 4), q = lane & 15;
+            uint4 out = make_uint4(0, 0, 0, 0);
+            uint16_t *row = nullptr;
+            if (sc < total) {
+                row = xs + (size_t)(sc / nsc) * XS + (sc % nsc) * 128;
+                const uint4 val = *reinterpret_cast<const uint4 *>(row + q * 8);
+                const uint32_t in[4] = {val.x, val.y, val.z, val.w};
+                uint32_t o[4];
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    const float x0 = bf16_lo(in[j]), x1 = bf16_hi(in[j]);
+                    const __half2 h = __floats2half2_rn(mul_pow2(x0, -sigma), mul_pow2(x1, -sigma));
+                    const float2 back = __half22float2(h);
+                    bad |= (mul_pow2(back.x, sigma) != x0) | (mul_pow2(back.y, sigma) != x1);
+                    o[j] = *reinterpret_cast<const uint32_t *>(&h);
+                }
+                out = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+            __syncwarp();
+            if (sc < total) *reinterpret_cast<uint4 *>(row + ((q & 3) * 4 + (q >> 2)) * 8) = out;
+            __syncwarp();
+        }
+        if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) atomicOr(&flags[1], 1);
+    }
+    named_barrier_sync(1, kTcWarps * 32);
+    const bool fast = flags[1] == 0;
+    if (!fast) {
+        // an x could not be converted exactly: restage the bf16 values in natural order
+        const int nvec = kcs / 8;
+        for (int i = threadIdx.x; i < M * nvec; i += kTcWarps * 32) {
+            const int m = i / nvec, v = i % nvec;
+            *reinterpret_cast<uint4 *>(xs + (size_t)m * XS + v * 8) =
+                __ldg(reinterpret_cast<const uint4 *>(a.x + (size_t)m * K + k0) + v);
+        }
+        named_barrier_sync(1, kTcWarps * 32);
+    }
+    const int yexp = fast ? sigma : 0;   // undo the x scaling
+
+    const int g = lane >> 2, t4 = lane & 3;
+    int st_idx = 0;
+    for (int tile = 0; tile < ntiles; tile++) {
+        const long long rt = r0 + (long long)tile * kTcRows;
+        const int rows = (int)min((long long)kTcRows, r1 - rt);
+        float acc[NT][8][4];   // one accumulator per MMA of a super-chunk: no MMA waits on another
+        float facc[kTcFbRows][M];
+#pragma unroll
+        for (int n = 0; n < NT; n++)
+#pragma unroll
+            for (int q = 0; q < 8; q++)
+#pragma unroll
+                for (int i = 0; i < 4; i++) acc[n][q][i] = 0.0f;
+#pragma unroll
+        for (int j = 0; j < kTcFbRows; j++)
+#pragma unroll
+            for (int m = 0; m < M; m++) facc[j][m] = 0.0f;
+
+        for (int piece = 0; piece < npieces; piece++, st_idx++) {
+            const int st = st_idx % NS;
+            // on expiry the tile is garbage, but the warp still reaches every barrier
+            mbar_wait(full + st, (st_idx / NS) & 1, abort);
+            const uint8_t *tp = stages + (size_t)st * a.tile_bytes;
+            const int kbase = piece * KP;                 // offset inside the slice
+            const int kps = min(KP, kcs - kbase);
+            if (fast) {
+                const int SC = kps / 128;
+                const int sb = warp * SC / kTcParts, se = (warp + 1) * SC / kTcParts;
+                const uint8_t *c0p = tp + g * CS + 16 * t4;
+                const uint8_t *c1p = c0p + 8 * CS;
+                const uint8_t *s0p = tp + kTcRows * CS + g * SS + 2 * t4;
+                const uint8_t *s1p = s0p + 8 * SS;
+#pragma unroll 2
+                for (int s = sb; s < se; s++) {
+                    uint32_t h0[16], h1[16];
+                    decode_row32(*reinterpret_cast<const uint4 *>(c0p + s * 64),
+                                 *reinterpret_cast<const uint16_t *>(s0p + s * 8), h0);
+                    decode_row32(*reinterpret_cast<const uint4 *>(c1p + s * 64),
+                                 *reinterpret_cast<const uint16_t *>(s1p + s * 8), h1);
+#pragma unroll
+                    for (int n = 0; n < NT; n++) {
+                        const int m = n * 8 + g;
+#pragma unroll
+                        for (int j = 0; j < 4; j++) {   // MMAs 2j, 2j+1: k = 32t + 8j .. +7
+                            uint4 xb = make_uint4(0, 0, 0, 0);
+                            if (m < M)
+                                xb = *reinterpret_cast<const uint4 *>(xs + (size_t)m * XS + kbase + s * 128 + j * 32 +
+                                                                      t4 * 8);
+                            mma_f16_16816(acc[n][2 * j], h0[4 * j], h1[4 * j], h0[4 * j + 1], h1[4 * j + 1], xb.x, xb.y);
+                            mma_f16_16816(acc[n][2 * j + 1], h0[4 * j + 2], h1[4 * j + 2], h0[4 * j + 3],
+                                          h1[4 * j + 3], xb.z, xb.w);
+                        }
+                    }
+                }
+            } else {
+                // binary32 CUDA-core path: warp w handles rows kTcFbRows*w ..
+                const int ngr = kps / 16;
+#pragma unroll
+                for (int j = 0; j < kTcFbRows; j++) {
+                    const int row = kTcFbRows * warp + j;
+                    if (row < rows) {
+                        for (int q = lane; q < ngr; q += 32) {
+                            const uint2 c = *reinterpret_cast<const uint2 *>(tp + row * CS + q * 8);
+                            const float sv = e4m3_to_f32(tp[kTcRows * CS + row * SS + q]);
+                            float2 w[8];
+                            decode_nvfp4(c, w);
+#pragma unroll
+                            for (int m = 0; m < M; m++) {
+                                float2 xv[8];
+                                load_x16(xs + (size_t)m * XS + kbase + q * 16, xv);
+                                facc[j][m] = dot_group<8>(w, xv, sv, facc[j][m]);
+                            }
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty + st);
+        }
+
+        // ---- this tile's partial sums -> shared memory ----
+        const bool all_at_end = a.red_tiles >= ntiles;
+        float *rb = red + (size_t)(all_at_end ? tile : (tile & 1)) * kTcParts * kTcRows * M;
+        if (fast) {
+#pragma unroll
+            for (int n = 0; n < NT; n++) {
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    const int row = g + ((i & 2) ? 8 : 0);
+                    const int m = n * 8 + 2 * t4 + (i & 1);
+                    float v = 0.0f;
+#pragma unroll
+                    for (int q = 0; q < 8; q++) v += acc[n][q][i];
+                    if (m < M) rb[(warp * kTcRows + row) * M + m] = v;
+                }
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < kTcFbRows; j++)
+#pragma unroll
+                for (int m = 0; m < M; m++) {
+                    float v = facc[j][m];
+#pragma unroll
+                    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+                    if (lane == 0) rb[(kTcFbRows * warp + j) * M + m] = v;
+                }
+        }
+        if (!all_at_end) {
+            named_barrier_sync(1, kTcWarps * 32);
+            reduce_tile(a, rb, rt, rows, fast ? kTcParts : 1, gs, yexp, slice, M);
+        }
+    }
+    if (a.red_tiles >= ntiles) {
+        // every tile's parts are in shared memory: one barrier, then all threads sum
+        named_barrier_sync(1, kTcWarps * 32);
+        const int nparts = fast ? kTcParts : 1;
+        const int per_tile = kTcRows * M;
+        for (int i = threadIdx.x; i < ntiles * per_tile; i += kTcWarps * 32) {
+            const int tile = i / per_tile, row = (i % per_tile) / M, m = i % M;
+            const long long n = r0 + (long long)tile * kTcRows + row;
+            if (n >= r1) continue;
+            const float *rb = red + (size_t)tile * kTcParts * kTcRows * M;
+            float s = 0.0f;
+            for (int q = 0; q < nparts; q++) s += rb[(q * kTcRows + row) * M + m];
+            if (gridDim.y == 1)
+                a.y[(size_t)m * N + n] = gs * mul_pow2(s, yexp);
+            else
+                a.partial[((size_t)slice * M + m) * N + n] = mul_pow2(s, yexp);
+        }
+    }
+}
+
+}  // namespace w4

@@ -8,6 +8,7 @@
 #include "common.cuh"
 #include "pack.cuh"
 #include "gemv.cuh"
+#include "gemv_tc.cuh"
 #include "gemm.cuh"
 
 using namespace w4;
@@ -157,6 +158,150 @@ w4_status launch_gemv_fmt(const w4_weights *w, const void *x, int M, float *y, v
     return W4_ERR_ARG;
 }
 
+// NVFP4 decode GEMV on the tensor cores (gemv_tc.cuh).
+struct GemvTcPlan {
+    int S = 1, kc = 0, KP = 0, NS = 0, xstride = 0, tile_bytes = 0, grid = 0;
+    int rows_mode = 0, tiles_per_cta = 0, box_min_rows = 4, red_tiles = 2;
+    size_t smem = 0, ws_bytes = 0;
+};
+
+constexpr int kTcPieceMax = 4096;      // k per stage (TMA box: 256 8-byte elements of codes)
+constexpr double kSmBytesPerUs = 48e3;  // bytes per us one SM streams with a deep copy ring
+constexpr double kHbmBytesPerUs = 7e6;  // whole-device streaming rate
+constexpr double kCopyUs = 0.2;         // cost of one bulk / tensor copy on an SM
+
+w4_status plan_gemv_tc(int K, int N, int M, bool pdl, GemvTcPlan &p) {
+    DeviceInfo d;
+    if (device_info(d) != W4_OK) return W4_ERR_CUDA;
+    const int unit = 256;
+    const int units = K / unit;
+    int per = (int)std::max<size_t>(1, kXBudget / ((size_t)2 * M * unit));
+    per = std::min(per, units);
+    p.kc = per * unit;
+    p.S = (units + per - 1) / per;
+    const int npieces = (p.kc + kTcPieceMax - 1) / kTcPieceMax;
+    p.KP = ((p.kc + npieces - 1) / npieces + unit - 1) / unit * unit;
+    p.xstride = p.kc + 32;
+    p.tile_bytes = (kTcRows * (p.KP / 2 + p.KP / 16) + 127) & ~127;
+    const size_t xs = ((size_t)M * p.xstride * 2 + 127) & ~(size_t)127;
+    const size_t tail = 16 + 4 * kTcWarps;   // flags
+    const size_t budget = std::min<size_t>(pdl ? 110 * 1024 : 200 * 1024, (size_t)d.smem_optin);
+
+    // rows per CTA: balanced ranges (a partial last tile per CTA) or whole tiles
+    const double rowB = (double)K / 2 + K / 16;
+    const int T = (N + kTcRows - 1) / kTcRows;
+    const int gA = std::min(d.sms, N);
+    const int rowsA = (N + gA - 1) / gA, tailA = rowsA % kTcRows, fullA = rowsA / kTcRows;
+    const int readA = fullA * kTcRows + (tailA >= p.box_min_rows ? kTcRows : tailA);
+    const int copiesA = 2 * fullA + (tailA == 0 ? 0 : (tailA >= p.box_min_rows ? 2 : 2 * tailA));
+    const double costA = std::max(readA * rowB / kSmBytesPerUs, (double)N * rowB / kHbmBytesPerUs) +
+                         copiesA * p.S * kCopyUs;
+    const int q = (T + d.sms - 1) / d.sms, gB = (T + q - 1) / q;
+    const double costB = std::max(q * kTcRows * rowB / kSmBytesPerUs, (double)T * kTcRows * rowB / kHbmBytesPerUs) +
+                         2 * q * p.S * kCopyUs;
+    int tiles_max;
+    if (costB <= costA) {
+        p.rows_mode = 1;
+        p.tiles_per_cta = q;
+        p.grid = gB;
+        tiles_max = q;
+    } else {
+        p.rows_mode = 0;
+        p.tiles_per_cta = 0;
+        p.grid = gA;
+        tiles_max = (rowsA + kTcRows - 1) / kTcRows;
+    }
+    // partial sums of all of a CTA's tiles at once when they fit (one barrier per CTA)
+    const size_t part_bytes = (size_t)kTcParts * kTcRows * M * 4;
+    p.red_tiles = (tiles_max * part_bytes <= 24 * 1024) ? std::max(tiles_max, 2) : 2;
+    const size_t red = (size_t)p.red_tiles * part_bytes;
+
+    int NS = 8;
+    while (NS > 2 && xs + (size_t)NS * p.tile_bytes + red + 16 * NS + tail > budget) NS--;
+    p.NS = NS;
+    p.smem = xs + (size_t)NS * p.tile_bytes + red + 16 * NS + tail;
+    if (p.smem > (size_t)d.smem_optin) return W4_ERR_UNSUPPORTED;
+    p.ws_bytes = p.S > 1 ? (size_t)p.S * M * N * sizeof(float) : 0;
+    return W4_OK;
+}
+
+template <int M>
+w4_status launch_gemv_tc_m(const w4_weights *w, const void *x, float *y, void *ws, const GemvTcPlan &p, bool pdl,
+                           cudaStream_t st) {
+    auto kern = gemv_nvfp4_tc_kernel<M>;
+    static size_t configured = 0;
+    if (p.smem > configured) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem) != cudaSuccess)
+            return W4_ERR_CUDA;
+        configured = p.smem;
+    }
+    PFN_encodeTiled enc = get_encode_tiled();
+    if (!enc) return W4_ERR_CUDA;
+    const int K = w->K, N = w->N;
+    CUtensorMap cmap, smap;
+    const cuuint64_t cdims[2] = {(cuuint64_t)K / 16, (cuuint64_t)N};   // codes as 8-byte elements
+    const cuuint64_t cstr[1] = {(cuuint64_t)K / 2};
+    const cuuint32_t cbox[2] = {(cuuint32_t)p.KP / 16, (cuuint32_t)kTcRows};
+    const cuuint64_t sdims[2] = {(cuuint64_t)K / 16, (cuuint64_t)N};
+    const cuuint64_t sstr[1] = {(cuuint64_t)K / 16};
+    const cuuint32_t sbox[2] = {(cuuint32_t)p.KP / 16, (cuuint32_t)kTcRows};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<uint8_t *>(w->codes), cdims, cstr, cbox, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+        enc(&smap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(w->scales), sdims, sstr, sbox, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return W4_ERR_CUDA;
+    GemvTcArgs a;
+    a.codes = w->codes;
+    a.scales = w->scales;
+    a.gscale = w->global_scale;
+    a.x = reinterpret_cast<const uint16_t *>(x);
+    a.y = y;
+    a.partial = reinterpret_cast<float *>(ws);
+    a.K = K;
+    a.N = N;
+    a.kc = p.kc;
+    a.KP = p.KP;
+    a.NS = p.NS;
+    a.xstride = p.xstride;
+    a.tile_bytes = p.tile_bytes;
+    a.rows_mode = p.rows_mode;
+    a.tiles_per_cta = p.tiles_per_cta;
+    a.box_min_rows = p.box_min_rows;
+    a.red_tiles = p.red_tiles;
+    a.pdl = pdl ? 1 : 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.grid, p.S, 1);
+    cfg.blockDim = dim3(kTcThreads, 1, 1);
+    cfg.dynamicSmemBytes = p.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, kern, cmap, smap, a) != cudaSuccess) return W4_ERR_CUDA;
+    if (p.S > 1) {
+        const int MN = M * N;
+        gemv_finalize_kernel<<<std::min((MN + 255) / 256, 1024), 256, 0, st>>>(a.partial, p.S, MN, w->global_scale, y);
+    }
+    return launch_status();
+}
+
+w4_status launch_gemv_tc(const w4_weights *w, const void *x, int M, float *y, void *ws, const GemvTcPlan &p, bool pdl,
+                         cudaStream_t st) {
+    switch (M) {
+#define W4_CASE(m) \
+    case m: return launch_gemv_tc_m<m>(w, x, y, ws, p, pdl, st);
+        W4_CASE(1) W4_CASE(2) W4_CASE(3) W4_CASE(4) W4_CASE(5) W4_CASE(6) W4_CASE(7) W4_CASE(8)
+        W4_CASE(9) W4_CASE(10) W4_CASE(11) W4_CASE(12) W4_CASE(13) W4_CASE(14) W4_CASE(15) W4_CASE(16)
+#undef W4_CASE
+    }
+    return W4_ERR_ARG;
+}
+
 w4_status check_weights(const w4_weights *w) {
     if (!w || !w->codes || w->K <= 0 || w->N <= 0) return W4_ERR_ARG;
     if (w->fmt == W4_FMT_NVFP4) {
@@ -228,6 +373,13 @@ w4_status pack_rocmfp4(const void *W, int K, int N, int block, int fmt, const fl
 
 size_t w4a16_workspace_bytes(const w4_weights *w, int M) {
     if (check_weights(w) != W4_OK || M < 1) return 0;
+    if (M <= 16 && w->fmt == W4_FMT_NVFP4) {
+        if (w->K % 256) return 0;
+        GemvTcPlan p, q;
+        if (plan_gemv_tc(w->K, w->N, M, false, p) != W4_OK) return 0;
+        if (plan_gemv_tc(w->K, w->N, M, true, q) != W4_OK) return p.ws_bytes;
+        return std::max(p.ws_bytes, q.ws_bytes);
+    }
     if (M <= 16) {
         if (w->K % k_unit(w->fmt)) return 0;
         GemvPlan p;
@@ -247,12 +399,17 @@ w4_status w4a16_gemv_ex(const w4_weights *w, const void *x, int M, float *y, voi
     if (!aligned16(x) || !aligned16(y) || (workspace && !aligned16(workspace))) return W4_ERR_ALIGN;
     if (w->K % k_unit(w->fmt)) return W4_ERR_UNSUPPORTED;
     const bool pdl = (flags & W4_LAUNCH_PDL) != 0;
+    cudaStream_t st = as_stream(stream);
+    if (w->fmt == W4_FMT_NVFP4) {
+        GemvTcPlan p;
+        if ((s = plan_gemv_tc(w->K, w->N, M, pdl, p)) != W4_OK) return s;
+        if (p.ws_bytes && (!workspace || workspace_bytes < p.ws_bytes)) return W4_ERR_WORKSPACE;
+        return launch_gemv_tc(w, x, M, y, workspace, p, pdl, st);
+    }
     GemvPlan p;
     if ((s = plan_gemv(w->fmt, w->K, w->N, M, pdl, p)) != W4_OK) return s;
     if (p.ws_bytes && (!workspace || workspace_bytes < p.ws_bytes)) return W4_ERR_WORKSPACE;
-    cudaStream_t st = as_stream(stream);
     switch (w->fmt) {
-    case W4_FMT_NVFP4: return launch_gemv_fmt<W4_FMT_NVFP4>(w, x, M, y, workspace, p, pdl, st);
     case W4_FMT_ROCMFP4_DUAL: return launch_gemv_fmt<W4_FMT_ROCMFP4_DUAL>(w, x, M, y, workspace, p, pdl, st);
     case W4_FMT_ROCMFP4_FAST: return launch_gemv_fmt<W4_FMT_ROCMFP4_FAST>(w, x, M, y, workspace, p, pdl, st);
     }
