@@ -159,6 +159,14 @@ w4_status w4a16_gemv(const w4_weights *w, const void *x, int M, float *y,
  * back-to-back layers.
  */
 #define W4_LAUNCH_PDL 1u
+/*
+ * W4_LAUNCH_TMEM (NVFP4, M == 1, K % 512 == 0, K <= 12288; otherwise ignored)
+ * selects the GEMV whose products run on tcgen05.mma with the decoded weights
+ * in tensor memory (A from TMEM, x from shared memory).  Results meet the same
+ * tolerance as the default path; on B200 it is currently slower than the
+ * default mma.sync kernel, so it is opt-in.
+ */
+#define W4_LAUNCH_TMEM 2u
 w4_status w4a16_gemv_ex(const w4_weights *w, const void *x, int M, float *y,
                         void *workspace, size_t workspace_bytes, unsigned flags,
                         void *stream);

@@ -159,3 +159,75 @@ def test_activation_range_cases(case, M):
     else:
         x[:, ::3] = 2.0 ** -130
     run_and_check(pw, wh, I.bf16_rne(x))
+
+
+@pytest.mark.parametrize("case", ["zeros", "one_block", "range_2p30", "far_blocks", "inf"])
+@pytest.mark.parametrize("K,N", [(2560, 300), (9728, 160)])
+def test_single_token_block_exponents(case, K, N):
+    """One token: x is converted per 16-k block with its own power of two, and a
+    warp whose blocks it cannot all convert exactly falls back to binary32."""
+    pw, wh = nvfp4_packed(I.sweep_weights(K, N, 3)[:N].contiguous())
+    x = I.activations(1, K, 5).double()
+    if case == "zeros":
+        x[:] = 0.0
+    elif case == "one_block":
+        x[:] = 0.0
+        x[:, 4 * 16:5 * 16] = I.activations(1, 16, 6).double()
+    elif case == "range_2p30":          # inside one block: still exact in f16 after scaling
+        x[:, 16:24] *= 2.0 ** 15
+        x[:, 24:32] *= 2.0 ** -15
+    elif case == "far_blocks":          # blocks of one warp 2^120 apart
+        x[:, :16] *= 2.0 ** 60
+        x[:, 16:32] *= 2.0 ** -60
+    else:
+        x[:, 100] = float("inf")
+    x = I.bf16_rne(x)
+    y = np_of(W4.w4a16_gemv(pw, x.cuda()))
+    yr, ar = O.matmul(x, wh)
+    if case == "inf":
+        # every row with a nonzero weight at k = 100 is +-inf or nan on both sides
+        assert np.array_equal(np.isfinite(y), np.isfinite(yr))
+        fin = np.isfinite(yr)
+        assert_within_tolerance(y[fin], yr[fin], ar[fin])
+    else:
+        assert_within_tolerance(y, yr, ar)
+
+
+@pytest.mark.parametrize("K,N", [(2560, 4096), (9728, 2560), (1024, 1024), (512, 7), (2560, 333), (9728, 2),
+                                 (12288, 5), (4096, 2560)])
+def test_tensor_memory_path(K, N):
+    """The opt-in tcgen05 GEMV (decoded weights in tensor memory) meets the same bound."""
+    pw, wh = nvfp4_packed(I.sweep_weights(K, N, 4)[:N].contiguous())
+    x = I.activations(1, K, 21).double()
+    x = I.bf16_rne(x)
+    for flags in (W4.LAUNCH_TMEM, W4.LAUNCH_TMEM | W4.LAUNCH_PDL):
+        run_and_check(pw, wh, x, flags=flags)
+
+
+@pytest.mark.parametrize("case", ["zeros", "scaled_up", "scaled_down", "wide_range", "inf"])
+def test_tensor_memory_path_ranges(case):
+    """x that the tensor-memory path converts exactly to f16 after scaling, and x it
+    cannot (the binary32 path of the same kernel)."""
+    K, N = 2560, 300
+    pw, wh = nvfp4_packed(I.sweep_weights(K, N, 5)[:N].contiguous())
+    x = I.activations(1, K, 22).double()
+    if case == "zeros":
+        x[:] = 0.0
+    elif case == "scaled_up":
+        x *= 2.0 ** 100
+    elif case == "scaled_down":
+        x *= 2.0 ** -100
+    elif case == "wide_range":
+        x[:, :8] *= 2.0 ** 40
+        x[:, 8:16] *= 2.0 ** -40
+    else:
+        x[:, 700] = float("inf")
+    x = I.bf16_rne(x)
+    y = np_of(W4.w4a16_gemv(pw, x.cuda(), flags=W4.LAUNCH_TMEM))
+    yr, ar = O.matmul(x, wh)
+    if case == "inf":
+        assert np.array_equal(np.isfinite(y), np.isfinite(yr))
+        fin = np.isfinite(yr)
+        assert_within_tolerance(y[fin], yr[fin], ar[fin])
+    else:
+        assert_within_tolerance(y, yr, ar)

@@ -189,6 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                 if (*abort) break;
             }
         }
+        __syncwarp();   // the whole warp reaches the final barrier together (it is .aligned)
     } else if (warp == 1) {
         // ------------------------------- MMA issuer -------------------------------
         if (lane == 0) {
@@ -215,6 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                 mma_commit(&sh.acc_full[b]);
             }
         }
+        __syncwarp();
     } else if (warp < 6) {
         // -------------------------------- epilogue --------------------------------
         const int q = warp & 3;                 // TMEM lane quadrant of this warp

@@ -1,0 +1,342 @@
+// gemv_m1.cuh -- NVFP4 decode GEMV for one token (M = 1): the E2M1 x x products
+// on the tensor cores, the per-16 E4M3 block scales applied afterwards in
+// binary32.
+//
+// y[n] = g * sum_b s[n][b] * sum_{k in block b} e2m1[n][k] * x[k]
+// ("EdgeRock-4B-NVFP4" card, intro: E2M1 values, one E4M3 scale per 16 along K,
+// one FP32 global scale; the fused W4A16 decode kernel of the
+// "Nanbeige4.2-3B-NVFP4A16" card, Serving).
+//
+// Why a separate kernel for M = 1.  In the general tensor-core GEMV a lane
+// turns two codes into f16 with one cvt and multiplies them by their block
+// scale with one HMUL2 before the MMA; with one token only one of the MMA's
+// eight B columns carries data, and the conversion pipe (cvt + HMUL2) is what
+// limits the kernel.  Here the eight columns are the eight 16-k scale blocks of
+// a 128-k super-chunk: B[k][c] = x[k] when k lies in block c, else 0.  The MMA
+// then yields, for each of its 16 rows, the eight unscaled block partial sums
+// D[row][b]; a lane owns two of them per row (the blocks of its own codes) and
+// adds s * D with one FFMA each.  No HMUL2, no scale duplication, and every
+// MMA column is used.
+//
+// x is converted to f16 once per CTA with a power-of-two exponent per 16-k
+// block (sigma_b from the block's largest |x|, so its largest |x'| lies in
+// [2^14, 2^15)).  x' = x * 2^-sigma_b is exact in f16 whenever every nonzero
+// |x'| >= 2^-17 (8 significant bits above f16's 2^-24 quantum).  Each warp
+// converts exactly the blocks it later multiplies, so no CTA barrier is needed;
+// its partial sums are kept relative to 2^sigma_ref (the warp's largest
+// sigma_b) and the per-block factor 2^(sigma_b - sigma_ref) is folded into the
+// scale.  A warp with a block it cannot convert exactly (range above 2^31
+// inside a block, factors below binary32's normal range, Inf/NaN) computes its
+// share in binary32 on the CUDA cores from the bf16 x in global memory.
+//
+// Shared memory: x' [kc + 32] f16 (permuted per super-chunk as in the general
+// kernel), the per-block factors [kc/16] binary32, the NS weight stages, the
+// per-warp partial sums, mbarriers and flags.
+#pragma once
+
+#include "gemv_tc.cuh"
+
+namespace w4 {
+
+// Offsets (bytes) of the M = 1 kernel's shared-memory regions.
+struct M1Layout {
+    size_t pw, stages, red, bars, total;
+};
+
+__host__ __device__ __forceinline__ M1Layout m1_layout(int xstride, int kc, int NS, int tile_bytes, int red_tiles) {
+    M1Layout L;
+    L.pw = ((size_t)xstride * 2 + 127) & ~(size_t)127;
+    L.stages = (L.pw + (size_t)(kc / 16) * 4 + 127) & ~(size_t)127;
+    L.red = L.stages + (size_t)NS * tile_bytes;
+    L.bars = L.red + (size_t)red_tiles * kTcParts * kTcRows * 4;
+    L.total = L.bars + (size_t)(2 * NS + 1) * 8 + 16;
+    return L;
+}
+
+constexpr int kNoSigma = -100000;   // block of zeros (or an unused lane)
+
+// Largest |bf16| bit pattern of 16 values.
+__device__ __forceinline__ uint32_t absmax_bits16(uint4 v0, uint4 v1) {
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    uint32_t m = 0;
+#pragma unroll
+    for (int i = 0; i < 8; i++) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
+    return max(m & 0xFFFFu, m >> 16);
+}
+
+// Two bf16 (one word) -> f16x2 of x * 2^-sigma; `bad` when a nonzero result is
+// below 2^-17 (may be inexact in f16) -- results above f16's range cannot occur
+// for x of the block that sigma was taken from.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_scaled(uint32_t w, int neg_sigma, bool &bad) {
+    const float x0 = mul_pow2(bf16_lo(w), neg_sigma), x1 = mul_pow2(bf16_hi(w), neg_sigma);
+    const float tiny = 7.62939453125e-06f;   // 2^-17
+    bad |= (x0 != 0.0f && fabsf(x0) < tiny) | (x1 != 0.0f && fabsf(x1) < tiny);
+    const __half2 h = __floats2half2_rn(x0, x1);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// 16 code bytes of one row (32 k) -> 16 f16x2 (h[i] = elements 2i, 2i+1), exact.
+__device__ __forceinline__ void decode_codes32(uint4 c, uint32_t (&h)[16]) {
+    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+    for (int i = 0; i < 16; i++) h[i] = e2m1x2_to_f16x2(w[i >> 2] >> (8 * (i & 3)));
+}
+
+// E4M3 byte (bits 0..7 of v after the shift) -> its value * 2^-120 as binary32
+// bits: exponent and mantissa fields moved into place; an E4M3 subnormal becomes
+// a binary32 subnormal of the same scaled value.
+__device__ __forceinline__ float e4m3_lo_scaled(uint32_t v) { return __uint_as_float((v << 20) & 0x07F00000u); }
+__device__ __forceinline__ float e4m3_hi_scaled(uint32_t v) { return __uint_as_float((v << 12) & 0x07F00000u); }
+
+__global__ void __launch_bounds__(kTcThreads, 1)
+    gemv_nvfp4_m1_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant__ CUtensorMap smap,
+                         const GemvTcArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int K = a.K, N = a.N, kc = a.kc, KP = a.KP, NS = a.NS;
+    const int slice = blockIdx.y, k0 = slice * kc, kcs = min(kc, K - k0);
+    const int npieces = (kcs + KP - 1) / KP;
+    const int CS = KP / 2, SS = KP / 16;
+    const M1Layout L = m1_layout(a.xstride, kc, NS, a.tile_bytes, a.red_tiles);
+
+    uint16_t *xs = reinterpret_cast<uint16_t *>(smem);
+    float *pw = reinterpret_cast<float *>(smem + L.pw);   // per-block factor 2^(120 + sigma_b - sigma_ref)
+    uint8_t *stages = smem + L.stages;
+    float *red = reinterpret_cast<float *>(smem + L.red);  // [red_tiles][kTcParts][16]
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bars);
+    uint64_t *empty = full + NS;
+    uint64_t *xfull = empty + NS;
+    int *flags = reinterpret_cast<int *>(xfull + 1);
+    volatile int *abort = flags;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    long long r0, r1;
+    if (a.rows_mode == 0) {
+        r0 = (long long)blockIdx.x * N / gridDim.x;
+        r1 = (long long)(blockIdx.x + 1) * N / gridDim.x;
+    } else {
+        r0 = (long long)blockIdx.x * a.tiles_per_cta * kTcRows;
+        r1 = min((long long)N, r0 + (long long)a.tiles_per_cta * kTcRows);
+    }
+    const int ntiles = (int)((r1 - r0 + kTcRows - 1) / kTcRows);
+    const int nstages = ntiles * npieces;
+
+    if (threadIdx.x == 0) {
+        flags[0] = 0;
+        for (int i = 0; i < NS; i++) {
+            mbar_init(full + i, 1);
+            mbar_init(empty + i, kTcWarps);
+        }
+        mbar_init(xfull, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    pdl_allow_dependents();
+
+    if (warp == kTcWarps) {
+        if (lane == 0)
+            tc_produce(cmap, smap, a, 1, xs, stages, full, empty, xfull, abort, r0, r1, k0, kcs, npieces, nstages);
+        return;
+    }
+
+    // -------------------------------- consumers --------------------------------
+    const float gs = __ldg(a.gscale);
+    pdl_wait_prior_grid();   // y may be read by the previous kernel
+    mbar_wait(xfull, 0, abort);
+
+    // Warp w multiplies super-chunks [sb, se) of every piece (the same share in
+    // every tile), i.e. at most 32 blocks per piece: lane l takes block l.
+    // Pass 1: sigma_b per block, kept in pw[] as an int until sigma_ref is known.
+    bool bad = false;
+    int sref = kNoSigma;
+    for (int p = 0; p < npieces; p++) {
+        const int kb = p * KP, SC = min(KP, kcs - kb) / 128;
+        const int sb = warp * SC / kTcWarps, se = (warp + 1) * SC / kTcWarps;
+        if (lane < 8 * (se - sb)) {
+            const int blk = kb / 16 + 8 * sb + lane;
+            const uint4 *src = reinterpret_cast<const uint4 *>(xs + (size_t)blk * 16);
+            const uint32_t m = absmax_bits16(src[0], src[1]);
+            int sg = kNoSigma;
+            if (m != 0) {
+                bad |= m >= 0x7F80u;                        // Inf / NaN
+                sg = max((int)(m >> 7), 1) - 127 - 14;      // largest |x| * 2^-sg in [2^14, 2^15)
+            }
+            reinterpret_cast<int *>(pw)[blk] = sg;
+            sref = max(sref, sg);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) sref = max(sref, __shfl_xor_sync(0xFFFFFFFFu, sref, o));
+    if (sref == kNoSigma) sref = 0;   // all of this warp's x are zero
+    // Pass 2: convert in place to f16, permuting each super-chunk: the 8 values
+    // k = 32t + 8j .. +7 go to offset 32j + 8t (block b = 2t + j/2).
+    for (int p = 0; p < npieces; p++) {
+        const int kb = p * KP, SC = min(KP, kcs - kb) / 128;
+        const int sb = warp * SC / kTcWarps, se = (warp + 1) * SC / kTcWarps;
+        const bool mine = lane < 8 * (se - sb);
+        const int blk = kb / 16 + 8 * sb + lane;
+        uint4 o0 = make_uint4(0, 0, 0, 0), o1 = o0;
+        if (mine) {
+            const int sg = reinterpret_cast<const int *>(pw)[blk];
+            const uint4 *src = reinterpret_cast<const uint4 *>(xs + (size_t)blk * 16);
+            const uint4 v0 = src[0], v1 = src[1];
+            const int ns = sg == kNoSigma ? 0 : -sg;
+            o0 = make_uint4(bf16x2_to_f16x2_scaled(v0.x, ns, bad), bf16x2_to_f16x2_scaled(v0.y, ns, bad),
+                            bf16x2_to_f16x2_scaled(v0.z, ns, bad), bf16x2_to_f16x2_scaled(v0.w, ns, bad));
+            o1 = make_uint4(bf16x2_to_f16x2_scaled(v1.x, ns, bad), bf16x2_to_f16x2_scaled(v1.y, ns, bad),
+                            bf16x2_to_f16x2_scaled(v1.z, ns, bad), bf16x2_to_f16x2_scaled(v1.w, ns, bad));
+            int fe = 120;   // a zero block: D = 0, any finite factor
+            if (sg != kNoSigma) {
+                fe = 120 + sg - sref;
+                bad |= fe < 3;   // s * 2^(fe - 120) must stay a normal binary32
+            }
+            pw[blk] = __int_as_float((127 + max(fe, 3)) << 23);
+        }
+        __syncwarp();
+        if (mine) {
+            const int bi = blk & 7;
+            uint16_t *dst = xs + (size_t)(blk >> 3) * 128 + 64 * (bi & 1) + 8 * (bi >> 1);
+            *reinterpret_cast<uint4 *>(dst) = o0;
+            *reinterpret_cast<uint4 *>(dst + 32) = o1;
+        }
+        __syncwarp();
+    }
+    const bool fast = !__any_sync(0xFFFFFFFFu, bad);
+    if (!fast) sref = 0;   // binary32 path: partial sums in units of x itself
+
+    // MMA operands.  Lane (g, t) holds rows g, g+8 of the codes of k = 32t .. 32t+31
+    // (blocks 2t, 2t+1) and B column g.  Column g is block g: it is nonzero only for
+    // the k of lanes t = g/2, and only in the MMAs of block g (the first four MMAs
+    // for even g, the last four for odd g).  So the 8 lanes with g/2 == t load x,
+    // two 16-byte pieces each, and the rest feed zeros.
+    const int g = lane >> 2, t4 = lane & 3;
+    const bool xact = (g >> 1) == t4;
+    const bool odd = (g & 1) != 0;
+    // pieces j = 2*odd + {0, 1}; the order (odd lanes j = 3 first) keeps the 8
+    // active lanes of each load on distinct banks
+    const int xoffA = 32 * (odd ? 3 : 0) + 8 * t4, xoffB = 32 * (odd ? 2 : 1) + 8 * t4;
+
+    int st_idx = 0;
+    for (int tile = 0; tile < ntiles; tile++) {
+        float accA = 0.0f, accB = 0.0f;   // rows g, g+8 (fast) / row lane/2 (binary32)
+        for (int piece = 0; piece < npieces; piece++, st_idx++) {
+            const int st = st_idx % NS;
+            // on expiry the tile is garbage, but the warp still reaches every barrier
+            mbar_wait(full + st, (st_idx / NS) & 1, abort);
+            const uint8_t *tp = stages + (size_t)st * a.tile_bytes;
+            const int kbase = piece * KP;
+            const int kps = min(KP, kcs - kbase);
+            const int SC = kps / 128;
+            const int sb = warp * SC / kTcWarps, se = (warp + 1) * SC / kTcWarps;
+            if (fast) {
+                const uint8_t *c0p = tp + g * CS + 16 * t4;
+                const uint8_t *c1p = c0p + 8 * CS;
+                const uint8_t *s0p = tp + kTcRows * CS + g * SS + 2 * t4;
+                const uint8_t *s1p = s0p + 8 * SS;
+                const uint16_t *xp = xs + kbase;
+                const float *pp = pw + kbase / 16 + 2 * t4;
+#pragma unroll 2
+                for (int s = sb; s < se; s++) {
+                    const uint4 c0 = *reinterpret_cast<const uint4 *>(c0p + s * 64);
+                    const uint4 c1 = *reinterpret_cast<const uint4 *>(c1p + s * 64);
+                    const uint32_t sc0 = *reinterpret_cast<const uint16_t *>(s0p + s * 8);
+                    const uint32_t sc1 = *reinterpret_cast<const uint16_t *>(s1p + s * 8);
+                    const float2 pv = *reinterpret_cast<const float2 *>(pp + s * 8);
+                    uint4 xa = make_uint4(0, 0, 0, 0), xb = xa;
+                    if (xact) {
+                        xa = *reinterpret_cast<const uint4 *>(xp + s * 128 + xoffA);
+                        xb = *reinterpret_cast<const uint4 *>(xp + s * 128 + xoffB);
+                    }
+                    // B pieces of MMA pairs j = 0..3 (x of k = 32t + 8j .. +7, or zero)
+                    const uint4 z = make_uint4(0, 0, 0, 0);
+                    const uint4 b0 = odd ? z : xa, b1 = odd ? z : xb, b2 = odd ? xb : z, b3 = odd ? xa : z;
+                    uint32_t h0[16], h1[16];
+                    decode_codes32(c0, h0);
+                    decode_codes32(c1, h1);
+                    float d0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, d1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                    mma_f16_16816(d0, h0[0], h1[0], h0[1], h1[1], b0.x, b0.y);
+                    mma_f16_16816(d0, h0[2], h1[2], h0[3], h1[3], b0.z, b0.w);
+                    mma_f16_16816(d0, h0[4], h1[4], h0[5], h1[5], b1.x, b1.y);
+                    mma_f16_16816(d0, h0[6], h1[6], h0[7], h1[7], b1.z, b1.w);
+                    mma_f16_16816(d1, h0[8], h1[8], h0[9], h1[9], b2.x, b2.y);
+                    mma_f16_16816(d1, h0[10], h1[10], h0[11], h1[11], b2.z, b2.w);
+                    mma_f16_16816(d1, h0[12], h1[12], h0[13], h1[13], b3.x, b3.y);
+                    mma_f16_16816(d1, h0[14], h1[14], h0[15], h1[15], b3.z, b3.w);
+                    // d0 holds block 2t in column 2t, d1 block 2t+1 in column 2t+1
+                    accA = __fmaf_rn(e4m3_lo_scaled(sc0) * pv.x, d0[0], accA);
+                    accA = __fmaf_rn(e4m3_hi_scaled(sc0) * pv.y, d1[1], accA);
+                    accB = __fmaf_rn(e4m3_lo_scaled(sc1) * pv.x, d0[2], accB);
+                    accB = __fmaf_rn(e4m3_hi_scaled(sc1) * pv.y, d1[3], accB);
+                }
+            } else {
+                // binary32 on the CUDA cores: lane l takes row l/2, 64 k of each super-chunk
+                const int row = lane >> 1, half = lane & 1;
+                for (int s = sb; s < se; s++) {
+                    const uint8_t *cp = tp + row * CS + s * 64 + 32 * half;
+                    const uint8_t *sp = tp + kTcRows * CS + row * SS + s * 8 + 4 * half;
+                    const uint4 *xg = reinterpret_cast<const uint4 *>(a.x + k0 + kbase + s * 128 + 64 * half);
+#pragma unroll
+                    for (int q = 0; q < 4; q++) {
+                        const uint2 c = *reinterpret_cast<const uint2 *>(cp + 8 * q);
+                        float2 w[8], xv[8];
+                        decode_nvfp4(c, w);
+                        const uint4 u0 = __ldg(xg + 2 * q), u1 = __ldg(xg + 2 * q + 1);
+                        const uint32_t wv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+                        for (int i = 0; i < 8; i++) xv[i] = make_float2(bf16_lo(wv[i]), bf16_hi(wv[i]));
+                        accA = dot_group<8>(w, xv, e4m3_to_f32(sp[q]), accA);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty + st);
+        }
+
+        // ---- this warp's partial sums of the tile -> shared memory ----
+        const bool all_at_end = a.red_tiles >= ntiles;
+        float *rb = red + (size_t)(all_at_end ? tile : (tile & 1)) * kTcParts * kTcRows;
+        if (fast) {
+            accA += __shfl_xor_sync(0xFFFFFFFFu, accA, 1);
+            accA += __shfl_xor_sync(0xFFFFFFFFu, accA, 2);
+            accB += __shfl_xor_sync(0xFFFFFFFFu, accB, 1);
+            accB += __shfl_xor_sync(0xFFFFFFFFu, accB, 2);
+            if (t4 == 0) {
+                rb[warp * kTcRows + g] = mul_pow2(accA, sref);
+                rb[warp * kTcRows + g + 8] = mul_pow2(accB, sref);
+            }
+        } else {
+            accA += __shfl_xor_sync(0xFFFFFFFFu, accA, 1);
+            if ((lane & 1) == 0) rb[warp * kTcRows + (lane >> 1)] = accA;
+        }
+        if (!all_at_end) {
+            named_barrier_sync(1, kTcWarps * 32);
+            const long long rt = r0 + (long long)tile * kTcRows;
+            const int rows = (int)min((long long)kTcRows, r1 - rt);
+            if (threadIdx.x < rows) {
+                float s = 0.0f;
+                for (int q = 0; q < kTcParts; q++) s += rb[q * kTcRows + threadIdx.x];
+                const long long n = rt + threadIdx.x;
+                if (gridDim.y == 1)
+                    a.y[n] = gs * s;
+                else
+                    a.partial[(size_t)slice * N + n] = s;
+            }
+            // the buffer of tile+2 is written only after every warp passed tile+1's barrier
+        }
+    }
+    if (a.red_tiles >= ntiles) {
+        named_barrier_sync(1, kTcWarps * 32);
+        for (int i = threadIdx.x; i < ntiles * kTcRows; i += kTcWarps * 32) {
+            const long long n = r0 + i;
+            if (n >= r1) continue;
+            const float *rb = red + (size_t)(i / kTcRows) * kTcParts * kTcRows + (i % kTcRows);
+            float s = 0.0f;
+            for (int q = 0; q < kTcParts; q++) s += rb[q * kTcRows];
+            if (gridDim.y == 1)
+                a.y[n] = gs * s;
+            else
+                a.partial[(size_t)slice * N + n] = s;
+        }
+    }
+}
+
+}  // namespace w4

@@ -118,6 +118,52 @@ __device__ __forceinline__ void reduce_tile(const GemvTcArgs &a, const float *rb
     }
 }
 
+// The producer lane: x (after the dependency wait) and the weight stages of a
+// CTA's row range, in order, into the NS-deep ring.  Under programmatic launch
+// the first NS weight stages go out before the wait (weights do not depend on
+// earlier kernels); otherwise x goes first.
+__device__ __forceinline__ void tc_produce(const CUtensorMap &cmap, const CUtensorMap &smap, const GemvTcArgs &a,
+                                           int M, uint16_t *xs, uint8_t *stages, uint64_t *full, uint64_t *empty,
+                                           uint64_t *xfull, volatile int *abort, long long r0, long long r1, int k0,
+                                           int kcs, int npieces, int nstages) {
+    const int K = a.K, KP = a.KP, NS = a.NS, XS = a.xstride;
+    const int CS = KP / 2, SS = KP / 16;
+    const uint64_t pol = policy_evict_first();
+    const int before = a.pdl ? min(NS, nstages) : 0;
+    for (int t = 0; t < nstages + 1; t++) {
+        if (t == before) {
+            pdl_wait_prior_grid();
+            mbar_arrive_expect_tx(xfull, (uint32_t)(M * kcs * 2));
+            for (int m = 0; m < M; m++)
+                bulk_g2s(xs + (size_t)m * XS, a.x + (size_t)m * K + k0, (uint32_t)(kcs * 2), xfull, pol);
+            continue;
+        }
+        const int tt = t > before ? t - 1 : t;   // weight stage index
+        const int st = tt % NS;
+        if (tt >= NS && !mbar_wait(empty + st, ((tt / NS) - 1) & 1, abort)) break;
+        const long long rt = r0 + (long long)(tt / npieces) * kTcRows;
+        const int rows = (int)min((long long)kTcRows, r1 - rt);
+        const int kpos = k0 + (tt % npieces) * KP;
+        const int kps = min(KP, k0 + kcs - kpos);
+        uint8_t *dst = stages + (size_t)st * a.tile_bytes;
+        uint8_t *dsts = dst + kTcRows * CS;
+        if (rows == kTcRows || rows >= a.box_min_rows) {
+            // two boxes of 16 rows x KP (k beyond K and rows beyond N are zero-filled)
+            mbar_arrive_expect_tx(full + st, (uint32_t)(kTcRows * (CS + SS)));
+            tma_load_2d(dst, &cmap, kpos / 16, (int)rt, full + st);
+            tma_load_2d(dsts, &smap, kpos / 16, (int)rt, full + st);
+        } else {
+            // a short tail: row-piece copies of exactly the bytes needed
+            mbar_arrive_expect_tx(full + st, (uint32_t)(rows * (kps / 2 + kps / 16)));
+            for (int i = 0; i < rows; i++) {
+                bulk_g2s(dst + i * CS, a.codes + (rt + i) * (K / 2) + kpos / 2, (uint32_t)(kps / 2), full + st, pol);
+                bulk_g2s(dsts + i * SS, a.scales + (rt + i) * (K / 16) + kpos / 16, (uint32_t)(kps / 16), full + st,
+                         pol);
+            }
+        }
+    }
+}
+
 template <int M>
 __global__ void __launch_bounds__(kTcThreads, 1)
     gemv_nvfp4_tc_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant__ CUtensorMap smap,
@@ -165,46 +211,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const float gs = __ldg(a.gscale);   // weights do not depend on earlier kernels
 
     if (warp == kTcWarps) {
-        // ------------------------------ producer ------------------------------
-        if (lane == 0) {
-            const uint64_t pol = policy_evict_first();
-            // x depends on the previous kernel: copy it after the dependency wait.  Under
-            // programmatic launch the first NS weight stages go out before that wait.
-            const int before = a.pdl ? min(NS, nstages) : 0;
-            for (int t = 0; t < nstages + 1; t++) {
-                if (t == before) {
-                    pdl_wait_prior_grid();
-                    mbar_arrive_expect_tx(xfull, (uint32_t)(M * kcs * 2));
-                    for (int m = 0; m < M; m++)
-                        bulk_g2s(xs + (size_t)m * XS, a.x + (size_t)m * K + k0, (uint32_t)(kcs * 2), xfull, pol);
-                    continue;
-                }
-                const int tt = t > before ? t - 1 : t;   // weight stage index
-                const int st = tt % NS;
-                if (tt >= NS && !mbar_wait(empty + st, ((tt / NS) - 1) & 1, abort)) break;
-                const long long rt = r0 + (long long)(tt / npieces) * kTcRows;
-                const int rows = (int)min((long long)kTcRows, r1 - rt);
-                const int kpos = k0 + (tt % npieces) * KP;
-                const int kps = min(KP, k0 + kcs - kpos);
-                uint8_t *dst = stages + (size_t)st * a.tile_bytes;
-                uint8_t *dsts = dst + kTcRows * CS;
-                if (rows == kTcRows || rows >= a.box_min_rows) {
-                    // two boxes of 16 rows x KP (k beyond K and rows beyond N are zero-filled)
-                    mbar_arrive_expect_tx(full + st, (uint32_t)(kTcRows * (CS + SS)));
-                    tma_load_2d(dst, &cmap, kpos / 16, (int)rt, full + st);
-                    tma_load_2d(dsts, &smap, kpos / 16, (int)rt, full + st);
-                } else {
-                    // a short tail: row-piece copies of exactly the bytes needed
-                    mbar_arrive_expect_tx(full + st, (uint32_t)(rows * (kps / 2 + kps / 16)));
-                    for (int i = 0; i < rows; i++) {
-                        bulk_g2s(dst + i * CS, a.codes + (rt + i) * (K / 2) + kpos / 2, (uint32_t)(kps / 2),
-                                 full + st, pol);
-                        bulk_g2s(dsts + i * SS, a.scales + (rt + i) * (K / 16) + kpos / 16, (uint32_t)(kps / 16),
-                                 full + st, pol);
-                    }
-                }
-            }
-        }
+        if (lane == 0)
+            tc_produce(cmap, smap, a, M, xs, stages, full, empty, xfull, abort, r0, r1, k0, kcs, npieces, nstages);
         return;
     }
 

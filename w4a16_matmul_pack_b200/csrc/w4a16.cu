@@ -9,6 +9,8 @@
 #include "pack.cuh"
 #include "gemv.cuh"
 #include "gemv_tc.cuh"
+#include "gemv_m1.cuh"
+#include "gemv_umma.cuh"
 #include "gemm.cuh"
 
 using namespace w4;
@@ -216,10 +218,14 @@ w4_status plan_gemv_tc(int K, int N, int M, bool pdl, GemvTcPlan &p) {
     p.red_tiles = (tiles_max * part_bytes <= 24 * 1024) ? std::max(tiles_max, 2) : 2;
     const size_t red = (size_t)p.red_tiles * part_bytes;
 
+    auto total = [&](int ns) -> size_t {
+        if (M == 1) return m1_layout(p.xstride, p.kc, ns, p.tile_bytes, p.red_tiles).total;
+        return xs + (size_t)ns * p.tile_bytes + red + 16 * ns + tail;
+    };
     int NS = 8;
-    while (NS > 2 && xs + (size_t)NS * p.tile_bytes + red + 16 * NS + tail > budget) NS--;
+    while (NS > 2 && total(NS) > budget) NS--;
     p.NS = NS;
-    p.smem = xs + (size_t)NS * p.tile_bytes + red + 16 * NS + tail;
+    p.smem = total(NS);
     if (p.smem > (size_t)d.smem_optin) return W4_ERR_UNSUPPORTED;
     p.ws_bytes = p.S > 1 ? (size_t)p.S * M * N * sizeof(float) : 0;
     return W4_OK;
@@ -228,7 +234,8 @@ w4_status plan_gemv_tc(int K, int N, int M, bool pdl, GemvTcPlan &p) {
 template <int M>
 w4_status launch_gemv_tc_m(const w4_weights *w, const void *x, float *y, void *ws, const GemvTcPlan &p, bool pdl,
                            cudaStream_t st) {
-    auto kern = gemv_nvfp4_tc_kernel<M>;
+    // one token: block scales applied after the MMA (gemv_m1.cuh)
+    auto kern = M == 1 ? gemv_nvfp4_m1_kernel : gemv_nvfp4_tc_kernel<M>;
     static size_t configured = 0;
     if (p.smem > configured) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem) != cudaSuccess)
@@ -287,6 +294,93 @@ w4_status launch_gemv_tc_m(const w4_weights *w, const void *x, float *y, void *w
         const int MN = M * N;
         gemv_finalize_kernel<<<std::min((MN + 255) / 256, 1024), 256, 0, st>>>(a.partial, p.S, MN, w->global_scale, y);
     }
+    return launch_status();
+}
+
+// One token on tcgen05 (gemv_umma.cuh, opt-in with W4_LAUNCH_TMEM): K a
+// multiple of 512 and small enough that x (twice) and two weight stages fit
+// next to a co-resident CTA.
+constexpr int kUmmaMaxK = 12288;
+
+struct UmmaPlan {
+    int TB = 1, NS = 2, grid = 0;
+    size_t smem = 0;
+};
+
+bool umma_applies(int K, int M) { return M == 1 && K % um::kStepK == 0 && K <= kUmmaMaxK; }
+
+w4_status plan_umma(int K, int N, bool pdl, UmmaPlan &p) {
+    DeviceInfo d;
+    if (device_info(d) != W4_OK) return W4_ERR_CUDA;
+    const int T = (N + um::kTileRows - 1) / um::kTileRows;
+    p.grid = std::min(d.sms, T);
+    const double tile_bytes = um::kTileRows * (K / 2.0 + K / 16.0);
+    // stages of about 16-24 KB (bulk copies below that lose bandwidth), at most
+    // the CTA's own tile count
+    const int tiles_per_cta = (T + p.grid - 1) / p.grid;
+    p.TB = std::max(1, std::min({8, tiles_per_cta, (int)(20480.0 / tile_bytes + 0.5)}));
+    const size_t budget = std::min<size_t>(pdl ? 110 * 1024 : 200 * 1024, (size_t)d.smem_optin);
+    p.NS = 8;
+    while (p.NS > 2 && um::layout(K, p.TB, p.NS).total > budget) p.NS--;
+    p.smem = um::layout(K, p.TB, p.NS).total;
+    if (p.smem > (size_t)d.smem_optin) return W4_ERR_UNSUPPORTED;
+    return W4_OK;
+}
+
+w4_status launch_umma(const w4_weights *w, const void *x, float *y, const UmmaPlan &p, bool pdl, cudaStream_t st) {
+    static size_t configured = 0;
+    if (p.smem > configured) {
+        if (cudaFuncSetAttribute(um::gemv_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem) !=
+            cudaSuccess)
+            return W4_ERR_CUDA;
+        configured = p.smem;
+    }
+    PFN_encodeTiled enc = get_encode_tiled();
+    if (!enc) return W4_ERR_CUDA;
+    const int K = w->K, N = w->N;
+    // codes as [N][K/512][32 x 8 bytes], scales as [N][K/512][32 bytes]; boxes of
+    // 4*TB rows (full stages) and 4 rows (a CTA's last, partial stage)
+    CUtensorMap cmap, smap, cmap1, smap1;
+    const cuuint64_t cdims[3] = {32, (cuuint64_t)K / 512, (cuuint64_t)N};
+    const cuuint64_t cstr[2] = {256, (cuuint64_t)K / 2};
+    const cuuint64_t sdims[3] = {32, (cuuint64_t)K / 512, (cuuint64_t)N};
+    const cuuint64_t sstr[2] = {32, (cuuint64_t)K / 16};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    auto encode = [&](CUtensorMap *m, CUtensorMapDataType dt, const void *base, const cuuint64_t *dims,
+                      const cuuint64_t *str, int rows) {
+        const cuuint32_t box[3] = {32, (cuuint32_t)K / 512, (cuuint32_t)rows};
+        return enc(m, dt, 3, const_cast<void *>(base), dims, str, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    };
+    if (!encode(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT64, w->codes, cdims, cstr, um::kTileRows * p.TB) ||
+        !encode(&smap, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->scales, sdims, sstr, um::kTileRows * p.TB) ||
+        !encode(&cmap1, CU_TENSOR_MAP_DATA_TYPE_UINT64, w->codes, cdims, cstr, um::kTileRows) ||
+        !encode(&smap1, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->scales, sdims, sstr, um::kTileRows))
+        return W4_ERR_CUDA;
+    um::Args a;
+    a.codes = w->codes;
+    a.scales = w->scales;
+    a.gscale = w->global_scale;
+    a.x = reinterpret_cast<const uint16_t *>(x);
+    a.y = y;
+    a.K = K;
+    a.N = N;
+    a.TB = p.TB;
+    a.NS = p.NS;
+    a.pdl = pdl ? 1 : 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.grid, 1, 1);
+    cfg.blockDim = dim3(um::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = p.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, um::gemv_umma_kernel, cmap, smap, cmap1, smap1, a) != cudaSuccess)
+        return W4_ERR_CUDA;
     return launch_status();
 }
 
@@ -374,7 +468,7 @@ w4_status pack_rocmfp4(const void *W, int K, int N, int block, int fmt, const fl
 size_t w4a16_workspace_bytes(const w4_weights *w, int M) {
     if (check_weights(w) != W4_OK || M < 1) return 0;
     if (M <= 16 && w->fmt == W4_FMT_NVFP4) {
-        if (w->K % 256) return 0;
+        if (w->K % 256) return 0;   // (the tensor-memory path needs none either)
         GemvTcPlan p, q;
         if (plan_gemv_tc(w->K, w->N, M, false, p) != W4_OK) return 0;
         if (plan_gemv_tc(w->K, w->N, M, true, q) != W4_OK) return p.ws_bytes;
@@ -395,12 +489,17 @@ w4_status w4a16_gemv_ex(const w4_weights *w, const void *x, int M, float *y, voi
                         size_t workspace_bytes, unsigned flags, void *stream) {
     w4_status s = check_weights(w);
     if (s != W4_OK) return s;
-    if (!x || !y || M < 1 || M > 16 || (flags & ~W4_LAUNCH_PDL)) return W4_ERR_ARG;
+    if (!x || !y || M < 1 || M > 16 || (flags & ~(W4_LAUNCH_PDL | W4_LAUNCH_TMEM))) return W4_ERR_ARG;
     if (!aligned16(x) || !aligned16(y) || (workspace && !aligned16(workspace))) return W4_ERR_ALIGN;
     if (w->K % k_unit(w->fmt)) return W4_ERR_UNSUPPORTED;
     const bool pdl = (flags & W4_LAUNCH_PDL) != 0;
     cudaStream_t st = as_stream(stream);
     if (w->fmt == W4_FMT_NVFP4) {
+        if ((flags & W4_LAUNCH_TMEM) && umma_applies(w->K, M)) {
+            UmmaPlan u;
+            if ((s = plan_umma(w->K, w->N, pdl, u)) != W4_OK) return s;
+            return launch_umma(w, x, y, u, pdl, st);
+        }
         GemvTcPlan p;
         if ((s = plan_gemv_tc(w->K, w->N, M, pdl, p)) != W4_OK) return s;
         if (p.ws_bytes && (!workspace || workspace_bytes < p.ws_bytes)) return W4_ERR_WORKSPACE;
