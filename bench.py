@@ -400,9 +400,10 @@ def run_ours(args, world, rank, local):
     achieved = step_bytes / ms_step / 1e6 / 1.0
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": TRAFFIC_PER_LAUNCH,
-            "kernel": "w4::gemv_kernel<NVFP4, M=1, R=4>",
-            "note": f"algorithmic bytes per launch averaged over the 5 sweep shapes ({step_bytes / 5:.0f} B) "
-                    f"/ average launch duration in the timed PDL graph; peak = {pk['source']} copy bandwidth"}
+            "kernel": "w4::gemv_nvfp4_m1_kernel",
+            "note": f"every launch of the step is this kernel: algorithmic bytes per launch averaged over the 5 "
+                    f"sweep shapes ({step_bytes / 5:.0f} B) / average launch duration in the timed PDL graph "
+                    f"(CUDA events on the launching stream); peak = {pk['source']} copy bandwidth"}
 
     # end-to-end through the public API with pinned host buffers
     xh = [m["x"].cpu().pin_memory() for m in mats]

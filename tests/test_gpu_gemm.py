@@ -28,9 +28,9 @@ def half_ulp_bf16(v):
     return np.where(a > 0, 2.0 ** (e - 8), 2.0 ** -134)
 
 
-def check(pw, cs, x, rows=None):
+def check(pw, cs, x, rows=None, workspace=None):
     c, s, g = cs
-    y32, y16 = W4.w4a16_gemm(pw, x.cuda())
+    y32, y16 = W4.w4a16_gemm(pw, x.cuda(), workspace=workspace)
     torch.cuda.synchronize()
     y32, y16 = np_of(y32), np_of(y16.float())
     N = pw.N
@@ -81,3 +81,28 @@ def test_unsupported_inputs():
     with pytest.raises(W4.W4Error) as e:
         W4.w4a16_gemm(pr, I.activations(4, 128, 1).cuda())
     assert e.value.status == 3
+
+
+def test_operand_modes_per_token_tile():
+    """Token tiles whose rows convert exactly to f16 (after a power-of-two scale per
+    row) run on f16 operands; a tile holding a row with a wider range than f16 can
+    represent runs on BF16 operands.  Both meet the bound, in one call."""
+    M, N, K = 600, 256, 1024
+    W = I.matrix("student_t4", N, K, 11, 0.02, 1e-3)
+    x = I.activations(M, K, 12, outlier_cols=16).double()
+    x[300, :8] *= 2.0 ** 40            # token tile 1: not exact in f16 -> BF16 operands
+    x[300, 8:16] *= 2.0 ** -40
+    x[520:530] *= 2.0 ** 100           # token tile 2: large but exact after scaling
+    x[540:545] *= 2.0 ** -100
+    x[560] = 0.0
+    pw, cs = packed(W)
+    check(pw, cs, I.bf16_rne(x))
+
+
+def test_bf16_operands_without_workspace():
+    """Without a workspace every tile runs on BF16 operands."""
+    M, N, K = 300, 200, 512
+    W = I.matrix("student_t4", N, K, 13, 0.02, 1e-3)
+    x = I.activations(M, K, 14, outlier_cols=16)
+    pw, cs = packed(W)
+    check(pw, cs, x, workspace=torch.empty(0, dtype=torch.uint8, device="cuda"))

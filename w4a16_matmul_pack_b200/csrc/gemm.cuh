@@ -12,17 +12,29 @@
 // swizzle.  Persistent CTAs, one per SM, walk the tiles n-major so that CTAs
 // running together share the same packed weight rows in L2.
 //
-// Warp roles (14 warps):
+// Warp roles (15 warps):
 //   warp 0      TMA producer of x tiles (cp.async.bulk.tensor, no multicast);
 //               allocates / frees the 512 TMEM columns.
 //   warp 1      MMA issuer (one thread): 4 x (128x256x16) per stage, commits to
 //               the stage barriers, and to the accumulator barrier per tile.
+//               It never waits on an mbarrier itself (see below): warp 14 does,
+//               and releases it through named barrier 2 once per stage.
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
 //               32*(w%4)..+31), times g, float32 / BF16 stores.
 //   warps 6-13  dequantise: thread (row r, half h) turns 32 codes + 2 scales of
 //               row r into BF16 in the swizzled A stage.
 // Two accumulators of 256 columns let the epilogue of a tile overlap the MMAs
 // of the next.  Every mbarrier wait is bounded (common.cuh: mbar_wait).
+//
+// Operand precision per tile of 256 tokens.  e2m1 * scale is exact in f16 as
+// well as in BF16, and in f16 it costs one cvt (E2M1 -> f16x2) and one HMUL2
+// per pair of weights instead of a round trip through binary32.  So when the
+// caller provides a workspace, x_to_f16_kernel first converts each token row to
+// f16 as x * 2^-sigma_m (sigma_m from the row's largest |x|) and flags the rows
+// it cannot convert exactly (a nonzero |x * 2^-sigma_m| below 2^-17, or Inf /
+// NaN).  A tile whose 256 rows all converted exactly runs kind::f16 with f16
+// operands and the epilogue multiplies token m by 2^sigma_m; any other tile (or
+// every tile, without a workspace) runs the BF16 operands described above.
 #pragma once
 
 #include "common.cuh"
@@ -35,7 +47,7 @@ constexpr int BM = 128;      // weight rows per tile (MMA M)
 constexpr int BN = 256;      // tokens per tile (MMA N)
 constexpr int BK = 64;       // k per stage (one 128-byte swizzle row of BF16)
 constexpr int STAGES = 4;
-constexpr int kWarps = 14;
+constexpr int kWarps = 15;
 constexpr int kThreads = kWarps * 32;
 constexpr int kDequantThreads = 256;
 constexpr int kEpiThreads = 128;
@@ -50,6 +62,10 @@ constexpr uint32_t W_STAGE_BYTES = BM * WK / 2;   // 16 KB of codes (128 rows x 
 // B = BF16 (bits 10-12), both K-major, N >> 3 at bit 17, M >> 4 at bit 24.
 constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                            ((uint32_t)(BM >> 4) << 24);
+// The same with A = B = F16 (format 0).
+constexpr uint32_t IDESC_F16 = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+constexpr int kMaxTilesM = 256;
+constexpr int kWaitWarp = 14;     // waits on mbarriers for the MMA issuer (warp 1)   // token tiles whose operand mode is kept in shared memory (M <= 65536)
 
 struct SharedStorage {
     uint8_t x[STAGES][X_STAGE_BYTES];   // 1024-byte aligned (swizzle atoms)
@@ -61,6 +77,7 @@ struct SharedStorage {
     uint64_t acc_full[2], acc_empty[2];
     uint32_t tmem_base;
     int abort;
+    int f16_tile[kMaxTilesM];   // token tile mt runs with f16 operands (else BF16)
 };
 
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row atoms of
@@ -77,12 +94,13 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+__device__ __forceinline__ void mma_f16kind(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(IDESC), "r"(accumulate));
+        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
@@ -116,17 +134,82 @@ __device__ __forceinline__ uint4 dequant8(uint32_t cw, float s) {
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// The same 8 weights as f16x2 words: cvt E2M1 -> f16x2, HMUL2 by the scale
+// (s2 = the scale in both halves).  Exact (at most 6 significant bits, in
+// [2^-10, 2688]).
+__device__ __forceinline__ uint4 dequant8_f16(uint32_t cw, uint32_t s2) {
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const uint32_t h = e2m1x2_to_f16x2(cw >> (8 * i));
+        const __half2 v = __hmul2(*reinterpret_cast<const __half2 *>(&h), *reinterpret_cast<const __half2 *>(&s2));
+        o[i] = *reinterpret_cast<const uint32_t *>(&v);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// Row m of x -> f16 as x * 2^-sigma_m, sigma_m chosen so that the row's largest
+// |x * 2^-sigma_m| lies in [2^14, 2^15); bad[m] = 1 when some nonzero value
+// lands below 2^-17 (then it may be inexact in f16) or the row holds Inf / NaN.
+// One block per row; every launch rewrites sigma and bad of every row.
+__global__ void __launch_bounds__(256) x_to_f16_kernel(const uint16_t *x, uint16_t *xh, int *sigma, int *bad, int K) {
+    __shared__ uint32_t red[8];
+    const int m = blockIdx.x;
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)m * K);
+    uint4 *dst = reinterpret_cast<uint4 *>(xh + (size_t)m * K);
+    const int nv = K / 8;
+    uint32_t mx = 0;
+    for (int i = threadIdx.x; i < nv; i += blockDim.x) {
+        const uint4 v = __ldg(src + i);
+        mx = __vmaxu2(mx, v.x & 0x7FFF7FFFu);
+        mx = __vmaxu2(mx, v.y & 0x7FFF7FFFu);
+        mx = __vmaxu2(mx, v.z & 0x7FFF7FFFu);
+        mx = __vmaxu2(mx, v.w & 0x7FFF7FFFu);
+    }
+    mx = max(mx & 0xFFFFu, mx >> 16);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    for (int i = 0; i < 8; i++) mx = max(mx, red[i]);
+    const int sg = (mx == 0) ? 0 : max((int)(mx >> 7), 1) - 127 - 14;
+    const float tiny = 7.62939453125e-06f;   // 2^-17
+    bool b = mx >= 0x7F80u;
+    for (int i = threadIdx.x; i < nv; i += blockDim.x) {
+        const uint4 v = __ldg(src + i);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const float x0 = __uint_as_float(w[j] << 16), x1 = __uint_as_float(w[j] & 0xFFFF0000u);
+            const float a0 = ldexpf(x0, -sg), a1 = ldexpf(x1, -sg);
+            b |= (a0 != 0.0f && fabsf(a0) < tiny) | (a1 != 0.0f && fabsf(a1) < tiny);
+            const __half2 hv = __floats2half2_rn(a0, a1);
+            o[j] = *reinterpret_cast<const uint32_t *>(&hv);
+        }
+        dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    const int any = __syncthreads_or(b ? 1 : 0);
+    if (threadIdx.x == 0) {
+        sigma[m] = sg;
+        bad[m] = any;
+    }
+}
+
 struct Params {
     const uint8_t *codes;
     const uint8_t *scales;
     const float *gscale;
     float *y32;
     __nv_bfloat16 *y16;
+    const int *bad;      // [M] rows not exact in f16, or null (every tile BF16)
+    const int *sigma;    // [M] power of two of each f16 row
     int M, N, K;
     int tiles_m, tiles_n;
 };
 
 __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ CUtensorMap xmap,
+                                                            const __grid_constant__ CUtensorMap xmap16,
                                                             const __grid_constant__ CUtensorMap cmap, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     SharedStorage &sh = *reinterpret_cast<SharedStorage *>(
@@ -154,6 +237,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         }
         fence_mbar_init();
     }
+    const bool use_f16 = p.bad != nullptr && p.tiles_m <= kMaxTilesM;
+    for (int i = threadIdx.x; i < kMaxTilesM; i += kThreads) sh.f16_tile[i] = use_f16 ? 1 : 0;
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                      ::"r"(smem_addr(&sh.tmem_base)), "r"(TMEM_COLS));
@@ -163,6 +248,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sh.tmem_base;
+    if (use_f16) {
+        // a token tile runs on f16 operands only if all of its rows converted exactly
+        for (int i = threadIdx.x; i < p.M; i += kThreads)
+            if (__ldg(p.bad + i)) atomicAnd(&sh.f16_tile[i / BN], 0);
+        __syncthreads();
+    }
 
     if (warp == 0) {
         // ---------------------------- x producer (TMA) ----------------------------
@@ -184,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                     if (it >= STAGES) mbar_wait(&sh.x_empty[s], ((it / STAGES) - 1) & 1, abort);
                     if (*abort) break;
                     mbar_arrive_expect_tx(&sh.x_full[s], X_STAGE_BYTES);
-                    tma_load_2d(sh.x[s], &xmap, kt * BK, m0, &sh.x_full[s]);
+                    tma_load_2d(sh.x[s], sh.f16_tile[t % p.tiles_m] ? &xmap16 : &xmap, kt * BK, m0, &sh.x_full[s]);
                 }
                 if (*abort) break;
             }
@@ -192,31 +283,47 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         __syncwarp();   // the whole warp reaches the final barrier together (it is .aligned)
     } else if (warp == 1) {
         // ------------------------------- MMA issuer -------------------------------
-        if (lane == 0) {
-            int it = 0, lt = 0;
-            for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, lt++) {
-                const int b = lt & 1;
-                if (lt >= 2) mbar_wait(&sh.acc_empty[b], ((lt >> 1) - 1) & 1, abort);
+        // A thread that has MMAs queued stalls on any shared-memory access (an
+        // mbarrier wait included) until they drain, which would leave the tensor
+        // pipe idle between stages.  So this warp never waits on an mbarrier:
+        // warp kWaitWarp waits for each stage (and each accumulator) and then
+        // meets it at named barrier 2; lane 0 issues.
+        int it = 0;
+        for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+            const int b = ((t - blockIdx.x) / gridDim.x) & 1;
+            const uint32_t dtm = tmem + (uint32_t)(b * BN);
+            const uint32_t idesc = sh.f16_tile[t % p.tiles_m] ? IDESC_F16 : IDESC;
+            for (int kt = 0; kt < KT; kt++, it++) {
+                const int s = it % STAGES;
+                named_barrier_sync(2, 64);   // stage s (and, at kt == 0, accumulator b) is ready
                 tc_fence_after();
-                const uint32_t dtm = tmem + (uint32_t)(b * BN);
-                for (int kt = 0; kt < KT; kt++, it++) {
-                    const int s = it % STAGES;
-                    const uint32_t ph = (it / STAGES) & 1;
-                    mbar_wait(&sh.x_full[s], ph, abort);
-                    mbar_wait(&sh.a_full[s], ph, abort);
-                    if (*abort) break;
-                    tc_fence_after();
+                if (lane == 0) {
                     const uint32_t ab = smem_addr(sh.a[s]), xb = smem_addr(sh.x[s]);
 #pragma unroll
                     for (int j = 0; j < BK / 16; j++)
-                        mma_bf16(dtm, sw128_desc(ab + 32 * j), sw128_desc(xb + 32 * j), (kt | j) ? 1u : 0u);
+                        mma_f16kind(dtm, sw128_desc(ab + 32 * j), sw128_desc(xb + 32 * j), idesc, (kt | j) ? 1u : 0u);
                     mma_commit(&sh.x_empty[s]);
                     mma_commit(&sh.a_empty[s]);
+                    if (kt == KT - 1) mma_commit(&sh.acc_full[b]);
                 }
-                mma_commit(&sh.acc_full[b]);
+                __syncwarp();
             }
         }
-        __syncwarp();
+    } else if (warp == kWaitWarp) {
+        // ------------------------- waits on behalf of the MMA issuer -------------------------
+        int it = 0, lt = 0;
+        for (int t = blockIdx.x; t < ntiles; t += gridDim.x, lt++) {
+            const int b = lt & 1;
+            if (lt >= 2) mbar_wait(&sh.acc_empty[b], ((lt >> 1) - 1) & 1, abort);
+            for (int kt = 0; kt < KT; kt++, it++) {
+                const int s = it % STAGES;
+                const uint32_t ph = (it / STAGES) & 1;
+                // on expiry (abort) the stage is garbage, but both warps still meet every barrier
+                mbar_wait(&sh.x_full[s], ph, abort);
+                mbar_wait(&sh.a_full[s], ph, abort);
+                named_barrier_sync(2, 64);
+            }
+        }
     } else if (warp < 6) {
         // -------------------------------- epilogue --------------------------------
         const int q = warp & 3;                 // TMEM lane quadrant of this warp
@@ -228,16 +335,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             mbar_wait(&sh.acc_full[b], (lt >> 1) & 1, abort);
             tc_fence_after();
             const int n = n0 + q * 32 + lane;
+            const bool f16 = sh.f16_tile[t % p.tiles_m] != 0;
             for (int c = 0; c < BN / 32; c++) {
                 uint32_t v[32];
                 W4_TMEM_LD32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * BN + c * 32), v);
                 asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-                if (n < p.N) {
+                // f16 tiles: token m was scaled by 2^-sigma_m (lane j holds sigma of token c*32+j)
+                const int mlane = m0 + c * 32 + lane;
+                const int sgl = (f16 && mlane < p.M) ? __ldg(p.sigma + mlane) : 0;
 #pragma unroll
-                    for (int j = 0; j < 32; j++) {
-                        const int m = m0 + c * 32 + j;
+                for (int j = 0; j < 32; j++) {
+                    const int sg = __shfl_sync(0xFFFFFFFFu, sgl, j);   // every lane takes part
+                    const int m = m0 + c * 32 + j;
+                    if (n < p.N) {
                         if (m < p.M) {
-                            const float val = g * __uint_as_float(v[j]);
+                            const float val = g * (f16 ? mul_pow2(__uint_as_float(v[j]), sg) : __uint_as_float(v[j]));
                             if (p.y32) p.y32[(size_t)m * p.N + n] = val;
                             if (p.y16) p.y16[(size_t)m * p.N + n] = __float2bfloat16_rn(val);
                         }
@@ -260,6 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
             const int n = (t / p.tiles_m) * BM + r;
             const bool valid = n < p.N;
+            const bool f16 = sh.f16_tile[t % p.tiles_m] != 0;
             const uint8_t *srow = p.scales + (size_t)(valid ? n : 0) * (p.K / 16);
             uint32_t sc[KQ], sn[KQ];
 #pragma unroll
@@ -271,29 +384,49 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                     sn[q] = (valid && kw + KQ + q < KT) ? __ldg(reinterpret_cast<const uint32_t *>(srow) + kw + KQ + q) : 0u;
                 mbar_wait(&sh.w_full[ws], (wit / WSTAGES) & 1, abort);
                 const uint8_t *wrow = sh.w[ws] + r * 128;
+                // two k-steps per round: one proxy fence and one pair of arrivals per two A
+                // stages halves the per-stage synchronisation latency of this chain
 #pragma unroll
-                for (int q = 0; q < KQ; q++) {
-                    if (kw + q < KT) {
-                        const int s = it % STAGES;
-                        if (it >= STAGES) mbar_wait(&sh.a_empty[s], ((it / STAGES) - 1) & 1, abort);
-                        const uint4 cw = *reinterpret_cast<const uint4 *>(wrow + (((q * 2 + h) ^ (r & 7)) * 16));
-                        const uint32_t sw = sc[q] >> (16 * h);
-                        const float s0 = e4m3_to_f32(sw & 0xFFu), s1 = e4m3_to_f32((sw >> 8) & 0xFFu);
-                        uint8_t *arow = sh.a[s] + r * 128;
-                        const uint32_t cws[4] = {cw.x, cw.y, cw.z, cw.w};
+                for (int q = 0; q < KQ; q += 2) {
+                    const int nq = min(2, KT - (kw + q));
+                    if (nq <= 0) break;
 #pragma unroll
-                        for (int cc = 0; cc < 4; cc++) {
-                            const uint4 o = valid ? dequant8(cws[cc], cc < 2 ? s0 : s1) : make_uint4(0, 0, 0, 0);
-                            const int chunk = (h * 4 + cc) ^ (r & 7);
-                            *reinterpret_cast<uint4 *>(arow + chunk * 16) = o;
+                    for (int j = 0; j < 2; j++) {
+                        if (j < nq) {
+                            const int s = (it + j) % STAGES;
+                            if (it + j >= STAGES) mbar_wait(&sh.a_empty[s], (((it + j) / STAGES) - 1) & 1, abort);
+                            const uint4 cw = *reinterpret_cast<const uint4 *>(wrow + ((((q + j) * 2 + h) ^ (r & 7)) * 16));
+                            const uint32_t sw = sc[q + j] >> (16 * h);
+                            uint8_t *arow = sh.a[s] + r * 128;
+                            const uint32_t cws[4] = {cw.x, cw.y, cw.z, cw.w};
+                            if (f16) {
+                                const uint32_t s01 = e4m3x2_to_f16x2(sw & 0xFFFFu);
+                                const uint32_t s0 = __byte_perm(s01, 0, 0x1010), s1 = __byte_perm(s01, 0, 0x3232);
+#pragma unroll
+                                for (int cc = 0; cc < 4; cc++) {
+                                    const uint4 o =
+                                        valid ? dequant8_f16(cws[cc], cc < 2 ? s0 : s1) : make_uint4(0, 0, 0, 0);
+                                    const int chunk = (h * 4 + cc) ^ (r & 7);
+                                    *reinterpret_cast<uint4 *>(arow + chunk * 16) = o;
+                                }
+                            } else {
+                                const float s0 = e4m3_to_f32(sw & 0xFFu), s1 = e4m3_to_f32((sw >> 8) & 0xFFu);
+#pragma unroll
+                                for (int cc = 0; cc < 4; cc++) {
+                                    const uint4 o = valid ? dequant8(cws[cc], cc < 2 ? s0 : s1) : make_uint4(0, 0, 0, 0);
+                                    const int chunk = (h * 4 + cc) ^ (r & 7);
+                                    *reinterpret_cast<uint4 *>(arow + chunk * 16) = o;
+                                }
+                            }
                         }
-                        // each thread makes its stores visible to the tensor core's
-                        // (async) proxy; the warp then arrives once
-                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&sh.a_full[s]);
-                        it++;
                     }
+                    // each thread makes its stores visible to the tensor core's (async)
+                    // proxy; the warp then arrives once per stage
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0)
+                        for (int j = 0; j < nq; j++) mbar_arrive(&sh.a_full[(it + j) % STAGES]);
+                    it += nq;
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sh.w_empty[ws]);
@@ -315,12 +448,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
 
 // ---------------------------------------------------------------- host side --
 
-inline size_t gemm_workspace_bytes(const w4_weights *, int) { return 0; }
+// Workspace of the GEMM: x in f16 [M][K] (16-byte aligned), then sigma [M] and
+// bad [M] (int32).  Without it every tile runs on BF16 operands.
+inline size_t gemm_workspace_bytes(const w4_weights *w, int M) {
+    if (!w || M < 1) return 0;
+    return (((size_t)M * w->K * 2 + 15) & ~(size_t)15) + (((size_t)M * 8 + 15) & ~(size_t)15);
+}
 
 inline size_t gemm_smem_bytes() { return sizeof(gemm::SharedStorage) + 1024; }
 
-inline w4_status gemm_launch(const w4_weights *w, const void *x, int M, float *y32, void *y16, void *, size_t,
-                             cudaStream_t st) {
+inline w4_status gemm_launch(const w4_weights *w, const void *x, int M, float *y32, void *y16, void *ws,
+                             size_t ws_bytes, cudaStream_t st) {
     using namespace gemm;
     if (w->fmt != W4_FMT_NVFP4) return W4_ERR_UNSUPPORTED;
     const int K = w->K, N = w->N;
@@ -335,6 +473,18 @@ inline w4_status gemm_launch(const w4_weights *w, const void *x, int M, float *y
     if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return W4_ERR_CUDA;
+    // f16 copy of x in the workspace (when there is room for it)
+    const bool f16 = ws && ws_bytes >= gemm_workspace_bytes(w, M);
+    uint16_t *xh = reinterpret_cast<uint16_t *>(ws);
+    int *sigma = f16 ? reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(ws) +
+                                               (((size_t)M * K * 2 + 15) & ~(size_t)15))
+                     : nullptr;
+    int *bad = f16 ? sigma + M : nullptr;
+    CUtensorMap map16 = map;
+    if (f16 && enc(&map16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xh, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return W4_ERR_CUDA;
     CUtensorMap cmap;
     const cuuint64_t cdims[2] = {(cuuint64_t)K / 2, (cuuint64_t)N};
@@ -365,8 +515,11 @@ inline w4_status gemm_launch(const w4_weights *w, const void *x, int M, float *y
     p.K = K;
     p.tiles_m = (M + BN - 1) / BN;
     p.tiles_n = (N + BM - 1) / BM;
+    p.bad = bad;
+    p.sigma = sigma;
+    if (f16) x_to_f16_kernel<<<M, 256, 0, st>>>(reinterpret_cast<const uint16_t *>(x), xh, sigma, bad, K);
     const int ntiles = p.tiles_m * p.tiles_n;
-    gemm_kernel<<<std::min(ntiles, sms), kThreads, smem, st>>>(map, cmap, p);
+    gemm_kernel<<<std::min(ntiles, sms), kThreads, smem, st>>>(map, map16, cmap, p);
     return cudaGetLastError() == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
 

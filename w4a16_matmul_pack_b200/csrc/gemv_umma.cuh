@@ -22,7 +22,7 @@
 // 32 lanes read 256 contiguous code bytes per step (one 8-byte load each) and
 // 32 contiguous scale bytes.
 //
-// Roles (14 warps):
+// Roles (15 warps):
 //   warps 0-7   decode: the CTA's tiles form one sequence of MMA steps, grouped
 //               four to an A slot; warp w writes row w%4, steps {2h, 2h+1}
 //               (h = w/4) of each slot: LDS.64 codes -> cvt e2m1x2 -> HMUL2 by
@@ -30,7 +30,10 @@
 //               next slot is decoded while the previous store completes.  They
 //               also convert x, once the A ring is full (so decoding of the
 //               prefetched weights overlaps the wait for x).
-//   warp 8      allocates TMEM; lane 0 issues the MMAs and commits.
+//   warp 8      allocates TMEM; lane 0 issues the MMAs and commits.  It never
+//               waits on an mbarrier (a thread with MMAs queued stalls on any
+//               shared-memory access until they drain): warp 14 waits and
+//               releases it through a named barrier once per A slot.
 //   warp 9      lane 0: TMA producer (x after the dependency wait, weight
 //               stages of TB tiles, prefetched before the wait under PDL).
 //   warps 10-13 epilogue: row w%4 of each tile (tcgen05.ld of D, diagonal,
@@ -51,7 +54,8 @@ constexpr int kDecWarps = 8;
 constexpr int kMmaWarp = 8;
 constexpr int kProdWarp = 9;
 constexpr int kEpiWarp0 = 10;
-constexpr int kThreads = 14 * 32;
+constexpr int kWaitWarp = 14;   // waits on mbarriers for the MMA issuer
+constexpr int kThreads = 15 * 32;
 constexpr int kSlots = 6;              // A ring slots of 4 steps (32 columns)
 constexpr int kSlotSteps = 4;
 constexpr uint32_t kTmemCols = 256;
@@ -354,32 +358,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // ------------------------------ MMA issuer ------------------------------
-        if (lane == 0) {
-            mbar_wait(xready, 0, abort);
-            if (flags[1] == 0 && total > 0) {
-                const uint32_t xb_addr = smem_addr(xb);
-                for (int g = 0; g < nslots; g++) {
-                    const int slot = g % kSlots;
-                    mbar_wait(a_full + slot, (g / kSlots) & 1, abort);
-                    fence_after();
+        // A thread with MMAs queued stalls on any shared-memory access (an mbarrier
+        // wait included) until they drain.  So this warp never waits on an
+        // mbarrier: warp kWaitWarp does, and meets it at named barrier 2 once per
+        // A slot (after x is converted, and before each slot).
+        named_barrier_sync(2, 64);
+        const bool run = flags[1] == 0 && total > 0;   // read before any MMA is queued
+        if (run) {
+            const uint32_t xb_addr = smem_addr(xb);
+            for (int g = 0; g < nslots; g++) {
+                const int slot = g % kSlots;
+                named_barrier_sync(2, 64);   // slot g written; the accumulators it starts are free
+                fence_after();
+                if (lane == 0) {
                     const int G1 = min(total, (g + 1) * kSlotSteps);
                     for (int G = g * kSlotSteps; G < G1; G++) {
                         const int t = G / steps, s = G - t * steps, db = t & 1;
-                        if (s == 0 && t >= 2) {
-                            mbar_wait(d_empty + db, ((t >> 1) - 1) & 1, abort);
-                            fence_after();
-                        }
                         mma_ts(tmem + kDCol0 + 32u * db, tmem + 32u * slot + 8u * (G - g * kSlotSteps),
                                b_desc(xb_addr + 1024u * s), s > 0 ? 1u : 0u);
                         if (s == steps - 1) mma_commit(d_full + db);
                     }
                     mma_commit(a_empty + slot);
                 }
-                // the last products must be complete before tensor memory is released
-                mbar_wait_bounded(d_full + ((ntiles - 1) & 1), ((ntiles - 1) >> 1) & 1);
+                __syncwarp();
+            }
+            // the last products must be complete before tensor memory is released
+            mbar_wait_bounded(d_full + ((ntiles - 1) & 1), ((ntiles - 1) >> 1) & 1);
+        }
+    } else if (warp == kWaitWarp) {
+        // ---------------------- waits on behalf of the MMA issuer ----------------------
+        mbar_wait(xready, 0, abort);
+        named_barrier_sync(2, 64);
+        if (flags[1] == 0 && total > 0) {
+            for (int g = 0; g < nslots; g++) {
+                const int slot = g % kSlots;
+                mbar_wait(a_full + slot, (g / kSlots) & 1, abort);
+                const int G1 = min(total, (g + 1) * kSlotSteps);
+                for (int G = g * kSlotSteps; G < G1; G++) {
+                    const int t = G / steps, s = G - t * steps;
+                    if (s == 0 && t >= 2) mbar_wait(d_empty + (t & 1), ((t >> 1) - 1) & 1, abort);
+                }
+                named_barrier_sync(2, 64);
             }
         }
-        __syncwarp();   // the whole warp reaches the final barrier together (it is .aligned)
     } else if (warp < kDecWarps) {
         // ------------------------------ decode warps ------------------------------
         const int q = warp & 3, h = warp >> 2;
