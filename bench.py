@@ -496,8 +496,11 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
-# ncu-measured DRAM bytes per launch of the dominant kernel (profiles/), or None
-TRAFFIC_PER_LAUNCH = None
+# ncu-measured DRAM bytes (read + write) per launch of the dominant kernel,
+# w4::gemv_nvfp4_m1_kernel, averaged over its launches in
+# `bench.py --steps 3 --warmup 3 --no-extras` (profiles/launches_bench_decode_sweep_m1.md).
+# Set to None when that kernel changes until it is measured again.
+TRAFFIC_PER_LAUNCH = 8307220
 
 
 def main():

@@ -2,39 +2,49 @@
 //
 // y[m][n] = g * sum_k x[m][k] * (e2m1[n][k] * scale[n][k/16])   (NVFP4 weights,
 // "EdgeRock-4B-NVFP4" card, intro; BF16 activations).  e2m1 * scale has at most
-// 6 significant bits and lies in [2^-10, 2688], so it is exact in BF16: the
-// weights are dequantised once per tile into shared memory and multiplied with
-// tcgen05.mma kind::f16 (BF16 x BF16 -> FP32 in tensor memory).  The global
-// scale g is applied in the epilogue.
+// 6 significant bits and lies in [2^-10, 2688], so it is exact in BF16 and in
+// f16: the dequant warps write it, per 64-k stage, into tensor memory, where it
+// is the A operand of tcgen05.mma kind::f16 (A from TMEM, B = x from shared
+// memory, FP32 accumulators in TMEM).  The global scale g is applied in the
+// epilogue.
 //
-// Tile: 128 weight rows (MMA M, operand A = dequantised W) x 256 tokens (MMA N,
-// operand B = x) x 64 k per stage; both operands K-major with the 128-byte
-// swizzle.  Persistent CTAs, one per SM, walk the tiles n-major so that CTAs
-// running together share the same packed weight rows in L2.
+// Tile: 128 weight rows (MMA M, A) x 192 tokens (MMA N, B = x, K-major with the
+// 128-byte swizzle, staged by TMA) x 64 k per stage.  Tensor memory holds four
+// A stages (32 columns each) and two 192-column accumulators (512 columns), so
+// the epilogue of a tile overlaps the MMAs of the next.  Persistent CTAs, one
+// per SM, walk the tiles n-major so that CTAs running together share the same
+// packed weight rows in L2.
 //
 // Warp roles (15 warps):
-//   warp 0      TMA producer of x tiles (cp.async.bulk.tensor, no multicast);
-//               allocates / frees the 512 TMEM columns.
-//   warp 1      MMA issuer (one thread): 4 x (128x256x16) per stage, commits to
-//               the stage barriers, and to the accumulator barrier per tile.
-//               It never waits on an mbarrier itself (see below): warp 14 does,
-//               and releases it through named barrier 2 once per stage.
+//   warp 0      TMA producer: x tiles and the packed codes (128-byte swizzle,
+//               256 k per codes stage), no multicast.
+//   warp 1      allocates / frees the 512 TMEM columns; MMA issuer (one lane):
+//               4 x (128x192x16) per stage, commits to the stage barriers and
+//               to the accumulator barrier per tile.  It never waits on an
+//               mbarrier: a thread with MMAs queued stalls on any shared-memory
+//               access until they drain (measured: one wait per four
+//               128x256x16 MMAs turns 128 cycles per MMA into 270), so warp 14
+//               waits and releases it through named barrier 2 once per stage.
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
-//               32*(w%4)..+31), times g, float32 / BF16 stores.
-//   warps 6-13  dequantise: thread (row r, half h) turns 32 codes + 2 scales of
-//               row r into BF16 in the swizzled A stage.
-// Two accumulators of 256 columns let the epilogue of a tile overlap the MMAs
-// of the next.  Every mbarrier wait is bounded (common.cuh: mbar_wait).
+//               32*(w%4)..+31), times g (and 2^sigma_m, below), float32 / BF16
+//               stores.
+//   warps 6-13  dequantise: warp w owns TMEM lanes 32*(w%4)..+31 = weight rows;
+//               thread (row r, k-half h) turns 32 codes + 2 scales of row r into
+//               16 words and stores them with one tcgen05.st, two stages per
+//               round (one store wait and one arrival per round).
+//   warp 14     waits on the x / A stage barriers and the accumulator barriers
+//               for the MMA issuer.
+// Every mbarrier wait is bounded (common.cuh: mbar_wait).
 //
-// Operand precision per tile of 256 tokens.  e2m1 * scale is exact in f16 as
-// well as in BF16, and in f16 it costs one cvt (E2M1 -> f16x2) and one HMUL2
-// per pair of weights instead of a round trip through binary32.  So when the
-// caller provides a workspace, x_to_f16_kernel first converts each token row to
-// f16 as x * 2^-sigma_m (sigma_m from the row's largest |x|) and flags the rows
-// it cannot convert exactly (a nonzero |x * 2^-sigma_m| below 2^-17, or Inf /
-// NaN).  A tile whose 256 rows all converted exactly runs kind::f16 with f16
-// operands and the epilogue multiplies token m by 2^sigma_m; any other tile (or
-// every tile, without a workspace) runs the BF16 operands described above.
+// Operand precision per tile of 192 tokens.  In f16, e2m1 * scale costs one cvt
+// (E2M1 -> f16x2) and one HMUL2 per pair of weights instead of a round trip
+// through binary32.  So when the caller provides a workspace, x_to_f16_kernel
+// first converts each token row to f16 as x * 2^-sigma_m (sigma_m from the
+// row's largest |x|) and flags the rows it cannot convert exactly (a nonzero
+// |x * 2^-sigma_m| below 2^-17, or Inf / NaN).  A tile whose rows all converted
+// exactly runs kind::f16 with f16 operands and the epilogue multiplies token m
+// by 2^sigma_m; any other tile (or every tile, without a workspace) runs on
+// BF16 operands (e2m1 -> f16 -> binary32 * scale -> BF16).
 #pragma once
 
 #include "common.cuh"
@@ -44,18 +54,18 @@ namespace w4 {
 namespace gemm {
 
 constexpr int BM = 128;      // weight rows per tile (MMA M)
-constexpr int BN = 256;      // tokens per tile (MMA N)
+constexpr int BN = 192;      // tokens per tile (MMA N)
 constexpr int BK = 64;       // k per stage (one 128-byte swizzle row of BF16)
 constexpr int STAGES = 4;
 constexpr int kWarps = 15;
 constexpr int kThreads = kWarps * 32;
 constexpr int kDequantThreads = 256;
 constexpr int kEpiThreads = 128;
-constexpr uint32_t X_STAGE_BYTES = BN * BK * 2;   // 32 KB
-constexpr uint32_t A_STAGE_BYTES = BM * BK * 2;   // 16 KB
-constexpr uint32_t TMEM_COLS = 512;               // two 256-column fp32 accumulators
+constexpr uint32_t X_STAGE_BYTES = BN * BK * 2;   // 24 KB
+constexpr uint32_t TMEM_COLS = 512;               // 4 A stages (32 columns each) + two 192-column accumulators
+constexpr uint32_t ACC_COL0 = STAGES * (BK / 2);  // accumulators after the A stages
 constexpr int WK = 256;                           // k per packed-weight stage (4 k-steps)
-constexpr int WSTAGES = 2;
+constexpr int WSTAGES = 4;
 constexpr uint32_t W_STAGE_BYTES = BM * WK / 2;   // 16 KB of codes (128 rows x 128 bytes)
 
 // Instruction descriptor, kind::f16: D = F32 (bit 4), A = BF16 (bits 7-9),
@@ -69,7 +79,6 @@ constexpr int kWaitWarp = 14;     // waits on mbarriers for the MMA issuer (warp
 
 struct SharedStorage {
     uint8_t x[STAGES][X_STAGE_BYTES];   // 1024-byte aligned (swizzle atoms)
-    uint8_t a[STAGES][A_STAGE_BYTES];
     uint8_t w[WSTAGES][W_STAGE_BYTES];  // packed codes, 128-byte swizzle
     uint64_t w_full[WSTAGES], w_empty[WSTAGES];
     uint64_t x_full[STAGES], x_empty[STAGES];
@@ -101,6 +110,31 @@ __device__ __forceinline__ void mma_f16kind(uint32_t tmem_d, uint64_t adesc, uin
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
         ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+
+// The same with A from tensor memory (K-major: lane = row, 32-bit column = two k).
+__device__ __forceinline__ void mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(tmem_d), "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
 }
 
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
@@ -291,17 +325,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         int it = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
             const int b = ((t - blockIdx.x) / gridDim.x) & 1;
-            const uint32_t dtm = tmem + (uint32_t)(b * BN);
+            const uint32_t dtm = tmem + ACC_COL0 + (uint32_t)(b * BN);
             const uint32_t idesc = sh.f16_tile[t % p.tiles_m] ? IDESC_F16 : IDESC;
             for (int kt = 0; kt < KT; kt++, it++) {
                 const int s = it % STAGES;
                 named_barrier_sync(2, 64);   // stage s (and, at kt == 0, accumulator b) is ready
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t ab = smem_addr(sh.a[s]), xb = smem_addr(sh.x[s]);
+                    const uint32_t xb = smem_addr(sh.x[s]);
 #pragma unroll
-                    for (int j = 0; j < BK / 16; j++)
-                        mma_f16kind(dtm, sw128_desc(ab + 32 * j), sw128_desc(xb + 32 * j), idesc, (kt | j) ? 1u : 0u);
+                    for (int j = 0; j < BK / 16; j++)   // A (16 k = 8 columns) from tensor memory
+                        mma_ts(dtm, tmem + (uint32_t)(s * (BK / 2) + 8 * j), sw128_desc(xb + 32 * j), idesc,
+                               (kt | j) ? 1u : 0u);
                     mma_commit(&sh.x_empty[s]);
                     mma_commit(&sh.a_empty[s]);
                     if (kt == KT - 1) mma_commit(&sh.acc_full[b]);
@@ -338,7 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             const bool f16 = sh.f16_tile[t % p.tiles_m] != 0;
             for (int c = 0; c < BN / 32; c++) {
                 uint32_t v[32];
-                W4_TMEM_LD32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * BN + c * 32), v);
+                W4_TMEM_LD32(tmem + ((uint32_t)(q * 32) << 16) + ACC_COL0 + (uint32_t)(b * BN + c * 32), v);
                 asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
                 // f16 tiles: token m was scaled by 2^-sigma_m (lane j holds sigma of token c*32+j)
                 const int mlane = m0 + c * 32 + lane;
@@ -365,8 +400,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         // thread (row r, half h): 32 codes of row r per k-step from the swizzled
         // codes stage (conflict-free: 8 consecutive rows read 8 distinct 16-byte
         // chunks), 2 scales from a register ring filled one codes stage ahead.
-        const int dt = threadIdx.x - 6 * 32;    // 0..255
-        const int r = dt & (BM - 1), h = dt >> 7;
+        // warp w writes TMEM lanes 32*(w%4) .. +31 (the lanes it may access): row r,
+        // k-half h of each 64-k stage
+        const int r = 32 * (warp & 3) + lane, h = (warp - 6) >> 2;
+        const uint32_t a_lane = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
         constexpr int KQ = WK / BK;             // k-steps per codes stage
         int it = 0, wit = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
@@ -390,39 +427,46 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                 for (int q = 0; q < KQ; q += 2) {
                     const int nq = min(2, KT - (kw + q));
                     if (nq <= 0) break;
+                    // both A stages free first, then both loads, both decodes and both
+                    // stores, so that the two k-steps overlap in this warp
+#pragma unroll
+                    for (int j = 0; j < 2; j++)
+                        if (j < nq && it + j >= STAGES)
+                            mbar_wait(&sh.a_empty[(it + j) % STAGES], (((it + j) / STAGES) - 1) & 1, abort);
+                    tc_fence_after();
+                    uint4 cw[2];
+#pragma unroll
+                    for (int j = 0; j < 2; j++)
+                        cw[j] = ld_shared_v4(smem_addr(wrow + ((((q + j) * 2 + h) ^ (r & 7)) * 16)));
+                    uint32_t av[2][16];
 #pragma unroll
                     for (int j = 0; j < 2; j++) {
-                        if (j < nq) {
-                            const int s = (it + j) % STAGES;
-                            if (it + j >= STAGES) mbar_wait(&sh.a_empty[s], (((it + j) / STAGES) - 1) & 1, abort);
-                            const uint4 cw = *reinterpret_cast<const uint4 *>(wrow + ((((q + j) * 2 + h) ^ (r & 7)) * 16));
-                            const uint32_t sw = sc[q + j] >> (16 * h);
-                            uint8_t *arow = sh.a[s] + r * 128;
-                            const uint32_t cws[4] = {cw.x, cw.y, cw.z, cw.w};
-                            if (f16) {
-                                const uint32_t s01 = e4m3x2_to_f16x2(sw & 0xFFFFu);
-                                const uint32_t s0 = __byte_perm(s01, 0, 0x1010), s1 = __byte_perm(s01, 0, 0x3232);
+                        const uint32_t sw = sc[q + j] >> (16 * h);
+                        const uint32_t cws[4] = {cw[j].x, cw[j].y, cw[j].z, cw[j].w};
+                        if (f16) {
+                            const uint32_t s01 = e4m3x2_to_f16x2(sw & 0xFFFFu);
+                            const uint32_t s0 = __byte_perm(s01, 0, 0x1010), s1 = __byte_perm(s01, 0, 0x3232);
 #pragma unroll
-                                for (int cc = 0; cc < 4; cc++) {
-                                    const uint4 o =
-                                        valid ? dequant8_f16(cws[cc], cc < 2 ? s0 : s1) : make_uint4(0, 0, 0, 0);
-                                    const int chunk = (h * 4 + cc) ^ (r & 7);
-                                    *reinterpret_cast<uint4 *>(arow + chunk * 16) = o;
-                                }
-                            } else {
-                                const float s0 = e4m3_to_f32(sw & 0xFFu), s1 = e4m3_to_f32((sw >> 8) & 0xFFu);
+                            for (int cc = 0; cc < 4; cc++) {
+                                const uint4 o = valid ? dequant8_f16(cws[cc], cc < 2 ? s0 : s1) : make_uint4(0, 0, 0, 0);
+                                av[j][4 * cc] = o.x, av[j][4 * cc + 1] = o.y, av[j][4 * cc + 2] = o.z, av[j][4 * cc + 3] = o.w;
+                            }
+                        } else {
+                            const float s0 = e4m3_to_f32(sw & 0xFFu), s1 = e4m3_to_f32((sw >> 8) & 0xFFu);
 #pragma unroll
-                                for (int cc = 0; cc < 4; cc++) {
-                                    const uint4 o = valid ? dequant8(cws[cc], cc < 2 ? s0 : s1) : make_uint4(0, 0, 0, 0);
-                                    const int chunk = (h * 4 + cc) ^ (r & 7);
-                                    *reinterpret_cast<uint4 *>(arow + chunk * 16) = o;
-                                }
+                            for (int cc = 0; cc < 4; cc++) {
+                                const uint4 o = valid ? dequant8(cws[cc], cc < 2 ? s0 : s1) : make_uint4(0, 0, 0, 0);
+                                av[j][4 * cc] = o.x, av[j][4 * cc + 1] = o.y, av[j][4 * cc + 2] = o.z, av[j][4 * cc + 3] = o.w;
                             }
                         }
                     }
-                    // each thread makes its stores visible to the tensor core's (async)
-                    // proxy; the warp then arrives once per stage
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    // 32 k of row r: columns 16h .. 16h+15 of A stage s
+#pragma unroll
+                    for (int j = 0; j < 2; j++)
+                        if (j < nq) tmem_st16(a_lane + (uint32_t)(((it + j) % STAGES) * (BK / 2) + 16 * h), av[j]);
+                    // the stores complete, then one arrival per warp and stage
+                    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                    tc_fence_before();
                     __syncwarp();
                     if (lane == 0)
                         for (int j = 0; j < nq; j++) mbar_arrive(&sh.a_full[(it + j) % STAGES]);
