@@ -172,6 +172,26 @@ w4_status w4a16_gemv_ex(const w4_weights *w, const void *x, int M, float *y,
                         void *stream);
 
 /*
+ * w4a16_gemv_grouped -- G independent one-token NVFP4 GEMVs in one launch:
+ * y[p][N_p] = x[p][K_p] . w_hat[p] for p < G (the decode GEMV of the
+ * "Nanbeige4.2-3B-NVFP4A16" card, Serving, applied to several weight matrices
+ * that are ready together: the q, k and v projections of a layer read the same
+ * x, as do gate and up).  The SMs are shared out in proportion to each
+ * problem's packed bytes, so small matrices do not each pay a launch and a
+ * pipeline fill.
+ *   w      array of G NVFP4 weights (K_p % 256 == 0, K_p <= 32768).
+ *   x      array of G device pointers to [K_p] BF16 (may repeat).
+ *   y      array of G device pointers to [N_p] float (must not overlap).
+ *   G      1..8.
+ *   flags  0 or W4_LAUNCH_PDL.
+ * The arrays are read on the host before the call returns; no workspace.
+ * Errors: W4_ERR_ARG (null pointers, G out of range, unknown flags),
+ * W4_ERR_ALIGN, W4_ERR_UNSUPPORTED (format or K), W4_ERR_CUDA.
+ */
+w4_status w4a16_gemv_grouped(const w4_weights *w, const void *const *x, float *const *y, int G,
+                             unsigned flags, void *stream);
+
+/*
  * w4a16_gemm -- y = x . w_hat for prefill-sized M: NVFP4 tiles are dequantised
  * to BF16 in shared memory (e2m1 * scale, exact in BF16) and multiplied on the
  * tensor cores with binary32 accumulation; the epilogue multiplies by the

@@ -231,3 +231,73 @@ def test_tensor_memory_path_ranges(case):
         assert_within_tolerance(y[fin], yr[fin], ar[fin])
     else:
         assert_within_tolerance(y, yr, ar)
+
+
+def check_group(pws, whs, xs, flags=0):
+    ys = W4.w4a16_gemv_grouped(pws, [x.cuda() for x in xs], flags=flags)
+    for y, wh, x in zip(ys, whs, xs):
+        yr, ar = O.matmul(x, wh)
+        assert_within_tolerance(np_of(y), yr, ar)
+    return ys
+
+
+def test_grouped_sweep():
+    """The five sweep matrices, each with its own x, in one launch."""
+    pws, whs, xs = [], [], []
+    for idx, (K, N) in enumerate(I.SWEEP_SHAPES):
+        pw, wh = nvfp4_packed(I.sweep_weights(K, N, idx))
+        pws.append(pw); whs.append(wh); xs.append(I.sweep_x(1, K, idx))
+    check_group(pws, whs, xs)
+    check_group(pws, whs, xs, flags=W4.LAUNCH_PDL)
+
+
+def test_grouped_shared_x_and_ragged():
+    """q, k, v reading one x; then ragged shapes (1 row, fewer rows than CTAs, K = 256)."""
+    K = 2560
+    mats = [nvfp4_packed(I.sweep_weights(K, N, 30 + i)[:N].contiguous()) for i, N in enumerate((4096, 1024, 1024))]
+    x = I.activations(1, K, 31)
+    check_group([m[0] for m in mats], [m[1] for m in mats], [x, x, x])
+    shapes = [(256, 7), (1024, 149), (2560, 333), (9728, 2), (512, 1), (4096, 4096)]
+    pws, whs, xs = [], [], []
+    for i, (K, N) in enumerate(shapes):
+        pw, wh = nvfp4_packed(I.sweep_weights(K, N, 40 + i)[:N].contiguous())
+        pws.append(pw); whs.append(wh); xs.append(I.activations(1, K, 50 + i))
+    check_group(pws, whs, xs)
+
+
+def test_grouped_eight_and_graph():
+    """The largest group; replayed in a CUDA graph with PDL it gives the same bits."""
+    shapes = [(2560, 1024)] * 4 + [(4096, 512)] * 2 + [(1024, 2048), (9728, 256)]
+    pws, whs, xs = [], [], []
+    for i, (K, N) in enumerate(shapes):
+        pw, wh = nvfp4_packed(I.sweep_weights(K, N, 60 + i)[:N].contiguous())
+        pws.append(pw); whs.append(wh); xs.append(I.activations(1, K, 70 + i))
+    ref = [y.clone() for y in check_group(pws, whs, xs)]
+    xd = [x.cuda() for x in xs]
+    outs = [torch.empty(1, w.N, device="cuda") for w in pws]
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        W4.w4a16_gemv_grouped(pws, xd, outs=outs, flags=W4.LAUNCH_PDL)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        W4.w4a16_gemv_grouped(pws, xd, outs=outs, flags=W4.LAUNCH_PDL)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    for a, b in zip(ref, outs):
+        assert torch.equal(a, b)
+
+
+def test_grouped_argument_errors():
+    pw, _ = nvfp4_packed(I.sweep_weights(256, 16, 80)[:16].contiguous())
+    x = I.activations(1, 256, 81).cuda()
+    with pytest.raises(W4.W4Error):
+        W4.w4a16_gemv_grouped([pw] * 9, [x] * 9)
+    with pytest.raises(W4.W4Error):
+        W4.w4a16_gemv_grouped([pw], [x], flags=W4.LAUNCH_TMEM)
+    pr = W4.pack_rocmfp4(I.matrix("laplace", 16, 256, 82, 0.015, 0.0, device="cuda"), "dual")
+    with pytest.raises(W4.W4Error):
+        W4.w4a16_gemv_grouped([pr], [x])

@@ -24,7 +24,7 @@ import torch
 
 __all__ = [
     "W4Error", "PackedWeights", "FMT_NVFP4", "FMT_ROCMFP4_DUAL", "FMT_ROCMFP4_FAST",
-    "LAUNCH_PDL", "LAUNCH_TMEM", "pack_nvfp4", "pack_rocmfp4", "w4a16_gemv", "w4a16_gemm",
+    "LAUNCH_PDL", "LAUNCH_TMEM", "pack_nvfp4", "pack_rocmfp4", "w4a16_gemv", "w4a16_gemv_grouped", "w4a16_gemm",
     "w4a16_workspace_bytes", "pack_nvfp4_workspace_bytes", "w4_encode_scalars",
     "w4_device_error", "lib", "library_path",
 ]
@@ -75,6 +75,7 @@ def lib():
             "pack_rocmfp4": ([P, I, I, I, I, P, P, P, P], I),
             "w4a16_gemv": ([WP, P, I, P, P, S, P], I),
             "w4a16_gemv_ex": ([WP, P, I, P, P, S, U, P], I),
+            "w4a16_gemv_grouped": ([WP, P, P, I, U, P], I),
             "w4a16_gemm": ([WP, P, I, P, P, P, S, P], I),
             "w4a16_workspace_bytes": ([WP, I], S),
             "w4_encode_scalars": ([P, S, P, P, P], I),
@@ -196,6 +197,23 @@ def w4a16_gemv(w: PackedWeights, x: torch.Tensor, *, out: Optional[torch.Tensor]
                                0 if workspace is None else workspace.numel(), flags, _stream(stream)),
            "w4a16_gemv")
     return out
+
+
+def w4a16_gemv_grouped(ws, xs, *, outs=None, flags: int = 0, stream=None):
+    """Several one-token NVFP4 GEMVs in one launch: returns [y_p[1][N_p] float32]."""
+    G = len(ws)
+    if len(xs) != G or (outs is not None and len(outs) != G):
+        raise W4Error(-1, "w4a16_gemv_grouped: ws, xs and outs must have the same length")
+    for x in xs:
+        _cuda(x, "x", torch.bfloat16)
+    if outs is None:
+        outs = [torch.empty(1, w.N, dtype=torch.float32, device=xs[0].device) for w in ws]
+    structs = (_Weights * G)(*[w.struct() for w in ws])
+    xp = (ctypes.c_void_p * G)(*[_ptr(x) for x in xs])
+    yp = (ctypes.c_void_p * G)(*[_ptr(y) for y in outs])
+    _check(lib().w4a16_gemv_grouped(structs, ctypes.cast(xp, ctypes.c_void_p), ctypes.cast(yp, ctypes.c_void_p), G,
+                                    flags, _stream(stream)), "w4a16_gemv_grouped")
+    return outs
 
 
 def w4a16_gemm(w: PackedWeights, x: torch.Tensor, *, want_f32: bool = True, want_bf16: bool = True,

@@ -88,12 +88,13 @@ __device__ __forceinline__ void decode_codes32(uint4 c, uint32_t (&h)[16]) {
 __device__ __forceinline__ float e4m3_lo_scaled(uint32_t v) { return __uint_as_float((v << 20) & 0x07F00000u); }
 __device__ __forceinline__ float e4m3_hi_scaled(uint32_t v) { return __uint_as_float((v << 12) & 0x07F00000u); }
 
-__global__ void __launch_bounds__(kTcThreads, 1)
-    gemv_nvfp4_m1_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant__ CUtensorMap smap,
-                         const GemvTcArgs a) {
+// The kernel body for one CTA: CTA `cta` of `ncta` working on rows of one
+// problem, K-slice `slice` of `nslices` (split-K partials when nslices > 1).
+__device__ __forceinline__ void m1_body(const CUtensorMap &cmap, const CUtensorMap &smap, const GemvTcArgs &a,
+                                        int cta, int ncta, int slice, int nslices) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int K = a.K, N = a.N, kc = a.kc, KP = a.KP, NS = a.NS;
-    const int slice = blockIdx.y, k0 = slice * kc, kcs = min(kc, K - k0);
+    const int k0 = slice * kc, kcs = min(kc, K - k0);
     const int npieces = (kcs + KP - 1) / KP;
     const int CS = KP / 2, SS = KP / 16;
     const M1Layout L = m1_layout(a.xstride, kc, NS, a.tile_bytes, a.red_tiles);
@@ -111,10 +112,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     long long r0, r1;
     if (a.rows_mode == 0) {
-        r0 = (long long)blockIdx.x * N / gridDim.x;
-        r1 = (long long)(blockIdx.x + 1) * N / gridDim.x;
+        r0 = (long long)cta * N / ncta;
+        r1 = (long long)(cta + 1) * N / ncta;
     } else {
-        r0 = (long long)blockIdx.x * a.tiles_per_cta * kTcRows;
+        r0 = (long long)cta * a.tiles_per_cta * kTcRows;
         r1 = min((long long)N, r0 + (long long)a.tiles_per_cta * kTcRows);
     }
     const int ntiles = (int)((r1 - r0 + kTcRows - 1) / kTcRows);
@@ -315,7 +316,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 float s = 0.0f;
                 for (int q = 0; q < kTcParts; q++) s += rb[q * kTcRows + threadIdx.x];
                 const long long n = rt + threadIdx.x;
-                if (gridDim.y == 1)
+                if (nslices == 1)
                     a.y[n] = gs * s;
                 else
                     a.partial[(size_t)slice * N + n] = s;
@@ -331,12 +332,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const float *rb = red + (size_t)(i / kTcRows) * kTcParts * kTcRows + (i % kTcRows);
             float s = 0.0f;
             for (int q = 0; q < kTcParts; q++) s += rb[q * kTcRows];
-            if (gridDim.y == 1)
+            if (nslices == 1)
                 a.y[n] = gs * s;
             else
                 a.partial[(size_t)slice * N + n] = s;
         }
     }
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1)
+    gemv_nvfp4_m1_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant__ CUtensorMap smap,
+                         const GemvTcArgs a) {
+    m1_body(cmap, smap, a, blockIdx.x, gridDim.x, blockIdx.y, gridDim.y);
+}
+
+// Several independent one-token problems in one launch (e.g. the q, k and v
+// projections of a layer, or any set of GEMVs that are ready at the same time):
+// CTAs [cta0[p], cta0[p+1]) work on problem p, each on its own balanced range
+// of rows, exactly as a CTA of the single-problem kernel does.
+constexpr int kMaxGroup = 8;
+
+struct GroupArgs {
+    CUtensorMap cmap[kMaxGroup];
+    CUtensorMap smap[kMaxGroup];
+    GemvTcArgs a[kMaxGroup];
+    int cta0[kMaxGroup + 1];
+    int G;
+};
+
+__global__ void __launch_bounds__(kTcThreads, 1) gemv_nvfp4_m1_grouped_kernel(const __grid_constant__ GroupArgs g) {
+    int p = 0;
+    while (p + 1 < g.G && (int)blockIdx.x >= g.cta0[p + 1]) p++;
+    m1_body(g.cmap[p], g.smap[p], g.a[p], (int)blockIdx.x - g.cta0[p], g.cta0[p + 1] - g.cta0[p], 0, 1);
 }
 
 }  // namespace w4

@@ -172,7 +172,9 @@ constexpr double kSmBytesPerUs = 48e3;  // bytes per us one SM streams with a de
 constexpr double kHbmBytesPerUs = 7e6;  // whole-device streaming rate
 constexpr double kCopyUs = 0.2;         // cost of one bulk / tensor copy on an SM
 
-w4_status plan_gemv_tc(int K, int N, int M, bool pdl, GemvTcPlan &p) {
+// force_grid > 0: exactly that many CTAs, each on a balanced range of rows (the
+// grouped launch gives every problem its own share of the SMs).
+w4_status plan_gemv_tc(int K, int N, int M, bool pdl, GemvTcPlan &p, int force_grid = 0) {
     DeviceInfo d;
     if (device_info(d) != W4_OK) return W4_ERR_CUDA;
     const int unit = 256;
@@ -202,7 +204,13 @@ w4_status plan_gemv_tc(int K, int N, int M, bool pdl, GemvTcPlan &p) {
     const double costB = std::max(q * kTcRows * rowB / kSmBytesPerUs, (double)T * kTcRows * rowB / kHbmBytesPerUs) +
                          2 * q * p.S * kCopyUs;
     int tiles_max;
-    if (costB <= costA) {
+    if (force_grid > 0) {
+        p.rows_mode = 0;
+        p.tiles_per_cta = 0;
+        p.grid = std::min(force_grid, N);
+        const int rows = (N + p.grid - 1) / p.grid;
+        tiles_max = (rows + kTcRows - 1) / kTcRows + 1;
+    } else if (costB <= costA) {
         p.rows_mode = 1;
         p.tiles_per_cta = q;
         p.grid = gB;
@@ -231,21 +239,13 @@ w4_status plan_gemv_tc(int K, int N, int M, bool pdl, GemvTcPlan &p) {
     return W4_OK;
 }
 
-template <int M>
-w4_status launch_gemv_tc_m(const w4_weights *w, const void *x, float *y, void *ws, const GemvTcPlan &p, bool pdl,
-                           cudaStream_t st) {
-    // one token: block scales applied after the MMA (gemv_m1.cuh)
-    auto kern = M == 1 ? gemv_nvfp4_m1_kernel : gemv_nvfp4_tc_kernel<M>;
-    static size_t configured = 0;
-    if (p.smem > configured) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem) != cudaSuccess)
-            return W4_ERR_CUDA;
-        configured = p.smem;
-    }
+// Tensor maps of one NVFP4 matrix for the GEMV stages (16-row x KP-k boxes) and
+// the kernel arguments.
+w4_status gemv_tc_setup(const w4_weights *w, const void *x, float *y, void *ws, const GemvTcPlan &p, bool pdl,
+                        CUtensorMap &cmap, CUtensorMap &smap, GemvTcArgs &a) {
     PFN_encodeTiled enc = get_encode_tiled();
     if (!enc) return W4_ERR_CUDA;
     const int K = w->K, N = w->N;
-    CUtensorMap cmap, smap;
     const cuuint64_t cdims[2] = {(cuuint64_t)K / 16, (cuuint64_t)N};   // codes as 8-byte elements
     const cuuint64_t cstr[1] = {(cuuint64_t)K / 2};
     const cuuint32_t cbox[2] = {(cuuint32_t)p.KP / 16, (cuuint32_t)kTcRows};
@@ -260,7 +260,6 @@ w4_status launch_gemv_tc_m(const w4_weights *w, const void *x, float *y, void *w
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return W4_ERR_CUDA;
-    GemvTcArgs a;
     a.codes = w->codes;
     a.scales = w->scales;
     a.gscale = w->global_scale;
@@ -279,6 +278,25 @@ w4_status launch_gemv_tc_m(const w4_weights *w, const void *x, float *y, void *w
     a.box_min_rows = p.box_min_rows;
     a.red_tiles = p.red_tiles;
     a.pdl = pdl ? 1 : 0;
+    return W4_OK;
+}
+
+template <int M>
+w4_status launch_gemv_tc_m(const w4_weights *w, const void *x, float *y, void *ws, const GemvTcPlan &p, bool pdl,
+                           cudaStream_t st) {
+    // one token: block scales applied after the MMA (gemv_m1.cuh)
+    auto kern = M == 1 ? gemv_nvfp4_m1_kernel : gemv_nvfp4_tc_kernel<M>;
+    static size_t configured = 0;
+    if (p.smem > configured) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem) != cudaSuccess)
+            return W4_ERR_CUDA;
+        configured = p.smem;
+    }
+    const int N = w->N;
+    CUtensorMap cmap, smap;
+    GemvTcArgs a;
+    const w4_status s0 = gemv_tc_setup(w, x, y, ws, p, pdl, cmap, smap, a);
+    if (s0 != W4_OK) return s0;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.grid, p.S, 1);
     cfg.blockDim = dim3(kTcThreads, 1, 1);
@@ -294,6 +312,78 @@ w4_status launch_gemv_tc_m(const w4_weights *w, const void *x, float *y, void *w
         const int MN = M * N;
         gemv_finalize_kernel<<<std::min((MN + 255) / 256, 1024), 256, 0, st>>>(a.partial, p.S, MN, w->global_scale, y);
     }
+    return launch_status();
+}
+
+// Several one-token NVFP4 problems in one launch (gemv_m1.cuh): the SMs are
+// shared out in proportion to each problem's packed bytes (at least one CTA
+// each, at most one per 16-row tile), and every CTA runs the single-problem
+// kernel body on a balanced range of its problem's rows.
+w4_status launch_gemv_grouped(const w4_weights *w, const void *const *x, float *const *y, int G, bool pdl,
+                              cudaStream_t st) {
+    DeviceInfo d;
+    if (device_info(d) != W4_OK) return W4_ERR_CUDA;
+    double bytes[kMaxGroup], total = 0.0;
+    int tiles[kMaxGroup], alloc[kMaxGroup], sum = 0;
+    for (int p = 0; p < G; p++) {
+        bytes[p] = (double)w[p].N * (w[p].K / 2 + w[p].K / 16);
+        total += bytes[p];
+        tiles[p] = (w[p].N + kTcRows - 1) / kTcRows;
+    }
+    for (int p = 0; p < G; p++) {
+        alloc[p] = std::max(1, std::min(tiles[p], (int)(d.sms * bytes[p] / total)));
+        sum += alloc[p];
+    }
+    while (sum < d.sms) {   // spare SMs to the problem with the most bytes per CTA
+        int best = -1;
+        for (int p = 0; p < G; p++)
+            if (alloc[p] < tiles[p] && (best < 0 || bytes[p] / alloc[p] > bytes[best] / alloc[best])) best = p;
+        if (best < 0) break;
+        alloc[best]++;
+        sum++;
+    }
+    while (sum > d.sms) {   // more problems than the rounding allows: take from the lightest CTAs
+        int best = -1;
+        for (int p = 0; p < G; p++)
+            if (alloc[p] > 1 && (best < 0 || bytes[p] / alloc[p] < bytes[best] / alloc[best])) best = p;
+        if (best < 0) break;
+        alloc[best]--;
+        sum--;
+    }
+    static GroupArgs g;   // host staging of the kernel parameter (copied at launch)
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lk(mu);
+    g.G = G;
+    g.cta0[0] = 0;
+    size_t smem = 0;
+    for (int p = 0; p < G; p++) {
+        GemvTcPlan plan;
+        w4_status s = plan_gemv_tc(w[p].K, w[p].N, 1, pdl, plan, alloc[p]);
+        if (s != W4_OK) return s;
+        if (plan.S != 1) return W4_ERR_UNSUPPORTED;
+        s = gemv_tc_setup(&w[p], x[p], y[p], nullptr, plan, pdl, g.cmap[p], g.smap[p], g.a[p]);
+        if (s != W4_OK) return s;
+        g.cta0[p + 1] = g.cta0[p] + plan.grid;
+        smem = std::max(smem, plan.smem);
+    }
+    static size_t configured = 0;
+    if (smem > configured) {
+        if (cudaFuncSetAttribute(gemv_nvfp4_m1_grouped_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem) != cudaSuccess)
+            return W4_ERR_CUDA;
+        configured = smem;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(g.cta0[G], 1, 1);
+    cfg.blockDim = dim3(kTcThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, gemv_nvfp4_m1_grouped_kernel, g) != cudaSuccess) return W4_ERR_CUDA;
     return launch_status();
 }
 
@@ -513,6 +603,20 @@ w4_status w4a16_gemv_ex(const w4_weights *w, const void *x, int M, float *y, voi
     case W4_FMT_ROCMFP4_FAST: return launch_gemv_fmt<W4_FMT_ROCMFP4_FAST>(w, x, M, y, workspace, p, pdl, st);
     }
     return W4_ERR_ARG;
+}
+
+w4_status w4a16_gemv_grouped(const w4_weights *w, const void *const *x, float *const *y, int G, unsigned flags,
+                             void *stream) {
+    if (!w || !x || !y || G < 1 || G > kMaxGroup || (flags & ~W4_LAUNCH_PDL)) return W4_ERR_ARG;
+    for (int p = 0; p < G; p++) {
+        const w4_status s = check_weights(&w[p]);
+        if (s != W4_OK) return s;
+        if (w[p].fmt != W4_FMT_NVFP4) return W4_ERR_UNSUPPORTED;
+        if (!x[p] || !y[p]) return W4_ERR_ARG;
+        if (!aligned16(x[p]) || !aligned16(y[p])) return W4_ERR_ALIGN;
+        if (w[p].K % 256) return W4_ERR_UNSUPPORTED;
+    }
+    return launch_gemv_grouped(w, x, y, G, (flags & W4_LAUNCH_PDL) != 0, as_stream(stream));
 }
 
 w4_status w4a16_gemv(const w4_weights *w, const void *x, int M, float *y, void *workspace, size_t workspace_bytes,
