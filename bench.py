@@ -5,8 +5,11 @@ Headline (one JSON line from rank 0): W4A16 GEMV HBM GB/s at M=1 on the decode
 GEMV sweep -- NVFP4 weights of the 4B-class decoder shapes (K, N) = (2560,4096),
 (2560,1024), (4096,2560), (2560,9728), (9728,2560), Student-t(4) weights of std
 0.02 with 0.01% of entries x20, BF16 activations N(0,1).  One step = one GEMV
-over each of the five matrices (a CUDA graph of five launches chained with
-programmatic dependent launch).  GB/s counts the packed bytes read (codes +
+over each of the five matrices, issued as one grouped launch
+(w4a16_gemv_grouped), six steps (one per rotating weight copy) captured in one
+CUDA graph; the same sweep as five separate launches chained with programmatic
+dependent launch is reported beside it.
+GB/s counts the packed bytes read (codes +
 scales + global scale, 4.5 bits per weight).  Six packed copies of every matrix
 rotate across steps (248 MB > the 126 MB L2), so no step finds its weights in
 L2.
@@ -185,6 +188,19 @@ def time_graphs(graphs, steps, warmup):
     return a.elapsed_time(b) / steps  # ms per replay
 
 
+def separate_sweep(W4, mats, reps=120):
+    """The sweep as five w4a16_gemv launches per step (CUDA graph, PDL-chained)."""
+    def step_fn(r):
+        def run():
+            for m in mats:
+                W4.w4a16_gemv(m["copies"][r], m["x"], out=m["y"], flags=W4.LAUNCH_PDL)
+        return run
+    graphs = [capture(step_fn(r)) for r in range(ROTATE)]
+    ms = time_graphs(graphs, reps, 2 * ROTATE)
+    step_bytes = sum(m["bytes"] for m in mats)
+    return {"us_per_step": round(ms * 1e3, 2), "GB/s": round(step_bytes / ms / 1e6, 1), "launches_per_step": 5}
+
+
 def per_shape(W4, mats, reps=40):
     out = {}
     for m in mats:
@@ -298,8 +314,31 @@ def stream_bench(W4, I):
             res[key] = {"tokens/s": round(M * 1e3 / ms, 1), "ms_per_token_pass": round(ms, 4),
                         "GB/s": round(loops * nbytes / ms / 1e6, 1)}
             del g
+    # one token with the projections that share an input issued together:
+    # {q,k,v} and {gate,up} as grouped launches, o and down alone (4 launches per layer)
+    x1 = {K: I.activations(1, K, 6000 + K, device="cuda") for K in (2560, 4096, 9728)}
+    y1 = [torch.empty(1, N, dtype=torch.float32, device="cuda") for (_, _, N) in I.LAYER]
+    groups = [(0, 1, 2), (3,), (4, 5), (6,)]
+    for loops in (1, 2):
+        def run():
+            for row in layers:
+                for _ in range(loops):
+                    for grp in groups:
+                        if len(grp) == 1:
+                            p = row[grp[0]]
+                            W4.w4a16_gemv(p, x1[p.K], out=y1[grp[0]], flags=W4.LAUNCH_PDL)
+                        else:
+                            W4.w4a16_gemv_grouped([row[j] for j in grp], [x1[row[j].K] for j in grp],
+                                                  outs=[y1[j] for j in grp])
+        g = capture(run)
+        ms = time_graphs([g], 5, 2)
+        key = "M1_grouped" + ("_looped" if loops == 2 else "")
+        res[key] = {"tokens/s": round(1e3 / ms, 1), "ms_per_token_pass": round(ms, 4),
+                    "GB/s": round(loops * nbytes / ms / 1e6, 1)}
+        del g
     res["packed_bytes_per_pass"] = nbytes
-    res["config"] = "36 layers x {q,k,v,o,gate,up,down}, NVFP4, one CUDA graph per token with PDL"
+    res["config"] = ("36 layers x {q,k,v,o,gate,up,down}, NVFP4, one CUDA graph per token; M1/M16: 7 launches "
+                     "per layer with PDL; M1_grouped: {q,k,v} and {gate,up} grouped, 4 launches per layer")
     return res
 
 
@@ -364,28 +403,37 @@ def run_ours(args, world, rank, local):
     mats = sweep_setup(W4, I, M=1)
     step_bytes = sum(m["bytes"] for m in mats)
 
+    xs, ys = [m["x"] for m in mats], [m["y"] for m in mats]
+
     def step_fn(r):
         def run():
-            for m in mats:
-                W4.w4a16_gemv(m["copies"][r], m["x"], out=m["y"], flags=W4.LAUNCH_PDL)
+            W4.w4a16_gemv_grouped([m["copies"][r] for m in mats], xs, outs=ys)
         return run
     graphs = [capture(step_fn(r)) for r in range(ROTATE)]
+    # the ROTATE steps of one rotation in a single graph (one graph launch per
+    # ROTATE steps); single-step graphs cover a remainder
+    graph_rot = capture(lambda: [step_fn(r)() for r in range(ROTATE)])
+
+    def run_steps(n):
+        for _ in range(n // ROTATE):
+            graph_rot.replay()
+        for i in range(n % ROTATE):
+            graphs[i].replay()
 
     clocks = Clocks(local)
     clocks.start()
     # untimed pre-heat (~1 s) so the timed steps run at load clocks, then W warm-up steps
     t_end = time.perf_counter() + 1.0
     while time.perf_counter() < t_end:
-        time_graphs(graphs, 60, 0)
-    for i in range(args.warmup):
-        graphs[i % ROTATE].replay()
+        run_steps(60)
+        torch.cuda.synchronize()
+    run_steps(args.warmup)
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
-    for i in range(args.steps):
-        graphs[i % ROTATE].replay()
+    run_steps(args.steps)
     b.record()
     torch.cuda.synchronize()
     barrier(world)
@@ -394,48 +442,48 @@ def run_ours(args, world, rank, local):
     ms_total = max_over_ranks(world, a.elapsed_time(b))
     ms_step = ms_total / args.steps
     value = replica_value(world, step_bytes, ms_total, args.steps)  # GB/s over all ranks
-    launches = 5 * args.steps
+    launches = args.steps
 
-    # per-launch duration of the dominant kernel (the M=1 GEMV; every launch in the step)
-    achieved = step_bytes / ms_step / 1e6 / 1.0
+    # the step is one launch of the dominant kernel (the grouped M=1 GEMV)
+    achieved = step_bytes / ms_step / 1e6
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": TRAFFIC_PER_LAUNCH,
-            "kernel": "w4::gemv_nvfp4_m1_kernel",
-            "note": f"every launch of the step is this kernel: algorithmic bytes per launch averaged over the 5 "
-                    f"sweep shapes ({step_bytes / 5:.0f} B) / average launch duration in the timed PDL graph "
-                    f"(CUDA events on the launching stream); peak = {pk['source']} copy bandwidth"}
+            "kernel": "w4::gemv_nvfp4_m1_grouped_kernel",
+            "note": f"one launch per step: algorithmic bytes of the 5 sweep matrices ({step_bytes} B) / "
+                    f"average step duration in the timed graphs (CUDA events on the launching stream); "
+                    f"peak = {pk['source']} copy bandwidth; traffic = ncu DRAM bytes of one launch"}
 
     # end-to-end through the public API with pinned host buffers
     xh = [m["x"].cpu().pin_memory() for m in mats]
     yh = [torch.empty_like(m["y"], device="cpu").pin_memory() for m in mats]
     xd = [torch.empty_like(m["x"]) for m in mats]
     e2e_steps = max(20, min(args.steps, 200))
-    for r in range(2):
-        for i, m in enumerate(mats):
+    def e2e_step(r):
+        for i in range(len(mats)):
             xd[i].copy_(xh[i], non_blocking=True)
-            W4.w4a16_gemv(m["copies"][r], xd[i], out=m["y"])
-            yh[i].copy_(m["y"], non_blocking=True)
-        torch.cuda.synchronize()
+        W4.w4a16_gemv_grouped([m["copies"][r] for m in mats], xd, outs=ys)
+        for i in range(len(mats)):
+            yh[i].copy_(ys[i], non_blocking=True)
+        torch.cuda.synchronize()  # the step's result is read on the host
+    for r in range(2):
+        e2e_step(r)
     barrier(world)
     ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ea.record()
     for s in range(e2e_steps):
-        for i, m in enumerate(mats):
-            xd[i].copy_(xh[i], non_blocking=True)
-            W4.w4a16_gemv(m["copies"][s % ROTATE], xd[i], out=m["y"])
-            yh[i].copy_(m["y"], non_blocking=True)
-        torch.cuda.synchronize()  # the step's result is read on the host
+        e2e_step(s % ROTATE)
     eb.record()
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(world, ea.elapsed_time(eb)) / e2e_steps
     e2e = {"value": round(world * step_bytes / e2e_ms / 1e6, 1), "unit": "GB/s",
            "h2d_bytes_per_step": sum(t.numel() * 2 for t in xh),
            "d2h_bytes_per_step": sum(t.numel() * 4 for t in yh),
-           "note": "per step: pinned x -> device, w4a16_gemv via the Python binding of the C ABI "
-                   "(no graph), y -> pinned host, synchronize; packed weights resident"}
+           "note": "per step: 5 pinned x -> device, one w4a16_gemv_grouped via the Python binding of the "
+                   "C ABI (no graph), 5 y -> pinned host, synchronize; packed weights resident"}
 
     extras = {}
     if not args.no_extras:
+        extras["sweep_separate_launches"] = separate_sweep(W4, mats)
         extras["per_shape_isolated"] = per_shape(W4, mats)
         extras["sweep_skinny"] = sweep_m_bench(W4, I, mats, pk)
         del graphs, mats
@@ -460,7 +508,8 @@ def run_ours(args, world, rank, local):
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4-w/bf16-x/f32-acc",
                 "data": "synthetic (seeded Student-t(4) weights, N(0,1) activations)",
-                "config": {"workload": WORKLOAD, "M": 1, "step": "5 GEMV launches (CUDA graph, PDL)",
+                "config": {"workload": WORKLOAD, "M": 1,
+                           "step": f"5 GEMVs in one grouped launch; {ROTATE} steps per CUDA graph",
                            "l2": f"{ROTATE} rotating packed copies per matrix (248 MB > L2)",
                            "bytes_per_step": step_bytes, "parallelism": f"replicas x{world}"},
                 "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
@@ -496,11 +545,11 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
-# ncu-measured DRAM bytes (read + write) per launch of the dominant kernel,
-# w4::gemv_nvfp4_m1_kernel, averaged over its launches in
-# `bench.py --steps 3 --warmup 3 --no-extras` (profiles/launches_bench_decode_sweep_m1.md).
+# ncu-measured DRAM bytes (read + write) of one launch of the dominant kernel,
+# w4::gemv_nvfp4_m1_grouped_kernel, on the five sweep matrices
+# (profiles/gemv_nvfp4_m1_grouped_sweep.md).
 # Set to None when that kernel changes until it is measured again.
-TRAFFIC_PER_LAUNCH = 8307220
+TRAFFIC_PER_LAUNCH = 41381888
 
 
 def main():

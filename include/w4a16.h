@@ -167,6 +167,17 @@ w4_status w4a16_gemv(const w4_weights *w, const void *x, int M, float *y,
  * default mma.sync kernel, so it is opt-in.
  */
 #define W4_LAUNCH_TMEM 2u
+/*
+ * W4_LAUNCH_FP4_MMA (NVFP4, M == 1, K % 256 == 0, N % 8 == 0, codes 32-byte
+ * aligned; otherwise ignored) runs the one-token GEMV on tcgen05.mma
+ * kind::f8f6f4: the packed E2M1 codes go to the tensor cores as stored (TMA
+ * unpacks them to the padded 4-bit operand layout), x is split per 16-k block
+ * into three exact E5M2 parts, and the E4M3 block scales are applied per row
+ * after the MMA (blocks whose x cannot be split exactly are summed in
+ * binary32).  Also accepted by w4a16_gemv_grouped, where it applies when every
+ * problem qualifies.
+ */
+#define W4_LAUNCH_FP4_MMA 4u
 w4_status w4a16_gemv_ex(const w4_weights *w, const void *x, int M, float *y,
                         void *workspace, size_t workspace_bytes, unsigned flags,
                         void *stream);
@@ -183,7 +194,7 @@ w4_status w4a16_gemv_ex(const w4_weights *w, const void *x, int M, float *y,
  *   x      array of G device pointers to [K_p] BF16 (may repeat).
  *   y      array of G device pointers to [N_p] float (must not overlap).
  *   G      1..8.
- *   flags  0 or W4_LAUNCH_PDL.
+ *   flags  0, W4_LAUNCH_PDL and / or W4_LAUNCH_FP4_MMA.
  * The arrays are read on the host before the call returns; no workspace.
  * Errors: W4_ERR_ARG (null pointers, G out of range, unknown flags),
  * W4_ERR_ALIGN, W4_ERR_UNSUPPORTED (format or K), W4_ERR_CUDA.

@@ -301,3 +301,110 @@ def test_grouped_argument_errors():
     pr = W4.pack_rocmfp4(I.matrix("laplace", 16, 256, 82, 0.015, 0.0, device="cuda"), "dual")
     with pytest.raises(W4.W4Error):
         W4.w4a16_gemv_grouped([pr], [x])
+
+
+@pytest.mark.parametrize("K,N", [(2560, 4096), (2560, 1024), (4096, 2560), (2560, 9728), (9728, 2560), (256, 8),
+                                 (512, 72), (1024, 136), (2560, 1000), (12288, 64), (2560, 333)])
+def test_fp4_mma_path(K, N):
+    """The one-token GEMV on kind::f8f6f4 (E2M1 codes unpacked by TMA, x in three
+    E5M2 parts per block) meets the bound; N % 8 != 0 takes the other kernel."""
+    pw, wh = nvfp4_packed(I.sweep_weights(K, N, 6)[:N].contiguous())
+    x = I.bf16_rne(I.activations(1, K, 23).double())
+    for flags in (W4.LAUNCH_FP4_MMA, W4.LAUNCH_FP4_MMA | W4.LAUNCH_PDL):
+        run_and_check(pw, wh, x, flags=flags)
+
+
+@pytest.mark.parametrize("case", ["zeros", "one_block", "scaled_up", "scaled_down", "range_2p20", "wide_range",
+                                  "subnormal", "far_blocks", "inf", "nan"])
+def test_fp4_mma_ranges(case):
+    """Blocks split exactly into E5M2 parts, and blocks that are not (spread over
+    more than 2^23, a factor outside binary32's normal range, Inf / NaN), which
+    the epilogue sums in binary32."""
+    K, N = 2560, 392
+    pw, wh = nvfp4_packed(I.sweep_weights(K, N, 7)[:N].contiguous())
+    x = I.activations(1, K, 24).double()
+    if case == "zeros":
+        x[:] = 0.0
+    elif case == "one_block":
+        x[:] = 0.0
+        x[:, 16 * 19:16 * 20] = I.activations(1, 16, 25).double()
+    elif case == "scaled_up":
+        x *= 2.0 ** 100
+    elif case == "scaled_down":
+        x *= 2.0 ** -100
+    elif case == "range_2p20":        # inside one block, still exact
+        x[:, 16:24] *= 2.0 ** 10
+        x[:, 24:32] *= 2.0 ** -10
+    elif case == "wide_range":        # 2^80 inside one block: that block falls back
+        x[:, :8] *= 2.0 ** 40
+        x[:, 8:16] *= 2.0 ** -40
+    elif case == "subnormal":
+        x[:, ::3] = 2.0 ** -130
+    elif case == "far_blocks":        # one block 2^240 below the largest: its factor underflows
+        x[:, 32:48] *= 2.0 ** -120
+        x[:, :16] *= 2.0 ** 120
+    elif case == "inf":
+        x[:, 700] = float("inf")
+    else:
+        x[:, 1234] = float("nan")
+    x = I.bf16_rne(x)
+    y = np_of(W4.w4a16_gemv(pw, x.cuda(), flags=W4.LAUNCH_FP4_MMA))
+    yr, ar = O.matmul(x, wh)
+    if case in ("inf", "nan"):
+        assert np.array_equal(np.isfinite(y), np.isfinite(yr))
+        fin = np.isfinite(yr)
+        assert_within_tolerance(y[fin], yr[fin], ar[fin])
+    else:
+        assert_within_tolerance(y, yr, ar)
+
+
+def test_fp4_mma_grouped():
+    """Grouped launches on kind::f8f6f4: the sweep, q/k/v sharing x, and a group
+    with a ragged N (which takes the decode kernel for the whole group)."""
+    pws, whs, xs = [], [], []
+    for idx, (K, N) in enumerate(I.SWEEP_SHAPES):
+        pw, wh = nvfp4_packed(I.sweep_weights(K, N, idx))
+        pws.append(pw); whs.append(wh); xs.append(I.sweep_x(1, K, idx))
+    check_group(pws, whs, xs, flags=W4.LAUNCH_FP4_MMA)
+    check_group(pws, whs, xs, flags=W4.LAUNCH_FP4_MMA | W4.LAUNCH_PDL)
+    K = 2560
+    mats = [nvfp4_packed(I.sweep_weights(K, N, 90 + i)[:N].contiguous()) for i, N in enumerate((4096, 1024, 1024))]
+    x = I.activations(1, K, 91)
+    check_group([m[0] for m in mats], [m[1] for m in mats], [x, x, x], flags=W4.LAUNCH_FP4_MMA)
+    shapes = [(256, 8), (1024, 152), (2560, 333), (9728, 16), (512, 8), (4096, 4096)]
+    pws, whs, xs = [], [], []
+    for i, (K, N) in enumerate(shapes):
+        pw, wh = nvfp4_packed(I.sweep_weights(K, N, 100 + i)[:N].contiguous())
+        pws.append(pw); whs.append(wh); xs.append(I.activations(1, K, 110 + i))
+    check_group(pws, whs, xs, flags=W4.LAUNCH_FP4_MMA)
+    check_group(pws[:2] + pws[3:], whs[:2] + whs[3:], xs[:2] + xs[3:], flags=W4.LAUNCH_FP4_MMA)
+
+
+def test_fp4_mma_graph_deterministic():
+    """Replayed in a CUDA graph with PDL the kernel gives the same bits every time."""
+    shapes = [(2560, 1024), (4096, 512), (9728, 256)]
+    pws, whs, xs = [], [], []
+    for i, (K, N) in enumerate(shapes):
+        pw, wh = nvfp4_packed(I.sweep_weights(K, N, 120 + i)[:N].contiguous())
+        pws.append(pw); whs.append(wh); xs.append(I.activations(1, K, 130 + i))
+    fl = W4.LAUNCH_FP4_MMA | W4.LAUNCH_PDL
+    ref = [y.clone() for y in check_group(pws, whs, xs, flags=fl)]
+    xd = [x.cuda() for x in xs]
+    outs = [torch.empty(1, w.N, device="cuda") for w in pws]
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        W4.w4a16_gemv_grouped(pws, xd, outs=outs, flags=fl)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        W4.w4a16_gemv_grouped(pws, xd, outs=outs, flags=fl)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    for a, b in zip(ref, outs):
+        assert torch.equal(a, b)
+    single = [W4.w4a16_gemv(p, x, flags=fl) for p, x in zip(pws, xd)]
+    for a, b in zip(ref, single):
+        assert torch.equal(a, b)

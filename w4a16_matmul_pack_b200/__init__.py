@@ -24,7 +24,7 @@ import torch
 
 __all__ = [
     "W4Error", "PackedWeights", "FMT_NVFP4", "FMT_ROCMFP4_DUAL", "FMT_ROCMFP4_FAST",
-    "LAUNCH_PDL", "LAUNCH_TMEM", "pack_nvfp4", "pack_rocmfp4", "w4a16_gemv", "w4a16_gemv_grouped", "w4a16_gemm",
+    "LAUNCH_PDL", "LAUNCH_TMEM", "LAUNCH_FP4_MMA", "pack_nvfp4", "pack_rocmfp4", "w4a16_gemv", "w4a16_gemv_grouped", "w4a16_gemm",
     "w4a16_workspace_bytes", "pack_nvfp4_workspace_bytes", "w4_encode_scalars",
     "w4_device_error", "lib", "library_path",
 ]
@@ -33,6 +33,7 @@ FMT_NVFP4, FMT_ROCMFP4_DUAL, FMT_ROCMFP4_FAST = 1, 2, 3
 SCALE_ABSMAX, SCALE_MSE = 0, 1
 LAUNCH_PDL = 1
 LAUNCH_TMEM = 2   # opt-in tcgen05 GEMV for one token (see include/w4a16.h)
+LAUNCH_FP4_MMA = 4   # one token on tcgen05 kind::f8f6f4, codes unpacked by TMA (see include/w4a16.h)
 BLOCK_BYTES = {FMT_ROCMFP4_DUAL: 18, FMT_ROCMFP4_FAST: 17}
 _FMT_NAMES = {"nvfp4": FMT_NVFP4, "dual": FMT_ROCMFP4_DUAL, "fast": FMT_ROCMFP4_FAST}
 

@@ -11,6 +11,7 @@
 #include "gemv_tc.cuh"
 #include "gemv_m1.cuh"
 #include "gemv_umma.cuh"
+#include "gemv_f4.cuh"
 #include "gemm.cuh"
 
 using namespace w4;
@@ -315,6 +316,37 @@ w4_status launch_gemv_tc_m(const w4_weights *w, const void *x, float *y, void *w
     return launch_status();
 }
 
+// SMs shared out among G problems in proportion to their packed bytes (at
+// least one CTA each, at most max_cta[p]).
+void share_sms(const w4_weights *w, int G, int sms, const int *max_cta, int *alloc) {
+    double bytes[kMaxGroup], total = 0.0;
+    int sum = 0;
+    for (int p = 0; p < G; p++) {
+        bytes[p] = (double)w[p].N * (w[p].K / 2 + w[p].K / 16);
+        total += bytes[p];
+    }
+    for (int p = 0; p < G; p++) {
+        alloc[p] = std::max(1, std::min(max_cta[p], (int)(sms * bytes[p] / total)));
+        sum += alloc[p];
+    }
+    while (sum < sms) {   // spare SMs to the problem with the most bytes per CTA
+        int best = -1;
+        for (int p = 0; p < G; p++)
+            if (alloc[p] < max_cta[p] && (best < 0 || bytes[p] / alloc[p] > bytes[best] / alloc[best])) best = p;
+        if (best < 0) break;
+        alloc[best]++;
+        sum++;
+    }
+    while (sum > sms) {   // more problems than the rounding allows: take from the lightest CTAs
+        int best = -1;
+        for (int p = 0; p < G; p++)
+            if (alloc[p] > 1 && (best < 0 || bytes[p] / alloc[p] < bytes[best] / alloc[best])) best = p;
+        if (best < 0) break;
+        alloc[best]--;
+        sum--;
+    }
+}
+
 // Several one-token NVFP4 problems in one launch (gemv_m1.cuh): the SMs are
 // shared out in proportion to each problem's packed bytes (at least one CTA
 // each, at most one per 16-row tile), and every CTA runs the single-problem
@@ -323,33 +355,9 @@ w4_status launch_gemv_grouped(const w4_weights *w, const void *const *x, float *
                               cudaStream_t st) {
     DeviceInfo d;
     if (device_info(d) != W4_OK) return W4_ERR_CUDA;
-    double bytes[kMaxGroup], total = 0.0;
-    int tiles[kMaxGroup], alloc[kMaxGroup], sum = 0;
-    for (int p = 0; p < G; p++) {
-        bytes[p] = (double)w[p].N * (w[p].K / 2 + w[p].K / 16);
-        total += bytes[p];
-        tiles[p] = (w[p].N + kTcRows - 1) / kTcRows;
-    }
-    for (int p = 0; p < G; p++) {
-        alloc[p] = std::max(1, std::min(tiles[p], (int)(d.sms * bytes[p] / total)));
-        sum += alloc[p];
-    }
-    while (sum < d.sms) {   // spare SMs to the problem with the most bytes per CTA
-        int best = -1;
-        for (int p = 0; p < G; p++)
-            if (alloc[p] < tiles[p] && (best < 0 || bytes[p] / alloc[p] > bytes[best] / alloc[best])) best = p;
-        if (best < 0) break;
-        alloc[best]++;
-        sum++;
-    }
-    while (sum > d.sms) {   // more problems than the rounding allows: take from the lightest CTAs
-        int best = -1;
-        for (int p = 0; p < G; p++)
-            if (alloc[p] > 1 && (best < 0 || bytes[p] / alloc[p] < bytes[best] / alloc[best])) best = p;
-        if (best < 0) break;
-        alloc[best]--;
-        sum--;
-    }
+    int tiles[kMaxGroup], alloc[kMaxGroup];
+    for (int p = 0; p < G; p++) tiles[p] = (w[p].N + kTcRows - 1) / kTcRows;
+    share_sms(w, G, d.sms, tiles, alloc);
     static GroupArgs g;   // host staging of the kernel parameter (copied at launch)
     static std::mutex mu;
     std::lock_guard<std::mutex> lk(mu);
@@ -474,6 +482,126 @@ w4_status launch_umma(const w4_weights *w, const void *x, float *y, const UmmaPl
     return launch_status();
 }
 
+// One token with the codes fed to tcgen05 kind::f8f6f4 (gemv_f4.cuh): NVFP4,
+// K a multiple of 256, N of 8, codes 32-byte aligned (the unpacking TMA type).
+constexpr int kF4MaxK = 32768;   // x (64 KB) and two stages fit in shared memory
+bool f4_applies(const w4_weights *w, int M) {
+    return M == 1 && w->fmt == W4_FMT_NVFP4 && w->K % f4::kStageK == 0 && w->K <= kF4MaxK && w->N % 8 == 0 &&
+           (reinterpret_cast<uintptr_t>(w->codes) & 31u) == 0;
+}
+
+// Stages that fit with x of length K (at most kMaxStages, at least 2).
+int f4_stages(const DeviceInfo &d, int K) {
+    int NS = f4::kMaxStages;
+    while (NS > 2 && f4::smem_bytes(NS, K) > (size_t)d.smem_optin) NS--;
+    return NS;
+}
+
+// CTAs of a single problem: at least 64 rows each (a 128-row MMA tile at least
+// half used), at most one per SM.
+int f4_grid(int N, int sms) { return std::max(1, std::min(sms, N / 64)); }
+
+w4_status f4_setup(const w4_weights *w, const void *x, float *y, int NS, CUtensorMap &amap, CUtensorMap &smap,
+                   f4::Args &a) {
+    PFN_encodeTiled enc = get_encode_tiled();
+    if (!enc) return W4_ERR_CUDA;
+    const int K = w->K, N = w->N;
+    const cuuint64_t adims[2] = {(cuuint64_t)K, (cuuint64_t)N};   // 4-bit elements
+    const cuuint64_t astr[1] = {(cuuint64_t)K / 2};
+    const cuuint32_t abox[2] = {128, (cuuint32_t)f4::kRows};
+    const cuuint64_t sdims[2] = {(cuuint64_t)K / 16, (cuuint64_t)N};
+    const cuuint64_t sstr[1] = {(cuuint64_t)K / 16};
+    const cuuint32_t sbox[2] = {(cuuint32_t)(f4::kStageK / 16), (cuuint32_t)f4::kRows};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&amap, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<uint8_t *>(w->codes), adims, astr, abox, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return W4_ERR_CUDA;
+    if (enc(&smap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(w->scales), sdims, sstr, sbox, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return W4_ERR_CUDA;
+    a.x = reinterpret_cast<const uint16_t *>(x);
+    a.y = y;
+    a.gscale = w->global_scale;
+    a.K = K;
+    a.N = N;
+    a.NS = NS;
+    return W4_OK;
+}
+
+w4_status launch_f4(const w4_weights *w, const void *x, float *y, bool pdl, cudaStream_t st) {
+    DeviceInfo d;
+    if (device_info(d) != W4_OK) return W4_ERR_CUDA;
+    const int NS = f4_stages(d, w->K);
+    const size_t smem = f4::smem_bytes(NS, w->K);
+    static size_t configured = 0;
+    if (smem > configured) {
+        if (cudaFuncSetAttribute(f4::gemv_nvfp4_f4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return W4_ERR_CUDA;
+        configured = smem;
+    }
+    CUtensorMap amap, smap;
+    f4::Args a;
+    w4_status s = f4_setup(w, x, y, NS, amap, smap, a);
+    if (s != W4_OK) return s;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(f4_grid(w->N, d.sms), 1, 1);
+    cfg.blockDim = dim3(f4::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, f4::gemv_nvfp4_f4_kernel, amap, smap, a) != cudaSuccess) return W4_ERR_CUDA;
+    return launch_status();
+}
+
+w4_status launch_f4_grouped(const w4_weights *w, const void *const *x, float *const *y, int G, bool pdl,
+                            cudaStream_t st) {
+    DeviceInfo d;
+    if (device_info(d) != W4_OK) return W4_ERR_CUDA;
+    int max_cta[kMaxGroup], alloc[kMaxGroup];
+    for (int p = 0; p < G; p++) max_cta[p] = std::max(1, w[p].N / 64);
+    share_sms(w, G, d.sms, max_cta, alloc);
+    int Kmax = 0;
+    for (int p = 0; p < G; p++) Kmax = std::max(Kmax, w[p].K);
+    const int NS = f4_stages(d, Kmax);
+    const size_t smem = f4::smem_bytes(NS, Kmax);
+    static f4::GroupArgs g;   // host staging of the kernel parameter (copied at launch)
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lk(mu);
+    g.G = G;
+    g.cta0[0] = 0;
+    for (int p = 0; p < G; p++) {
+        const w4_status s = f4_setup(&w[p], x[p], y[p], NS, g.amap[p], g.smap[p], g.a[p]);
+        if (s != W4_OK) return s;
+        g.cta0[p + 1] = g.cta0[p] + alloc[p];
+    }
+    static size_t configured = 0;
+    if (smem > configured) {
+        if (cudaFuncSetAttribute(f4::gemv_nvfp4_f4_grouped_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem) != cudaSuccess)
+            return W4_ERR_CUDA;
+        configured = smem;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(g.cta0[G], 1, 1);
+    cfg.blockDim = dim3(f4::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, f4::gemv_nvfp4_f4_grouped_kernel, g) != cudaSuccess) return W4_ERR_CUDA;
+    return launch_status();
+}
+
 w4_status launch_gemv_tc(const w4_weights *w, const void *x, int M, float *y, void *ws, const GemvTcPlan &p, bool pdl,
                          cudaStream_t st) {
     switch (M) {
@@ -579,12 +707,14 @@ w4_status w4a16_gemv_ex(const w4_weights *w, const void *x, int M, float *y, voi
                         size_t workspace_bytes, unsigned flags, void *stream) {
     w4_status s = check_weights(w);
     if (s != W4_OK) return s;
-    if (!x || !y || M < 1 || M > 16 || (flags & ~(W4_LAUNCH_PDL | W4_LAUNCH_TMEM))) return W4_ERR_ARG;
+    if (!x || !y || M < 1 || M > 16 || (flags & ~(W4_LAUNCH_PDL | W4_LAUNCH_TMEM | W4_LAUNCH_FP4_MMA)))
+        return W4_ERR_ARG;
     if (!aligned16(x) || !aligned16(y) || (workspace && !aligned16(workspace))) return W4_ERR_ALIGN;
     if (w->K % k_unit(w->fmt)) return W4_ERR_UNSUPPORTED;
     const bool pdl = (flags & W4_LAUNCH_PDL) != 0;
     cudaStream_t st = as_stream(stream);
     if (w->fmt == W4_FMT_NVFP4) {
+        if ((flags & W4_LAUNCH_FP4_MMA) && f4_applies(w, M)) return launch_f4(w, x, y, pdl, st);
         if ((flags & W4_LAUNCH_TMEM) && umma_applies(w->K, M)) {
             UmmaPlan u;
             if ((s = plan_umma(w->K, w->N, pdl, u)) != W4_OK) return s;
@@ -607,7 +737,7 @@ w4_status w4a16_gemv_ex(const w4_weights *w, const void *x, int M, float *y, voi
 
 w4_status w4a16_gemv_grouped(const w4_weights *w, const void *const *x, float *const *y, int G, unsigned flags,
                              void *stream) {
-    if (!w || !x || !y || G < 1 || G > kMaxGroup || (flags & ~W4_LAUNCH_PDL)) return W4_ERR_ARG;
+    if (!w || !x || !y || G < 1 || G > kMaxGroup || (flags & ~(W4_LAUNCH_PDL | W4_LAUNCH_FP4_MMA))) return W4_ERR_ARG;
     for (int p = 0; p < G; p++) {
         const w4_status s = check_weights(&w[p]);
         if (s != W4_OK) return s;
@@ -616,7 +746,11 @@ w4_status w4a16_gemv_grouped(const w4_weights *w, const void *const *x, float *c
         if (!aligned16(x[p]) || !aligned16(y[p])) return W4_ERR_ALIGN;
         if (w[p].K % 256) return W4_ERR_UNSUPPORTED;
     }
-    return launch_gemv_grouped(w, x, y, G, (flags & W4_LAUNCH_PDL) != 0, as_stream(stream));
+    const bool pdl = (flags & W4_LAUNCH_PDL) != 0;
+    bool f4 = (flags & W4_LAUNCH_FP4_MMA) != 0;
+    for (int p = 0; p < G; p++) f4 = f4 && f4_applies(&w[p], 1);
+    if (f4) return launch_f4_grouped(w, x, y, G, pdl, as_stream(stream));
+    return launch_gemv_grouped(w, x, y, G, pdl, as_stream(stream));
 }
 
 w4_status w4a16_gemv(const w4_weights *w, const void *x, int M, float *y, void *workspace, size_t workspace_bytes,

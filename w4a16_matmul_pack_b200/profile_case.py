@@ -3,6 +3,10 @@
     python -m w4a16_matmul_pack_b200.profile_case gemv --fmt nvfp4 --K 2560 --N 9728 --M 1 --reps 3
     python -m w4a16_matmul_pack_b200.profile_case gemm --M 2048 --K 2560 --N 9728 --reps 2
     python -m w4a16_matmul_pack_b200.profile_case pack --fmt dual --K 2560 --N 9728
+    python -m w4a16_matmul_pack_b200.profile_case grouped --reps 3 [--flags 4]
+
+`grouped` runs the five decode-sweep matrices (K,N) = (2560,4096), (2560,1024),
+(4096,2560), (2560,9728), (9728,2560) at one token as one grouped launch.
 
 Inputs are the seeded synthetic matrices (Student-t weights, N(0,1) x; Laplace
 weights for ROCmFP4).  Exits non-zero on any library or CUDA error.
@@ -25,14 +29,23 @@ import w4a16_matmul_pack_b200 as W4  # noqa: E402
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("op", choices=["gemv", "gemm", "pack"])
+    ap.add_argument("op", choices=["gemv", "gemm", "pack", "grouped"])
     ap.add_argument("--fmt", default="nvfp4", choices=["nvfp4", "dual", "fast"])
     ap.add_argument("--M", type=int, default=1)
     ap.add_argument("--K", type=int, default=2560)
     ap.add_argument("--N", type=int, default=9728)
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--flags", type=int, default=0, help="launch flags of the GEMV (e.g. 4 = W4_LAUNCH_FP4_MMA)")
     a = ap.parse_args()
     torch.cuda.set_device(0)
+    if a.op == "grouped":
+        ws = [W4.pack_nvfp4(I.sweep_weights(K, N, i, device="cuda")) for i, (K, N) in enumerate(I.SWEEP_SHAPES)]
+        xs = [I.sweep_x(1, K, i, device="cuda") for i, (K, _) in enumerate(I.SWEEP_SHAPES)]
+        torch.cuda.synchronize()
+        for _ in range(a.reps):
+            W4.w4a16_gemv_grouped(ws, xs, flags=a.flags)
+        finish()
+        return
     if a.fmt == "nvfp4":
         W = I.matrix("student_t4", a.N, a.K, 7, 0.02, 1e-4, 20.0, device="cuda")
     else:
@@ -49,9 +62,13 @@ def main():
         torch.cuda.synchronize()
         for _ in range(a.reps):
             if a.op == "gemv":
-                W4.w4a16_gemv(pw, x)
+                W4.w4a16_gemv(pw, x, flags=a.flags)
             else:
                 W4.w4a16_gemm(pw, x)
+    finish()
+
+
+def finish():
     torch.cuda.synchronize()
     err = W4.w4_device_error(clear=True)
     if err:
