@@ -50,6 +50,14 @@ def lib():
         L.orc_e4m3_encode.argtypes = [F]
         L.orc_cb10_index.argtypes = [F, F]
         L.orc_pack_nvfp4.argtypes = [P, I, I, P, P, P]
+        L.orc_pack_nvfp4_ex.argtypes = [P, I, I, I, P, P, P, P]
+        L.orc_nvfp4_error.restype = F
+        L.orc_nvfp4_error.argtypes = [P, P, I, F]
+        L.orc_nvfp4_search.argtypes = [P, P, F, P]
+        L.orc_rocm_error_w.restype = F
+        L.orc_rocm_error_w.argtypes = [P, P, I, I]
+        L.orc_rocm_search_w.argtypes = [P, P, I, P]
+        L.orc_pack_rocmfp4_w.argtypes = [P, I, I, I, P, P]
         L.orc_dequant_nvfp4.argtypes = [P, P, F, I, I, I, P]
         L.orc_rocm_error.restype = F
         L.orc_rocm_error.argtypes = [P, I, I]
@@ -128,15 +136,44 @@ def e2m1_encode_array(v) -> np.ndarray:
 
 
 # --- packers ------------------------------------------------------------------
-def pack_nvfp4(W):
-    """W: bf16 [N][K] -> (codes u8 [N][K/2], scales u8 [N][K/16], global scale float32)."""
+def _weights(imp, n):
+    if imp is None:
+        return None
+    w = np.ascontiguousarray(imp, np.float32)
+    assert w.size == n
+    return w
+
+
+def pack_nvfp4(W, mse: bool = False, importance=None):
+    """W: bf16 [N][K] -> (codes u8 [N][K/2], scales u8 [N][K/16], global scale float32).
+    mse: block scales by the error search (importance: K channel weights or None)."""
     b = _bits(W)
     N, K = b.shape
     codes = np.zeros((N, K // 2), np.uint8)
     scales = np.zeros((N, K // 16), np.uint8)
     g = np.zeros(1, np.float32)
-    _check(lib().orc_pack_nvfp4(_p(b), K, N, _p(codes), _p(scales), _p(g)))
+    w = _weights(importance, K)
+    _check(lib().orc_pack_nvfp4_ex(_p(b), K, N, 1 if mse else 0, None if w is None else _p(w),
+                                   _p(codes), _p(scales), _p(g)))
     return codes, scales, np.float32(g[0])
+
+
+def nvfp4_error(x, u: int, g, importance=None) -> float:
+    """Binary32 reconstruction error of 16 weights under E4M3 code u and global scale g."""
+    x = np.ascontiguousarray(x, np.float32)
+    assert x.size == 16
+    w = _weights(importance, 16)
+    return lib().orc_nvfp4_error(_p(x), None if w is None else _p(w), u, float(np.float32(g)))
+
+
+def nvfp4_search(x, g, importance=None):
+    """-> (best E4M3 code, its binary32 error) for 16 weights at global scale g."""
+    x = np.ascontiguousarray(x, np.float32)
+    assert x.size == 16
+    w = _weights(importance, 16)
+    e = np.zeros(1, np.float32)
+    u = lib().orc_nvfp4_search(_p(x), None if w is None else _p(w), float(np.float32(g)), _p(e))
+    return u, float(e[0])
 
 
 def dequant_nvfp4(codes, scales, g, n0: int = 0, rows: int | None = None) -> np.ndarray:
@@ -148,25 +185,29 @@ def dequant_nvfp4(codes, scales, g, n0: int = 0, rows: int | None = None) -> np.
     return out
 
 
-def rocm_error(x, u: int) -> float:
+def rocm_error(x, u: int, importance=None) -> float:
     x = np.ascontiguousarray(x, np.float32)
-    return lib().orc_rocm_error(_p(x), x.size, u)
+    w = _weights(importance, x.size)
+    return lib().orc_rocm_error_w(_p(x), None if w is None else _p(w), x.size, u)
 
 
-def rocm_search(x):
+def rocm_search(x, importance=None):
     """-> (best UE4M3 code, its binary32 error)."""
     x = np.ascontiguousarray(x, np.float32)
+    w = _weights(importance, x.size)
     e = np.zeros(1, np.float32)
-    u = lib().orc_rocm_search(_p(x), x.size, _p(e))
+    u = lib().orc_rocm_search_w(_p(x), None if w is None else _p(w), x.size, _p(e))
     return u, float(e[0])
 
 
-def pack_rocmfp4(W, fmt: int) -> np.ndarray:
-    """W: bf16 [N][K] -> blocks u8 [N][K/32][18 (Dual) | 17 (FAST)]."""
+def pack_rocmfp4(W, fmt: int, importance=None) -> np.ndarray:
+    """W: bf16 [N][K] -> blocks u8 [N][K/32][18 (Dual) | 17 (FAST)]; importance:
+    K channel weights (finite, >= 0) or None."""
     b = _bits(W)
     N, K = b.shape
     out = np.zeros((N, K // 32, BLOCK_BYTES[fmt]), np.uint8)
-    _check(lib().orc_pack_rocmfp4(_p(b), K, N, fmt, _p(out)))
+    w = _weights(importance, K)
+    _check(lib().orc_pack_rocmfp4_w(_p(b), K, N, fmt, None if w is None else _p(w), _p(out)))
     return out
 
 

@@ -44,6 +44,17 @@
  *  - UE4M3 candidates are the bytes 0x00..0x7E (zero included), weights are
  *    level * scale (no tensor scale).  Error E(u) = sum_i fma(d_i, d_i, E) in
  *    element order with d_i = x_i - s*l_i; argmin, ties to the smallest code.
+ *  - Importance weighting (the "rocmwhy" page, section 03: candidates scored by
+ *    reconstruction error "with optional importance weighting"; its example
+ *    gives an outlier low importance): one nonnegative weight per input channel
+ *    k, E(u) = sum_i fma(w_k * d_i, d_i, E); with no weights w = 1, which gives
+ *    exactly the unweighted sum.
+ *  - NVFP4 scale by search (the same recipe applied to NVFP4 blocks, global
+ *    scale g fixed by the abs-max rule): candidates are the E4M3 bytes
+ *    0x00..0x7E; under candidate u, d = E4M3(u) * g, each code is the E2M1
+ *    encoding of x / d exactly as in the abs-max packer, r = e2m1 * d (binary32),
+ *    E(u) = sum_i fma(w_k * (x_i - r_i), x_i - r_i, E); argmin, ties to the
+ *    smallest code.  The abs-max scale is one of the candidates.
  */
 #include <math.h>
 #include <stdint.h>
@@ -152,14 +163,65 @@ int orc_cb10_index(float a, float s)
 /* NVFP4 pack / dequant                                                     */
 /* ------------------------------------------------------------------------ */
 
+/* Reconstruction error of 16 weights x under E4M3 scale code u and global
+ * scale g, in binary32 (see the header); imp: 16 weights or NULL. */
+float orc_nvfp4_error(const float *x, const float *imp, int u, float g)
+{
+    const float d = (float)orc_e4m3_decode(u) * g;
+    float E = 0.0f;
+    for (int i = 0; i < 16; i++) {
+        int c = 0;
+        if (d != 0.0f)
+            c = orc_e2m1_encode(x[i] / d);
+        const float r = (float)orc_e2m1_decode(c) * d;
+        const float e = x[i] - r;
+        const float t = imp ? imp[i] * e : e;
+        E = fmaf(t, e, E);
+    }
+    return E;
+}
+
+/* Search over the 127 finite E4M3 codes; ties -> smallest code. */
+int orc_nvfp4_search(const float *x, const float *imp, float g, float *best_err)
+{
+    int best_u = 0;
+    float best = orc_nvfp4_error(x, imp, 0, g);
+    for (int u = 1; u < 127; u++) {
+        const float E = orc_nvfp4_error(x, imp, u, g);
+        if (E < best) {
+            best = E;
+            best_u = u;
+        }
+    }
+    if (best_err)
+        *best_err = best;
+    return best_u;
+}
+
+/* imp: NULL, or K weights that must be finite and >= 0. */
+static int check_importance(const float *imp, int K)
+{
+    if (!imp)
+        return ORC_OK;
+    for (int k = 0; k < K; k++)
+        if (!isfinite(imp[k]) || imp[k] < 0.0f)
+            return ORC_ERR_NONFINITE;
+    return ORC_OK;
+}
+
 /*
  * W: bf16 bit patterns, [N][K] (K contiguous).  K % 16 == 0.
  * codes: [N][K/2]; scales: [N][K/16]; *g_out: global scale.
+ * mse = 0: block scale E4M3(absmax / 6 / g) (imp must be NULL);
+ * mse = 1: block scale by the error search, imp = NULL or K channel weights.
  */
-int orc_pack_nvfp4(const uint16_t *W, int K, int N, uint8_t *codes, uint8_t *scales, float *g_out)
+int orc_pack_nvfp4_ex(const uint16_t *W, int K, int N, int mse, const float *imp, uint8_t *codes,
+                      uint8_t *scales, float *g_out)
 {
-    if (K <= 0 || N <= 0 || K % 16 != 0)
+    if (K <= 0 || N <= 0 || K % 16 != 0 || (mse != 0 && mse != 1) || (!mse && imp))
         return ORC_ERR_ARG;
+    if (check_importance(imp, K) != ORC_OK)
+        return ORC_ERR_NONFINITE;
     long long total = (long long)K * N;
 
     /* 1. tensor abs-max */
@@ -179,7 +241,7 @@ int orc_pack_nvfp4(const uint16_t *W, int K, int N, uint8_t *codes, uint8_t *sca
     const float g = amax / 2688.0f;
     *g_out = g;
 
-    /* 3. per 16-block: scale = E4M3(absmax / 6 / global), code = E2M1(x / (scale * global)) */
+    /* 3. per 16-block: the scale, then code = E2M1(x / (scale * global)) */
     #pragma omp parallel for schedule(static)
     for (int n = 0; n < N; n++) {
         const uint16_t *row = W + (long long)n * K;
@@ -192,7 +254,9 @@ int orc_pack_nvfp4(const uint16_t *W, int K, int N, uint8_t *codes, uint8_t *sca
                     bamax = fabsf(x[j]);
             }
             int s = 0;
-            if (g != 0.0f) {
+            if (mse) {
+                s = orc_nvfp4_search(x, imp ? imp + 16 * b : NULL, g, NULL);
+            } else if (g != 0.0f) {
                 float sf = (bamax / 6.0f) / g;
                 s = orc_e4m3_encode(sf);
             }
@@ -212,6 +276,11 @@ int orc_pack_nvfp4(const uint16_t *W, int K, int N, uint8_t *codes, uint8_t *sca
         }
     }
     return ORC_OK;
+}
+
+int orc_pack_nvfp4(const uint16_t *W, int K, int N, uint8_t *codes, uint8_t *scales, float *g_out)
+{
+    return orc_pack_nvfp4_ex(W, K, N, 0, NULL, codes, scales, g_out);
 }
 
 /* w_hat[r][k] for rows n0..n0+rows-1: e2m1 * E4M3(scale) * global, in binary64. */
@@ -234,8 +303,9 @@ void orc_dequant_nvfp4(const uint8_t *codes, const uint8_t *scales, float g, int
 /* ROCmFP4 pack / dequant                                                   */
 /* ------------------------------------------------------------------------ */
 
-/* Reconstruction error of x[0..n-1] under UE4M3 code u, in binary32. */
-float orc_rocm_error(const float *x, int n, int u)
+/* Reconstruction error of x[0..n-1] under UE4M3 code u, in binary32; imp:
+ * n channel weights or NULL. */
+float orc_rocm_error_w(const float *x, const float *imp, int n, int u)
 {
     float s = (float)orc_e4m3_decode(u);
     float E = 0.0f;
@@ -244,18 +314,24 @@ float orc_rocm_error(const float *x, int n, int u)
         float r = s * (float)CB10[idx];          /* exact: <= 8 significant bits */
         float w = signbit(x[i]) ? -r : r;
         float d = x[i] - w;
-        E = fmaf(d, d, E);
+        float t = imp ? imp[i] * d : d;
+        E = fmaf(t, d, E);
     }
     return E;
 }
 
+float orc_rocm_error(const float *x, int n, int u)
+{
+    return orc_rocm_error_w(x, NULL, n, u);
+}
+
 /* Exhaustive scale search over the 127 finite UE4M3 codes; ties -> smallest code. */
-int orc_rocm_search(const float *x, int n, float *best_err)
+int orc_rocm_search_w(const float *x, const float *imp, int n, float *best_err)
 {
     int best_u = 0;
-    float best = orc_rocm_error(x, n, 0);
+    float best = orc_rocm_error_w(x, imp, n, 0);
     for (int u = 1; u < 127; u++) {
-        float E = orc_rocm_error(x, n, u);
+        float E = orc_rocm_error_w(x, imp, n, u);
         if (E < best) {
             best = E;
             best_u = u;
@@ -264,6 +340,11 @@ int orc_rocm_search(const float *x, int n, float *best_err)
     if (best_err)
         *best_err = best;
     return best_u;
+}
+
+int orc_rocm_search(const float *x, int n, float *best_err)
+{
+    return orc_rocm_search_w(x, NULL, n, best_err);
 }
 
 /* Codebook10 code of x under scale code u. */
@@ -280,12 +361,15 @@ static int rocm_code(float x, int u)
 
 /*
  * fmt 2 = Dual (18-byte blocks), 3 = FAST (17-byte blocks).  W: bf16 [N][K],
- * K % 32 == 0.  blocks: [N][K/32][18|17].
+ * K % 32 == 0.  imp: NULL or K channel weights (finite, >= 0).
+ * blocks: [N][K/32][18|17].
  */
-int orc_pack_rocmfp4(const uint16_t *W, int K, int N, int fmt, uint8_t *blocks)
+int orc_pack_rocmfp4_w(const uint16_t *W, int K, int N, int fmt, const float *imp, uint8_t *blocks)
 {
     if (K <= 0 || N <= 0 || K % 32 != 0 || (fmt != 2 && fmt != 3))
         return ORC_ERR_ARG;
+    if (check_importance(imp, K) != ORC_OK)
+        return ORC_ERR_NONFINITE;
     long long total = (long long)K * N;
     for (long long i = 0; i < total; i++)
         if (!isfinite(bf16_to_float(W[i])))
@@ -301,9 +385,10 @@ int orc_pack_rocmfp4(const uint16_t *W, int K, int N, int fmt, uint8_t *blocks)
                 x[j] = bf16_to_float(W[(long long)n * K + 32 * b + j]);
             uint8_t *out = blocks + ((long long)n * nb + b) * bb;
             int code[32];
+            const float *wb = imp ? imp + 32 * b : NULL;
             if (fmt == 2) {
-                int u0 = orc_rocm_search(x, 16, NULL);
-                int u1 = orc_rocm_search(x + 16, 16, NULL);
+                int u0 = orc_rocm_search_w(x, wb, 16, NULL);
+                int u1 = orc_rocm_search_w(x + 16, wb ? wb + 16 : NULL, 16, NULL);
                 out[0] = (uint8_t)u0;
                 out[1] = (uint8_t)u1;
                 for (int j = 0; j < 16; j++) {
@@ -311,7 +396,7 @@ int orc_pack_rocmfp4(const uint16_t *W, int K, int N, int fmt, uint8_t *blocks)
                     code[j + 16] = rocm_code(x[j + 16], u1);
                 }
             } else {
-                int u = orc_rocm_search(x, 32, NULL);
+                int u = orc_rocm_search_w(x, wb, 32, NULL);
                 out[0] = (uint8_t)u;
                 for (int j = 0; j < 32; j++)
                     code[j] = rocm_code(x[j], u);
@@ -322,6 +407,11 @@ int orc_pack_rocmfp4(const uint16_t *W, int K, int N, int fmt, uint8_t *blocks)
         }
     }
     return ORC_OK;
+}
+
+int orc_pack_rocmfp4(const uint16_t *W, int K, int N, int fmt, uint8_t *blocks)
+{
+    return orc_pack_rocmfp4_w(W, K, N, fmt, NULL, blocks);
 }
 
 void orc_dequant_rocmfp4(const uint8_t *blocks, int fmt, int K, int n0, int rows, double *w_hat)
