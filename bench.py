@@ -214,9 +214,10 @@ def per_shape(W4, mats, reps=40):
 
 
 def sweep_m_bench(W4, I, mats, pk):
-    """The decode sweep at M = 4 and 16 (same packed copies, PDL graph per step)."""
+    """The decode sweep at M = 4, 9 (a speculative-verify step: one token plus
+    eight drafted ones) and 16 (same packed copies, PDL graph per step)."""
     out = {}
-    for M in (4, 16):
+    for M in (4, 9, 16):
         xs = [I.sweep_x(M, m["K"], idx, device="cuda") for idx, m in enumerate(mats)]
         ys = [torch.empty(M, m["N"], dtype=torch.float32, device="cuda") for m in mats]
         ws = torch.empty(max(W4.w4a16_workspace_bytes(m["copies"][0], M) for m in mats) + 16,
@@ -362,6 +363,23 @@ def pack_bench(W4, I):
         ms = a.elapsed_time(b)
         out[f"pack_rocmfp4_{fmt}"] = {"shape": "K=2560 N=9728 Laplace", "ms": round(ms, 3),
                                       "candidate_evals/s": round(127 * L.numel() / ms / 1e3, 1)}
+    imp = torch.rand(L.shape[1], generator=torch.Generator().manual_seed(5)).cuda() * 2.0
+    W4.pack_rocmfp4(L, "dual", importance=imp)
+    W4.pack_nvfp4(W, scale_search=W4.SCALE_MSE)
+    W4.pack_nvfp4(W, scale_search=W4.SCALE_MSE, importance=imp)
+    torch.cuda.synchronize()
+    for name, fn in (("pack_rocmfp4_dual_weighted", lambda: W4.pack_rocmfp4(L, "dual", importance=imp)),
+                     ("pack_nvfp4_scale_search", lambda: W4.pack_nvfp4(W, scale_search=W4.SCALE_MSE)),
+                     ("pack_nvfp4_scale_search_weighted",
+                      lambda: W4.pack_nvfp4(W, scale_search=W4.SCALE_MSE, importance=imp))):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b)
+        out[name] = {"shape": "K=2560 N=9728", "ms": round(ms, 3),
+                     "candidate_evals/s": round(127 * W.numel() / ms / 1e3, 1)}
     return out
 
 

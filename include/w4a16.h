@@ -105,7 +105,14 @@ typedef struct {
  * g == 0, or a block whose s * g is 0, gives all-zero scales and codes.
  *   W            [N][K] BF16, K % 16 == 0, K >= 16, N >= 1.
  *   block        must be 16.
- *   scale_search W4_SCALE_ABSMAX (W4_SCALE_MSE returns W4_ERR_UNSUPPORTED).
+ *   scale_search W4_SCALE_ABSMAX as above, or W4_SCALE_MSE: g as above, and
+ *                each block scale chosen by search over the E4M3 codes
+ *                u = 0x00..0x7E (the [rocmwhy] section 03 recipe applied to
+ *                NVFP4 blocks): under u, d = dec(u) * g, each code is
+ *                E2M1(x / d) as above, r = e2m1 * d, and the block error
+ *                E(u) = sum fma(x - r, x - r, E) over k in order, binary32;
+ *                the smallest E wins, ties to the smaller code.  The abs-max
+ *                scale is one of the candidates, so the error never grows.
  *   codes        out [N][K/2];  scales out [N][K/16];  global_scale out float.
  *   workspace    >= pack_nvfp4_workspace_bytes() bytes of device scratch.
  *   d_status     optional device int: set to W4_OK at the start of the call,
@@ -115,6 +122,22 @@ w4_status pack_nvfp4(const void *W, int K, int N, int block, int scale_search,
                      uint8_t *codes, uint8_t *scales, float *global_scale,
                      void *workspace, size_t workspace_bytes, int *d_status,
                      void *stream);
+
+/*
+ * pack_nvfp4_ex -- pack_nvfp4 with importance weights for the scale search
+ * ([rocmwhy] section 03: candidates scored by reconstruction error "with
+ * optional importance weighting").
+ *   importance  NULL, or device float[K]: one weight w_k per input channel,
+ *               finite and >= 0 (otherwise d_status = W4_ERR_NONFINITE and the
+ *               outputs are undefined); requires scale_search = W4_SCALE_MSE
+ *               (W4_ERR_ARG otherwise).  The block error becomes
+ *               E(u) = sum fma(w_k * (x - r), x - r, E); w = 1 gives exactly
+ *               the unweighted bytes.
+ */
+w4_status pack_nvfp4_ex(const void *W, int K, int N, int block, int scale_search,
+                        const float *importance, uint8_t *codes, uint8_t *scales,
+                        float *global_scale, void *workspace, size_t workspace_bytes,
+                        int *d_status, void *stream);
 size_t pack_nvfp4_workspace_bytes(void);
 
 /*
@@ -127,7 +150,11 @@ size_t pack_nvfp4_workspace_bytes(void);
  * ties to the smaller code.
  *   W        [N][K] BF16, K % 32 == 0.
  *   block    must be 32.  fmt = W4_FMT_ROCMFP4_DUAL or W4_FMT_ROCMFP4_FAST.
- *   importance must be NULL (weighted error returns W4_ERR_UNSUPPORTED).
+ *   importance NULL, or device float[K]: one weight w_k per input channel
+ *            ([rocmwhy] section 03, "optional importance weighting"), finite
+ *            and >= 0 (otherwise d_status = W4_ERR_NONFINITE, outputs
+ *            undefined); the error becomes E(u) = sum fma(w_k * d, d, E), and
+ *            w = 1 gives exactly the unweighted bytes.
  *   blocks   out [N][K/32][18 | 17] (layout as in w4_weights).
  *   d_status optional, as for pack_nvfp4.
  */

@@ -43,12 +43,15 @@ def test_host_validation_without_gpu(lib):
     # null matrix / bad block size / bad format: rejected before any CUDA call
     assert lib.pack_nvfp4(None, 64, 4, 16, 0, P(16), P(16), P(16), P(16), 16, None, None) == 1
     assert lib.pack_nvfp4(P(16), 64, 4, 32, 0, P(16), P(16), P(16), P(16), 16, None, None) == 1
-    assert lib.pack_nvfp4(P(16), 64, 4, 16, 1, P(16), P(16), P(16), P(16), 16, None, None) == 3
+    assert lib.pack_nvfp4(P(16), 64, 4, 16, 2, P(16), P(16), P(16), P(16), 16, None, None) == 1
+    # importance weights only with the scale search, and 16-byte aligned
+    assert lib.pack_nvfp4_ex(P(16), 64, 4, 16, 0, P(16), P(16), P(16), P(16), P(16), 16, None, None) == 1
+    assert lib.pack_nvfp4_ex(P(16), 64, 4, 16, 1, P(20), P(16), P(16), P(16), P(16), 16, None, None) == 2
     assert lib.pack_nvfp4(P(16), 64, 4, 16, 0, P(16), P(16), P(16), P(16), 4, None, None) == 7
     assert lib.pack_nvfp4(P(17), 64, 4, 16, 0, P(16), P(16), P(16), P(16), 16, None, None) == 2
     assert lib.pack_rocmfp4(P(16), 48, 4, 32, 2, None, P(16), None, None) == 1
     assert lib.pack_rocmfp4(P(16), 64, 4, 32, 9, None, P(16), None, None) == 1
-    assert lib.pack_rocmfp4(P(16), 64, 4, 32, 2, P(16), P(16), None, None) == 3
+    assert lib.pack_rocmfp4(P(16), 64, 4, 32, 2, P(20), P(16), None, None) == 2
     w = W4._Weights(1, 256, 8, 16, 16, 16)
     assert lib.w4a16_gemv(ctypes.byref(w), P(16), 17, P(16), None, 0, None) == 1
     assert lib.w4a16_gemv(ctypes.byref(w), P(16), 0, P(16), None, 0, None) == 1

@@ -51,7 +51,7 @@ def test_nvfp4_sweep(idx, M):
     run_and_check(pw, wh, I.sweep_x(M, K, idx))
 
 
-@pytest.mark.parametrize("M", [2, 3, 5, 7, 8, 12])
+@pytest.mark.parametrize("M", [2, 3, 5, 7, 8, 9, 12])
 def test_nvfp4_other_m(M):
     pw, wh = nvfp4_packed(I.sweep_weights(9728, 2560, 4))
     run_and_check(pw, wh, I.sweep_x(M, 9728, 4))

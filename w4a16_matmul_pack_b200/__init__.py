@@ -72,6 +72,7 @@ def lib():
         WP = ctypes.POINTER(_Weights)
         sig = {
             "pack_nvfp4": ([P, I, I, I, I, P, P, P, P, S, P, P], I),
+            "pack_nvfp4_ex": ([P, I, I, I, I, P, P, P, P, P, S, P, P], I),
             "pack_nvfp4_workspace_bytes": ([], S),
             "pack_rocmfp4": ([P, I, I, I, I, P, P, P, P], I),
             "w4a16_gemv": ([WP, P, I, P, P, S, P], I),
@@ -143,11 +144,14 @@ def pack_nvfp4_workspace_bytes() -> int:
     return lib().pack_nvfp4_workspace_bytes()
 
 
-def pack_nvfp4(W: torch.Tensor, *, scale_search: int = SCALE_ABSMAX, out: Optional[PackedWeights] = None,
-               workspace: Optional[torch.Tensor] = None, d_status: Optional[torch.Tensor] = None,
-               stream=None) -> PackedWeights:
-    """Quantise bf16 W[N][K] to NVFP4 (see pack_nvfp4 in include/w4a16.h)."""
+def pack_nvfp4(W: torch.Tensor, *, scale_search: int = SCALE_ABSMAX, importance: Optional[torch.Tensor] = None,
+               out: Optional[PackedWeights] = None, workspace: Optional[torch.Tensor] = None,
+               d_status: Optional[torch.Tensor] = None, stream=None) -> PackedWeights:
+    """Quantise bf16 W[N][K] to NVFP4 (see pack_nvfp4 / pack_nvfp4_ex in include/w4a16.h);
+    importance: float32 [K] channel weights for the W4_SCALE_MSE search."""
     _cuda(W, "W", torch.bfloat16)
+    if importance is not None:
+        _cuda(importance, "importance", torch.float32)
     N, K = W.shape
     dev = W.device
     if out is None:
@@ -157,23 +161,28 @@ def pack_nvfp4(W: torch.Tensor, *, scale_search: int = SCALE_ABSMAX, out: Option
                             torch.empty(1, dtype=torch.float32, device=dev))
     if workspace is None:
         workspace = torch.empty(pack_nvfp4_workspace_bytes(), dtype=torch.uint8, device=dev)
-    _check(lib().pack_nvfp4(_ptr(W), K, N, 16, scale_search, _ptr(out.codes), _ptr(out.scales),
-                            _ptr(out.global_scale), _ptr(workspace), workspace.numel(), _ptr(d_status),
-                            _stream(stream)), "pack_nvfp4")
+    _check(lib().pack_nvfp4_ex(_ptr(W), K, N, 16, scale_search, _ptr(importance), _ptr(out.codes),
+                               _ptr(out.scales), _ptr(out.global_scale), _ptr(workspace), workspace.numel(),
+                               _ptr(d_status), _stream(stream)), "pack_nvfp4_ex")
     return out
 
 
-def pack_rocmfp4(W: torch.Tensor, fmt="dual", *, out: Optional[torch.Tensor] = None,
-                 d_status: Optional[torch.Tensor] = None, stream=None) -> PackedWeights:
-    """Quantise bf16 W[N][K] to ROCmFP4 Dual ("dual") or FAST ("fast")."""
+def pack_rocmfp4(W: torch.Tensor, fmt="dual", *, importance: Optional[torch.Tensor] = None,
+                 out: Optional[torch.Tensor] = None, d_status: Optional[torch.Tensor] = None,
+                 stream=None) -> PackedWeights:
+    """Quantise bf16 W[N][K] to ROCmFP4 Dual ("dual") or FAST ("fast"); importance:
+    float32 [K] channel weights for the error search, or None."""
     fmt = _FMT_NAMES.get(fmt, fmt)
     _cuda(W, "W", torch.bfloat16)
+    if importance is not None:
+        _cuda(importance, "importance", torch.float32)
     N, K = W.shape
     if fmt not in BLOCK_BYTES:
         raise ValueError("fmt must be 'dual' or 'fast'")
     if out is None:
         out = torch.empty(N, K // 32, BLOCK_BYTES[fmt], dtype=torch.uint8, device=W.device)
-    _check(lib().pack_rocmfp4(_ptr(W), K, N, 32, fmt, None, _ptr(out), _ptr(d_status), _stream(stream)),
+    _check(lib().pack_rocmfp4(_ptr(W), K, N, 32, fmt, _ptr(importance), _ptr(out), _ptr(d_status),
+                              _stream(stream)),
            "pack_rocmfp4")
     return PackedWeights(fmt, K, N, out)
 

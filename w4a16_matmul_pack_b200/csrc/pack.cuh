@@ -10,6 +10,11 @@
 //   Codebook10 levels; one warp per 32-weight block, lanes split the 127
 //   candidates, a lexicographic (error, code) shuffle reduction picks the
 //   winner (ties to the smaller code).
+// Importance weighting (the same page, section 03: "optional importance
+//   weighting"): one weight w_k >= 0 per input channel, E = sum fma(w_k d, d, E).
+// NVFP4 block scale by search: the same warp-per-block search over the finite
+//   E4M3 codes with the global scale fixed by the abs-max rule; under each
+//   candidate the codes are the abs-max packer's E2M1(x / (scale * g)).
 #pragma once
 
 #include "common.cuh"
@@ -108,8 +113,8 @@ __global__ void __launch_bounds__(256) nvfp4_encode_kernel(const uint4 *__restri
 // midpoints s*{.5,1.5,2.5,3.5,5,7,9} are exact in binary32, and a tie goes to
 // the even level index, i.e. ">=" at the midpoints that lead to an even index
 // (1.5, 3.5, 7) and ">" at the others.
-template <int n>
-__device__ __forceinline__ float rocm_error(const float (&xs)[n], float s) {
+template <int n, bool WT = false>
+__device__ __forceinline__ float rocm_error(const float (&xs)[n], float s, const float (&wv)[n]) {
     const float t0 = s * 0.5f, t1 = s * 1.5f, t2 = s * 2.5f, t3 = s * 3.5f;
     const float t4 = s * 5.0f, t5 = s * 7.0f, t6 = s * 9.0f;
     float E = 0.0f;
@@ -120,7 +125,7 @@ __device__ __forceinline__ float rocm_error(const float (&xs)[n], float s) {
                   (a >= t3 ? 1.0f : 0.0f);
         L += 2.0f * ((a > t4 ? 1.0f : 0.0f) + (a >= t5 ? 1.0f : 0.0f) + (a > t6 ? 1.0f : 0.0f));
         const float d = __fsub_rn(a, __fmul_rn(s, L));
-        E = __fmaf_rn(d, d, E);
+        E = __fmaf_rn(WT ? __fmul_rn(wv[i], d) : d, d, E);
     }
     return E;
 }
@@ -150,8 +155,9 @@ __device__ __forceinline__ void argmin_lanes(float &E, uint32_t &u, int width) {
 // DUAL: lanes 0..15 search the scale of elements 0..15 (8 candidates each),
 // lanes 16..31 the scale of 16..31.  FAST: all 32 lanes search one scale (4
 // candidates each).  Lane l ends holding the winning scale of element l.
-template <bool DUAL>
-__global__ void __launch_bounds__(256) rocm_pack_kernel(const uint16_t *__restrict__ W, long long nblk,
+template <bool DUAL, bool WT>
+__global__ void __launch_bounds__(256) rocm_pack_kernel(const uint16_t *__restrict__ W, long long nblk, int K,
+                                                        const float *__restrict__ imp,
                                                         uint8_t *__restrict__ out,
                                                         int *__restrict__ d_status) {
     constexpr int BB = DUAL ? 18 : 17;
@@ -165,10 +171,21 @@ __global__ void __launch_bounds__(256) rocm_pack_kernel(const uint16_t *__restri
             if (d_status) atomicExch(d_status, W4_ERR_NONFINITE);
             record_error(W4_ERR_NONFINITE);
         }
+        float wl = 1.0f;   // this lane's channel weight
+        if (WT) {
+            wl = __ldg(imp + (blk % (K / 32)) * 32 + lane);
+            if (!(wl >= 0.0f && wl <= 3.402823466e38f)) {
+                if (d_status) atomicExch(d_status, W4_ERR_NONFINITE);
+                record_error(W4_ERR_NONFINITE);
+            }
+        }
         const int base = DUAL ? (lane & 16) : 0;
-        float xs[NG];
+        float xs[NG], wv[NG];
 #pragma unroll
-        for (int i = 0; i < NG; i++) xs[i] = __shfl_sync(0xFFFFFFFFu, xl, base + i);
+        for (int i = 0; i < NG; i++) {
+            xs[i] = __shfl_sync(0xFFFFFFFFu, xl, base + i);
+            wv[i] = WT ? __shfl_sync(0xFFFFFFFFu, wl, base + i) : 1.0f;
+        }
 
         float bestE = 0.0f;
         uint32_t bestU = 0xFFu;
@@ -177,7 +194,7 @@ __global__ void __launch_bounds__(256) rocm_pack_kernel(const uint16_t *__restri
         for (int t = 0; t < (DUAL ? 8 : 4); t++) {
             const uint32_t u = (uint32_t)(sub + t * NG);
             if (u > 0x7Eu) break;
-            const float E = rocm_error<NG>(xs, e4m3_to_f32(u));
+            const float E = rocm_error<NG, WT>(xs, e4m3_to_f32(u), wv);
             if (bestU == 0xFFu || E < bestE) {
                 bestE = E;
                 bestU = u;
@@ -198,6 +215,89 @@ __global__ void __launch_bounds__(256) rocm_pack_kernel(const uint16_t *__restri
             o[0] = (uint8_t)bestU;
         }
         if (lane < 16) o[(DUAL ? 2 : 1) + lane] = (uint8_t)(code | (hi << 4));
+    }
+}
+
+// NVFP4 block scale by search.  One warp per 16-element block: lane l scores
+// the E4M3 codes l, l+32, l+64, l+96 (up to 0x7E): d = E4M3(u) * g, each code
+// E2M1(x / d), r = e2m1 * d, E = sum over k in order of fma(w * (x - r), x - r, E)
+// (w = 1 without weights) in binary32; the lexicographic (E, u) minimum wins.
+// Lane 0 then encodes the block under the winner, as nvfp4_encode_kernel does.
+template <bool WT>
+__global__ void __launch_bounds__(256) nvfp4_search_kernel(const uint16_t *__restrict__ W, long long nblocks, int K,
+                                                           const unsigned *__restrict__ ws,
+                                                           const float *__restrict__ imp,
+                                                           uint2 *__restrict__ codes, uint8_t *__restrict__ scales,
+                                                           float *__restrict__ global_scale,
+                                                           int *__restrict__ d_status) {
+    const float amax = __uint_as_float(ws[0] << 16);
+    const float g = __fdiv_rn(amax, 2688.0f);  // absmax / (6 * 448)
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        *global_scale = g;
+        if (ws[1]) {
+            if (d_status) *d_status = W4_ERR_NONFINITE;
+            record_error(W4_ERR_NONFINITE);
+        }
+    }
+    const int lane = threadIdx.x & 31;
+    const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+    const int kb = K / 16;
+    for (long long blk = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5; blk < nblocks; blk += warps) {
+        const float xe = __uint_as_float((uint32_t)__ldg(W + blk * 16 + (lane & 15)) << 16);
+        float we = 1.0f;
+        if (WT) {
+            we = __ldg(imp + (blk % kb) * 16 + (lane & 15));
+            if (lane < 16 && !(we >= 0.0f && we <= 3.402823466e38f)) {
+                if (d_status) atomicExch(d_status, W4_ERR_NONFINITE);
+                record_error(W4_ERR_NONFINITE);
+            }
+        }
+        float xs[16], wv[16];
+#pragma unroll
+        for (int i = 0; i < 16; i++) {
+            xs[i] = __shfl_sync(0xFFFFFFFFu, xe, i);
+            wv[i] = WT ? __shfl_sync(0xFFFFFFFFu, we, i) : 1.0f;
+        }
+        float bestE = 0.0f;
+        uint32_t bestU = 0xFFu;
+#pragma unroll 1
+        for (int t = 0; t < 4; t++) {
+            const uint32_t u = (uint32_t)(lane + 32 * t);
+            if (u > 0x7Eu) break;
+            const float d = __fmul_rn(e4m3_to_f32(u), g);
+            float E = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                float2 r = make_float2(0.0f, 0.0f);
+                if (d != 0.0f) {
+                    const uint32_t byte = f32x2_to_e2m1x2(__fdiv_rn(xs[2 * j], d), __fdiv_rn(xs[2 * j + 1], d));
+                    const uint32_t h = e2m1x2_to_f16x2(byte);
+                    const float2 v = __half22float2(*reinterpret_cast<const __half2 *>(&h));
+                    r = make_float2(__fmul_rn(v.x, d), __fmul_rn(v.y, d));
+                }
+                const float e0 = __fsub_rn(xs[2 * j], r.x), e1 = __fsub_rn(xs[2 * j + 1], r.y);
+                E = __fmaf_rn(WT ? __fmul_rn(wv[2 * j], e0) : e0, e0, E);
+                E = __fmaf_rn(WT ? __fmul_rn(wv[2 * j + 1], e1) : e1, e1, E);
+            }
+            if (bestU == 0xFFu || E < bestE) {
+                bestE = E;
+                bestU = u;
+            }
+        }
+        argmin_lanes(bestE, bestU, 32);
+        if (lane == 0) {
+            const float d = __fmul_rn(e4m3_to_f32(bestU), g);
+            uint32_t c[2] = {0u, 0u};
+            if (d != 0.0f) {
+#pragma unroll
+                for (int j = 0; j < 8; j++) {
+                    const uint32_t byte = f32x2_to_e2m1x2(__fdiv_rn(xs[2 * j], d), __fdiv_rn(xs[2 * j + 1], d));
+                    c[j >> 2] |= byte << (8 * (j & 3));
+                }
+            }
+            codes[blk] = make_uint2(c[0], c[1]);
+            scales[blk] = (uint8_t)bestU;
+        }
     }
 }
 

@@ -637,14 +637,16 @@ extern "C" {
 
 size_t pack_nvfp4_workspace_bytes(void) { return 16; }
 
-w4_status pack_nvfp4(const void *W, int K, int N, int block, int scale_search, uint8_t *codes, uint8_t *scales,
-                     float *global_scale, void *workspace, size_t workspace_bytes, int *d_status, void *stream) {
+w4_status pack_nvfp4_ex(const void *W, int K, int N, int block, int scale_search, const float *importance,
+                        uint8_t *codes, uint8_t *scales, float *global_scale, void *workspace, size_t workspace_bytes,
+                        int *d_status, void *stream) {
     if (!W || !codes || !scales || !global_scale || K < 16 || N < 1 || K % 16 || block != 16) return W4_ERR_ARG;
-    if (scale_search == W4_SCALE_MSE) return W4_ERR_UNSUPPORTED;
-    if (scale_search != W4_SCALE_ABSMAX) return W4_ERR_ARG;
+    if (scale_search != W4_SCALE_ABSMAX && scale_search != W4_SCALE_MSE) return W4_ERR_ARG;
+    if (importance && scale_search != W4_SCALE_MSE) return W4_ERR_ARG;
     if (!workspace || workspace_bytes < pack_nvfp4_workspace_bytes()) return W4_ERR_WORKSPACE;
     if (!aligned16(W) || !aligned16(codes) || !aligned16(scales) || !aligned16(workspace) ||
-        (reinterpret_cast<uintptr_t>(global_scale) & 3) || (reinterpret_cast<uintptr_t>(d_status) & 3))
+        (importance && !aligned16(importance)) || (reinterpret_cast<uintptr_t>(global_scale) & 3) ||
+        (reinterpret_cast<uintptr_t>(d_status) & 3))
         return W4_ERR_ALIGN;
     DeviceInfo d;
     if (device_info(d) != W4_OK) return W4_ERR_CUDA;
@@ -657,6 +659,18 @@ w4_status pack_nvfp4(const void *W, int K, int N, int block, int scale_search, u
     nvfp4_absmax_kernel<<<g1, 256, 0, st>>>(reinterpret_cast<const uint4 *>(W), n8,
                                              reinterpret_cast<unsigned *>(workspace));
     const long long nb = total / 16;
+    if (scale_search == W4_SCALE_MSE) {
+        const int g3 = (int)std::min<long long>((nb + 7) / 8, (long long)d.sms * 16);
+        if (importance)
+            nvfp4_search_kernel<true><<<g3, 256, 0, st>>>(
+                reinterpret_cast<const uint16_t *>(W), nb, K, reinterpret_cast<const unsigned *>(workspace), importance,
+                reinterpret_cast<uint2 *>(codes), scales, global_scale, d_status);
+        else
+            nvfp4_search_kernel<false><<<g3, 256, 0, st>>>(
+                reinterpret_cast<const uint16_t *>(W), nb, K, reinterpret_cast<const unsigned *>(workspace), nullptr,
+                reinterpret_cast<uint2 *>(codes), scales, global_scale, d_status);
+        return launch_status();
+    }
     const int g2 = (int)std::min<long long>((nb + 255) / 256, (long long)d.sms * 16);
     nvfp4_encode_kernel<<<g2, 256, 0, st>>>(reinterpret_cast<const uint4 *>(W), nb,
                                              reinterpret_cast<const unsigned *>(workspace),
@@ -664,22 +678,37 @@ w4_status pack_nvfp4(const void *W, int K, int N, int block, int scale_search, u
     return launch_status();
 }
 
+w4_status pack_nvfp4(const void *W, int K, int N, int block, int scale_search, uint8_t *codes, uint8_t *scales,
+                     float *global_scale, void *workspace, size_t workspace_bytes, int *d_status, void *stream) {
+    return pack_nvfp4_ex(W, K, N, block, scale_search, nullptr, codes, scales, global_scale, workspace,
+                         workspace_bytes, d_status, stream);
+}
+
 w4_status pack_rocmfp4(const void *W, int K, int N, int block, int fmt, const float *importance, uint8_t *blocks,
                        int *d_status, void *stream) {
     if (!W || !blocks || K < 32 || N < 1 || K % 32 || block != 32) return W4_ERR_ARG;
     if (fmt != W4_FMT_ROCMFP4_DUAL && fmt != W4_FMT_ROCMFP4_FAST) return W4_ERR_ARG;
-    if (importance) return W4_ERR_UNSUPPORTED;
-    if (!aligned16(W) || !aligned16(blocks) || (reinterpret_cast<uintptr_t>(d_status) & 3)) return W4_ERR_ALIGN;
+    if (!aligned16(W) || !aligned16(blocks) || (importance && !aligned16(importance)) ||
+        (reinterpret_cast<uintptr_t>(d_status) & 3))
+        return W4_ERR_ALIGN;
     DeviceInfo d;
     if (device_info(d) != W4_OK) return W4_ERR_CUDA;
     cudaStream_t st = as_stream(stream);
     if (d_status && cudaMemsetAsync(d_status, 0, sizeof(int), st) != cudaSuccess) return W4_ERR_CUDA;
     const long long nblk = (long long)K * N / 32;
     const int grid = (int)std::min<long long>((nblk + 7) / 8, (long long)d.sms * 16);
-    if (fmt == W4_FMT_ROCMFP4_DUAL)
-        rocm_pack_kernel<true><<<grid, 256, 0, st>>>(reinterpret_cast<const uint16_t *>(W), nblk, blocks, d_status);
-    else
-        rocm_pack_kernel<false><<<grid, 256, 0, st>>>(reinterpret_cast<const uint16_t *>(W), nblk, blocks, d_status);
+    const uint16_t *w16 = reinterpret_cast<const uint16_t *>(W);
+    if (fmt == W4_FMT_ROCMFP4_DUAL) {
+        if (importance)
+            rocm_pack_kernel<true, true><<<grid, 256, 0, st>>>(w16, nblk, K, importance, blocks, d_status);
+        else
+            rocm_pack_kernel<true, false><<<grid, 256, 0, st>>>(w16, nblk, K, nullptr, blocks, d_status);
+    } else {
+        if (importance)
+            rocm_pack_kernel<false, true><<<grid, 256, 0, st>>>(w16, nblk, K, importance, blocks, d_status);
+        else
+            rocm_pack_kernel<false, false><<<grid, 256, 0, st>>>(w16, nblk, K, nullptr, blocks, d_status);
+    }
     return launch_status();
 }
 
