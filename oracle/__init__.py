@@ -18,8 +18,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "w4a16_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
-FMT_NVFP4, FMT_DUAL, FMT_FAST = 1, 2, 3
-BLOCK_BYTES = {FMT_DUAL: 18, FMT_FAST: 17}
+FMT_NVFP4, FMT_DUAL, FMT_FAST, FMT_Q4_0 = 1, 2, 3, 4
+BLOCK_BYTES = {FMT_DUAL: 18, FMT_FAST: 17, FMT_Q4_0: 18}
 
 
 def build(force: bool = False) -> str:
@@ -58,6 +58,12 @@ def lib():
         L.orc_rocm_error_w.argtypes = [P, P, I, I]
         L.orc_rocm_search_w.argtypes = [P, P, I, P]
         L.orc_pack_rocmfp4_w.argtypes = [P, I, I, I, P, P]
+        L.orc_fp16_decode.restype = ctypes.c_double
+        L.orc_fp16_decode.argtypes = [I]
+        L.orc_fp16_encode.argtypes = [F]
+        L.orc_pack_q4_0.argtypes = [P, I, I, P]
+        L.orc_dequant_q4_0.argtypes = [P, I, I, I, P]
+        L.orc_reconstruction_sse.argtypes = [P, P, ctypes.c_longlong, P]
         L.orc_dequant_nvfp4.argtypes = [P, P, F, I, I, I, P]
         L.orc_rocm_error.restype = F
         L.orc_rocm_error.argtypes = [P, I, I]
@@ -219,6 +225,43 @@ def dequant_rocmfp4(blocks, fmt: int, n0: int = 0, rows: int | None = None) -> n
     out = np.zeros((rows, K), np.float64)
     lib().orc_dequant_rocmfp4(_p(blocks), fmt, K, n0, rows, _p(out))
     return out
+
+
+def fp16_decode(h: int) -> float:
+    return lib().orc_fp16_decode(h)
+
+
+def fp16_encode(v: float) -> int:
+    return lib().orc_fp16_encode(float(np.float32(v)))
+
+
+def pack_q4_0(W) -> np.ndarray:
+    """Stock Q4_0 (comparison format): W bf16 [N][K] -> blocks u8 [N][K/32][18]."""
+    b = _bits(W)
+    N, K = b.shape
+    out = np.zeros((N, K // 32, 18), np.uint8)
+    _check(lib().orc_pack_q4_0(_p(b), K, N, _p(out)))
+    return out
+
+
+def dequant_q4_0(blocks, n0: int = 0, rows: int | None = None) -> np.ndarray:
+    blocks = np.ascontiguousarray(blocks)
+    N, nb = blocks.shape[0], blocks.shape[1]
+    K = nb * 32
+    rows = N - n0 if rows is None else rows
+    out = np.zeros((rows, K), np.float64)
+    lib().orc_dequant_q4_0(_p(blocks), K, n0, rows, _p(out))
+    return out
+
+
+def reconstruction_sse(W, w_hat: np.ndarray):
+    """-> (sum (W - w_hat)^2, sum W^2) in float64 over the whole matrix."""
+    b = _bits(W)
+    w = np.ascontiguousarray(w_hat, np.float64)
+    assert w.shape == b.shape
+    out = np.zeros(2, np.float64)
+    lib().orc_reconstruction_sse(_p(b), _p(w), b.size, _p(out))
+    return float(out[0]), float(out[1])
 
 
 # --- matmul ---------------------------------------------------------------------

@@ -55,6 +55,15 @@
  *    encoding of x / d exactly as in the abs-max packer, r = e2m1 * d (binary32),
  *    E(u) = sum_i fma(w_k * (x_i - r_i), x_i - r_i, E); argmin, ties to the
  *    smallest code.  The abs-max scale is one of the candidates.
+ *  - Stock Q4_0, the pages' comparison format ("rocmwhy" format table and
+ *    section 02: 32 weights, evenly spaced integer steps, one FP16 scale,
+ *    18-byte blocks, "signed abs-max" reference scale; the lab's outlier 8.2
+ *    gives the shared scale 1.025 = 8.2 / 8): m = the weight of largest
+ *    magnitude (the first in k order on ties), d = FP16(m / -8) (binary32
+ *    division, then round to nearest even with saturation at 65504), each code
+ *    q = the nearest integer (ties to even) of x / d in binary32, clamped to
+ *    [-8, 7], stored as q + 8; d == 0 gives codes 8.  Block = [d (FP16, little
+ *    endian), 16 code bytes], code byte j = code[j] | code[j+16] << 4.
  */
 #include <math.h>
 #include <stdint.h>
@@ -431,6 +440,120 @@ void orc_dequant_rocmfp4(const uint8_t *blocks, int fmt, int K, int n0, int rows
             }
         }
     }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Stock Q4_0 (comparison format) and reconstruction error                  */
+/* ------------------------------------------------------------------------ */
+
+/* binary16 value of bits h, exactly. */
+double orc_fp16_decode(int h)
+{
+    int s = (h >> 15) & 1, e = (h >> 10) & 31, m = h & 1023;
+    double v;
+    if (e == 0)
+        v = ldexp((double)m, -24);
+    else if (e == 31)
+        v = m ? NAN : INFINITY;
+    else
+        v = ldexp(1.0 + m / 1024.0, e - 15);
+    return s ? -v : v;
+}
+
+/* Nearest binary16 (ties to even), saturating at +-65504; by exact search over
+ * the finite non-negative codes (the magnitudes are increasing in the code). */
+int orc_fp16_encode(float v)
+{
+    double a = fabs((double)v);
+    int sign = signbit(v) ? 0x8000 : 0;
+    if (a >= 65504.0)
+        return sign | 0x7BFF;
+    int lo = 0, hi = 0x7BFF;            /* largest code with value <= a */
+    while (lo < hi) {
+        int mid = (lo + hi + 1) / 2;
+        if (orc_fp16_decode(mid) <= a)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    int c = lo;
+    if (orc_fp16_decode(c) != a && c < 0x7BFF) {
+        double d0 = a - orc_fp16_decode(c), d1 = orc_fp16_decode(c + 1) - a;
+        if (d1 < d0 || (d1 == d0 && (c & 1)))
+            c = c + 1;
+    }
+    return sign | c;
+}
+
+/* W: bf16 [N][K], K % 32 == 0.  blocks: [N][K/32][18]. */
+int orc_pack_q4_0(const uint16_t *W, int K, int N, uint8_t *blocks)
+{
+    if (K <= 0 || N <= 0 || K % 32 != 0)
+        return ORC_ERR_ARG;
+    long long total = (long long)K * N;
+    for (long long i = 0; i < total; i++)
+        if (!isfinite(bf16_to_float(W[i])))
+            return ORC_ERR_NONFINITE;
+    const int nb = K / 32;
+    #pragma omp parallel for schedule(static)
+    for (int n = 0; n < N; n++) {
+        for (int b = 0; b < nb; b++) {
+            float x[32];
+            int jm = 0;
+            for (int j = 0; j < 32; j++) {
+                x[j] = bf16_to_float(W[(long long)n * K + 32 * b + j]);
+                if (fabsf(x[j]) > fabsf(x[jm]))
+                    jm = j;
+            }
+            const int h = orc_fp16_encode(x[jm] / -8.0f);
+            const float d = (float)orc_fp16_decode(h);
+            uint8_t *out = blocks + ((long long)n * nb + b) * 18;
+            out[0] = (uint8_t)(h & 0xFF);
+            out[1] = (uint8_t)(h >> 8);
+            int code[32];
+            for (int j = 0; j < 32; j++) {
+                int q = 0;
+                if (d != 0.0f) {
+                    float r = nearbyintf(x[j] / d);   /* round to nearest even */
+                    q = r < -8.0f ? -8 : (r > 7.0f ? 7 : (int)r);
+                }
+                code[j] = q + 8;
+            }
+            for (int j = 0; j < 16; j++)
+                out[2 + j] = (uint8_t)(code[j] | (code[j + 16] << 4));
+        }
+    }
+    return ORC_OK;
+}
+
+void orc_dequant_q4_0(const uint8_t *blocks, int K, int n0, int rows, double *w_hat)
+{
+    const int nb = K / 32;
+    #pragma omp parallel for schedule(static)
+    for (int r = 0; r < rows; r++) {
+        for (int b = 0; b < nb; b++) {
+            const uint8_t *blk = blocks + ((long long)(n0 + r) * nb + b) * 18;
+            const double d = orc_fp16_decode(blk[0] | (blk[1] << 8));
+            for (int j = 0; j < 32; j++) {
+                int c = (j < 16) ? (blk[2 + j] & 15) : (blk[2 + j - 16] >> 4);
+                w_hat[(long long)r * K + 32 * b + j] = d * (double)(c - 8);
+            }
+        }
+    }
+}
+
+/* out[0] = sum (W - w_hat)^2, out[1] = sum W^2 over rows x K, in binary64. */
+void orc_reconstruction_sse(const uint16_t *W, const double *w_hat, long long count, double *out)
+{
+    double e = 0.0, q = 0.0;
+    for (long long i = 0; i < count; i++) {
+        const double w = (double)bf16_to_float(W[i]);
+        const double d = w - w_hat[i];
+        e += d * d;
+        q += w * w;
+    }
+    out[0] = e;
+    out[1] = q;
 }
 
 /* ------------------------------------------------------------------------ */
