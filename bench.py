@@ -343,6 +343,26 @@ def stream_bench(W4, I):
     return res
 
 
+def quality_report(W4, I):
+    """Relative reconstruction error sum (W - w_hat)^2 / sum W^2 of every format
+    on the 2560x9728 Student-t sweep matrix and the 2560x9728 Laplace matrix
+    (the pages' quality-per-byte comparison, computed on the GPU in binary64)."""
+    out = {}
+    for name, W in (("student_t4_2560x9728", I.sweep_weights(2560, 9728, 3, device="cuda")),
+                    ("laplace_2560x9728", I.rocm_weights(device="cuda"))):
+        row = {}
+        for fmt, bpw, pack in (("nvfp4_absmax", 4.5, lambda w: W4.pack_nvfp4(w)),
+                               ("nvfp4_scale_search", 4.5, lambda w: W4.pack_nvfp4(w, scale_search=W4.SCALE_MSE)),
+                               ("rocmfp4_dual", 4.5, lambda w: W4.pack_rocmfp4(w, "dual")),
+                               ("rocmfp4_fast", 4.25, lambda w: W4.pack_rocmfp4(w, "fast")),
+                               ("q4_0", 4.5, lambda w: W4.pack_q4_0(w))):
+            e, q = W4.reconstruction_error(pack(W), W)
+            row[fmt] = {"rel_sq_error": float(f"{e / q:.6g}"), "bits_per_weight": bpw}
+        out[name] = row
+        del W
+    return out
+
+
 def pack_bench(W4, I):
     out = {}
     W = I.sweep_weights(2560, 9728, 3, device="cuda")
@@ -363,6 +383,16 @@ def pack_bench(W4, I):
         ms = a.elapsed_time(b)
         out[f"pack_rocmfp4_{fmt}"] = {"shape": "K=2560 N=9728 Laplace", "ms": round(ms, 3),
                                       "candidate_evals/s": round(127 * L.numel() / ms / 1e3, 1)}
+    W4.pack_q4_0(L)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    W4.pack_q4_0(L)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    out["pack_q4_0"] = {"shape": "K=2560 N=9728 Laplace", "us": round(ms * 1e3, 2),
+                        "GB/s": round((L.numel() * 2 + L.numel() * 0.5625) / ms / 1e6, 1)}
     imp = torch.rand(L.shape[1], generator=torch.Generator().manual_seed(5)).cuda() * 2.0
     W4.pack_rocmfp4(L, "dual", importance=imp)
     W4.pack_nvfp4(W, scale_search=W4.SCALE_MSE)
@@ -509,6 +539,8 @@ def run_ours(args, world, rank, local):
         extras["gemm"] = gemm_bench(W4, I, pk)
         torch.cuda.empty_cache()
         extras["packers"] = pack_bench(W4, I)
+        torch.cuda.empty_cache()
+        extras["quality"] = quality_report(W4, I)
         torch.cuda.empty_cache()
         extras["rocm_gemv"] = rocm_gemv_bench(W4, I, pk)
         torch.cuda.empty_cache()

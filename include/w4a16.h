@@ -58,7 +58,8 @@ typedef enum {
 typedef enum {
     W4_FMT_NVFP4 = 1,         /* [EdgeRock] E2M1 + E4M3 per 16 + FP32 global */
     W4_FMT_ROCMFP4_DUAL = 2,  /* [rocmwhy] 18-byte blocks, two half scales   */
-    W4_FMT_ROCMFP4_FAST = 3   /* [rocmwhy] 17-byte blocks, one scale         */
+    W4_FMT_ROCMFP4_FAST = 3,  /* [rocmwhy] 17-byte blocks, one scale         */
+    W4_FMT_Q4_0 = 4           /* [rocmwhy] table: stock Q4_0, for comparison  */
 } w4_format;
 
 typedef enum {
@@ -80,6 +81,12 @@ typedef enum {
  *                     code[j] | code[j+16] << 4.  Code = Codebook10 nibble (bit
  *                     3 sign, bits 2..0 index into 0,1,2,3,4,6,8,10).  Scale =
  *                     unsigned E4M3 byte 0x00..0x7E.  w_hat = level * scale.
+ *            scales = NULL, global_scale = NULL.
+ *   Q4_0:    codes  = [N][K/32] blocks of 18 bytes: the FP16 scale d (little
+ *                     endian), then 16 code bytes, byte j = code[j] |
+ *                     code[j+16] << 4; w_hat = d * (code - 8).  A comparison
+ *                     format: packed and scored (w4_reconstruction_error), not
+ *                     accepted by the matmuls (W4_ERR_UNSUPPORTED).
  *            scales = NULL, global_scale = NULL.
  */
 typedef struct {
@@ -161,6 +168,35 @@ size_t pack_nvfp4_workspace_bytes(void);
 w4_status pack_rocmfp4(const void *W, int K, int N, int block, int fmt,
                        const float *importance, uint8_t *blocks, int *d_status,
                        void *stream);
+
+/*
+ * pack_q4_0 -- stock Q4_0, the pages' comparison format ([rocmwhy] format
+ * table: 32 weights, evenly spaced integers, one FP16 scale, 18-byte blocks,
+ * "signed abs-max" reference scale; section 02's lab: the outlier 8.2 gives the
+ * shared scale 1.025 = 8.2 / 8).  Per 32-weight block: m = the weight of
+ * largest magnitude (the first in k order on ties), d = FP16(m / -8) (binary32
+ * division, then nearest even, saturating at 65504), code = the nearest
+ * integer (ties to even) of x / d in binary32, clamped to [-8, 7], plus 8;
+ * d == 0 gives codes 8.
+ *   W        [N][K] BF16, K % 32 == 0.  block must be 32.
+ *   blocks   out [N][K/32][18] (layout as in w4_weights).
+ *   d_status optional, as for pack_nvfp4.
+ */
+w4_status pack_q4_0(const void *W, int K, int N, int block, uint8_t *blocks, int *d_status,
+                    void *stream);
+
+/*
+ * w4_reconstruction_error -- how well a packed matrix reproduces its source:
+ * out[0] = sum over all weights of (W - w_hat)^2, out[1] = sum of W^2, both in
+ * binary64 (w_hat exact in binary64 for every format), summed in a fixed order
+ * (the same bits on every call).  Any w4_format, including W4_FMT_Q4_0.
+ *   W          [N][K] BF16, the matrix w was packed from.
+ *   out        device double[2].
+ *   workspace  >= w4_reconstruction_workspace_bytes() bytes of device scratch.
+ */
+w4_status w4_reconstruction_error(const w4_weights *w, const void *W, double *out, void *workspace,
+                                  size_t workspace_bytes, void *stream);
+size_t w4_reconstruction_workspace_bytes(void);
 
 /* ---------------------------------------------------------------- matmul --- */
 

@@ -23,13 +23,14 @@ from typing import Optional
 import torch
 
 __all__ = [
-    "W4Error", "PackedWeights", "FMT_NVFP4", "FMT_ROCMFP4_DUAL", "FMT_ROCMFP4_FAST",
+    "W4Error", "PackedWeights", "FMT_NVFP4", "FMT_ROCMFP4_DUAL", "FMT_ROCMFP4_FAST", "FMT_Q4_0",
+    "pack_q4_0", "reconstruction_error",
     "LAUNCH_PDL", "LAUNCH_TMEM", "LAUNCH_FP4_MMA", "pack_nvfp4", "pack_rocmfp4", "w4a16_gemv", "w4a16_gemv_grouped", "w4a16_gemm",
     "w4a16_workspace_bytes", "pack_nvfp4_workspace_bytes", "w4_encode_scalars",
     "w4_device_error", "lib", "library_path",
 ]
 
-FMT_NVFP4, FMT_ROCMFP4_DUAL, FMT_ROCMFP4_FAST = 1, 2, 3
+FMT_NVFP4, FMT_ROCMFP4_DUAL, FMT_ROCMFP4_FAST, FMT_Q4_0 = 1, 2, 3, 4
 SCALE_ABSMAX, SCALE_MSE = 0, 1
 LAUNCH_PDL = 1
 LAUNCH_TMEM = 2   # opt-in tcgen05 GEMV for one token (see include/w4a16.h)
@@ -73,6 +74,9 @@ def lib():
         sig = {
             "pack_nvfp4": ([P, I, I, I, I, P, P, P, P, S, P, P], I),
             "pack_nvfp4_ex": ([P, I, I, I, I, P, P, P, P, P, S, P, P], I),
+            "pack_q4_0": ([P, I, I, I, P, P, P], I),
+            "w4_reconstruction_error": ([WP, P, P, P, S, P], I),
+            "w4_reconstruction_workspace_bytes": ([], S),
             "pack_nvfp4_workspace_bytes": ([], S),
             "pack_rocmfp4": ([P, I, I, I, I, P, P, P, P], I),
             "w4a16_gemv": ([WP, P, I, P, P, S, P], I),
@@ -185,6 +189,32 @@ def pack_rocmfp4(W: torch.Tensor, fmt="dual", *, importance: Optional[torch.Tens
                               _stream(stream)),
            "pack_rocmfp4")
     return PackedWeights(fmt, K, N, out)
+
+
+def pack_q4_0(W: torch.Tensor, *, out: Optional[torch.Tensor] = None, d_status: Optional[torch.Tensor] = None,
+              stream=None) -> PackedWeights:
+    """Stock Q4_0, the comparison format (see pack_q4_0 in include/w4a16.h)."""
+    _cuda(W, "W", torch.bfloat16)
+    N, K = W.shape
+    if out is None:
+        out = torch.empty(N, K // 32, 18, dtype=torch.uint8, device=W.device)
+    _check(lib().pack_q4_0(_ptr(W), K, N, 32, _ptr(out), _ptr(d_status), _stream(stream)), "pack_q4_0")
+    return PackedWeights(FMT_Q4_0, K, N, out)
+
+
+def reconstruction_error(w: PackedWeights, W: torch.Tensor, *, workspace: Optional[torch.Tensor] = None,
+                         stream=None):
+    """(sum (W - w_hat)^2, sum W^2) in binary64 for a packed matrix and its bf16
+    source (see w4_reconstruction_error); reads the two numbers back to the host."""
+    _cuda(W, "W", torch.bfloat16)
+    out = torch.empty(2, dtype=torch.float64, device=W.device)
+    if workspace is None:
+        workspace = torch.empty(lib().w4_reconstruction_workspace_bytes(), dtype=torch.uint8, device=W.device)
+    s = w.struct()
+    _check(lib().w4_reconstruction_error(ctypes.byref(s), _ptr(W), _ptr(out), _ptr(workspace), workspace.numel(),
+                                         _stream(stream)), "w4_reconstruction_error")
+    e, q = out.tolist()
+    return e, q
 
 
 def w4a16_workspace_bytes(w: PackedWeights, M: int) -> int:

@@ -301,6 +301,140 @@ __global__ void __launch_bounds__(256) nvfp4_search_kernel(const uint16_t *__res
     }
 }
 
+// ---------------------------------------------------------------- Q4_0 ----
+// Stock Q4_0, the pages' comparison format ("rocmwhy" format table and section
+// 02): one thread per 32-weight block; m = the first weight of largest
+// magnitude, d = FP16(m / -8) saturating at 65504, code = clamp(RNE(x / d),
+// -8, 7) + 8 in binary32, d == 0 -> codes 8.  Block = [d lo, d hi, 16 code
+// bytes], code byte j = code[j] | code[j+16] << 4.
+__global__ void __launch_bounds__(256) q4_0_pack_kernel(const uint4 *__restrict__ W, long long nblk,
+                                                        uint8_t *__restrict__ out, int *__restrict__ d_status) {
+    for (long long b = blockIdx.x * (long long)blockDim.x + threadIdx.x; b < nblk;
+         b += (long long)gridDim.x * blockDim.x) {
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const uint4 v = __ldg(W + 4 * b + i);
+            w[4 * i] = v.x, w[4 * i + 1] = v.y, w[4 * i + 2] = v.z, w[4 * i + 3] = v.w;
+        }
+        float x[32];
+        int jm = 0;
+        bool bad = false;
+#pragma unroll
+        for (int j = 0; j < 32; j++) {
+            x[j] = (j & 1) ? bf16_hi(w[j >> 1]) : bf16_lo(w[j >> 1]);
+            bad |= !isfinite(x[j]);
+        }
+        if (bad) {
+            if (d_status) atomicExch(d_status, W4_ERR_NONFINITE);
+            record_error(W4_ERR_NONFINITE);
+        }
+        float am = fabsf(x[0]);
+#pragma unroll
+        for (int j = 1; j < 32; j++)
+            if (fabsf(x[j]) > am) {
+                am = fabsf(x[j]);
+                jm = j;
+            }
+        const float dq = fminf(fmaxf(__fdiv_rn(x[jm], -8.0f), -65504.0f), 65504.0f);
+        const __half h = __float2half_rn(dq);
+        const float d = __half2float(h);
+        uint32_t code[32];
+#pragma unroll
+        for (int j = 0; j < 32; j++) {
+            float q = 0.0f;
+            if (d != 0.0f) q = fminf(fmaxf(rintf(__fdiv_rn(x[j], d)), -8.0f), 7.0f);
+            code[j] = (uint32_t)((int)q + 8);
+        }
+        uint8_t *o = out + b * 18;
+        const uint16_t hb = __half_as_ushort(h);
+        o[0] = (uint8_t)(hb & 0xFF);
+        o[1] = (uint8_t)(hb >> 8);
+#pragma unroll
+        for (int j = 0; j < 16; j++) o[2 + j] = (uint8_t)(code[j] | (code[j + 16] << 4));
+    }
+}
+
+// ------------------------------------------------------ reconstruction error ----
+// Sum over a packed matrix of (W - w_hat)^2 and W^2 in binary64: one 32-weight
+// block per thread step, a fixed-order block reduction to one partial per
+// CTA, then one thread adds the partials in order.
+constexpr int kReconMaxGrid = 1024;
+
+__device__ __forceinline__ double e2m1_value(uint32_t c) {
+    const double m[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+    return (c & 8u) ? -m[c & 7u] : m[c & 7u];
+}
+__device__ __forceinline__ double cb10_value(uint32_t c) {
+    const double m[8] = {0.0, 1.0, 2.0, 3.0, 4.0, 6.0, 8.0, 10.0};
+    return (c & 8u) ? -m[c & 7u] : m[c & 7u];
+}
+
+__global__ void __launch_bounds__(256) recon_partial_kernel(int fmt, int K, long long nblk,
+                                                            const uint8_t *__restrict__ codes,
+                                                            const uint8_t *__restrict__ scales,
+                                                            const float *__restrict__ gscale,
+                                                            const uint16_t *__restrict__ W,
+                                                            double2 *__restrict__ partial) {
+    const int nb = K / 32;
+    const double g = fmt == W4_FMT_NVFP4 ? (double)__ldg(gscale) : 1.0;
+    double se = 0.0, sq = 0.0;
+    for (long long blk = blockIdx.x * (long long)blockDim.x + threadIdx.x; blk < nblk;
+         blk += (long long)gridDim.x * blockDim.x) {
+        const long long n = blk / nb;
+        const int b = (int)(blk % nb);
+        for (int j = 0; j < 32; j++) {
+            const long long k = 32LL * b + j;
+            const double x = (double)__uint_as_float((uint32_t)__ldg(W + n * K + k) << 16);
+            double wh;
+            if (fmt == W4_FMT_NVFP4) {
+                const uint32_t byte = __ldg(codes + n * (K / 2) + k / 2);
+                const uint32_t c = (k & 1) ? (byte >> 4) : (byte & 15u);
+                wh = e2m1_value(c) * (double)e4m3_to_f32(__ldg(scales + n * (K / 16) + k / 16)) * g;
+            } else {
+                const int bb = fmt == W4_FMT_ROCMFP4_FAST ? 17 : 18;
+                const uint8_t *p = codes + blk * bb;
+                const int c0 = fmt == W4_FMT_ROCMFP4_FAST ? 1 : 2;
+                const uint32_t byte = __ldg(p + c0 + (j & 15));
+                const uint32_t c = j < 16 ? (byte & 15u) : (byte >> 4);
+                if (fmt == W4_FMT_Q4_0) {
+                    const uint16_t hb = (uint16_t)(__ldg(p) | (__ldg(p + 1) << 8));
+                    wh = (double)__half2float(__ushort_as_half(hb)) * (double)((int)c - 8);
+                } else {
+                    const uint32_t sb = (fmt == W4_FMT_ROCMFP4_DUAL && j >= 16) ? __ldg(p + 1) : __ldg(p);
+                    wh = cb10_value(c) * (double)e4m3_to_f32(sb);
+                }
+            }
+            const double e = x - wh;
+            se += e * e;
+            sq += x * x;
+        }
+    }
+    __shared__ double2 red[256];
+    red[threadIdx.x] = make_double2(se, sq);
+    __syncthreads();
+    for (int o = 128; o; o >>= 1) {
+        if ((int)threadIdx.x < o) {
+            red[threadIdx.x].x += red[threadIdx.x + o].x;
+            red[threadIdx.x].y += red[threadIdx.x + o].y;
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) partial[blockIdx.x] = red[0];
+}
+
+__global__ void recon_final_kernel(const double2 *__restrict__ partial, int n, double *__restrict__ out) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) {
+        double se = 0.0, sq = 0.0;
+        for (int i = 0; i < n; i++) {
+            se += partial[i].x;
+            sq += partial[i].y;
+        }
+        out[0] = se;
+        out[1] = sq;
+    }
+}
+
 // Elementwise conversion check kernel (the packers' encoders on raw floats).
 __global__ void encode_scalars_kernel(const float *__restrict__ v, long long n, uint8_t *__restrict__ e4,
                                       uint8_t *__restrict__ e2) {

@@ -623,10 +623,22 @@ w4_status check_weights(const w4_weights *w) {
     } else if (w->fmt == W4_FMT_ROCMFP4_DUAL || w->fmt == W4_FMT_ROCMFP4_FAST) {
         if (w->K % 32) return W4_ERR_ARG;
         if (!aligned16(w->codes)) return W4_ERR_ALIGN;
+    } else if (w->fmt == W4_FMT_Q4_0) {
+        return W4_ERR_UNSUPPORTED;   // a comparison format: packed and scored, not multiplied
     } else {
         return W4_ERR_ARG;
     }
     return W4_OK;
+}
+
+// As check_weights, for entry points that accept every format (Q4_0 included).
+w4_status check_weights_any(const w4_weights *w) {
+    if (w && w->fmt == W4_FMT_Q4_0) {
+        if (!w->codes || w->K <= 0 || w->N <= 0 || w->K % 32) return W4_ERR_ARG;
+        if (!aligned16(w->codes)) return W4_ERR_ALIGN;
+        return W4_OK;
+    }
+    return check_weights(w);
 }
 
 }  // namespace
@@ -709,6 +721,39 @@ w4_status pack_rocmfp4(const void *W, int K, int N, int block, int fmt, const fl
         else
             rocm_pack_kernel<false, false><<<grid, 256, 0, st>>>(w16, nblk, K, nullptr, blocks, d_status);
     }
+    return launch_status();
+}
+
+w4_status pack_q4_0(const void *W, int K, int N, int block, uint8_t *blocks, int *d_status, void *stream) {
+    if (!W || !blocks || K < 32 || N < 1 || K % 32 || block != 32) return W4_ERR_ARG;
+    if (!aligned16(W) || !aligned16(blocks) || (reinterpret_cast<uintptr_t>(d_status) & 3)) return W4_ERR_ALIGN;
+    DeviceInfo d;
+    if (device_info(d) != W4_OK) return W4_ERR_CUDA;
+    cudaStream_t st = as_stream(stream);
+    if (d_status && cudaMemsetAsync(d_status, 0, sizeof(int), st) != cudaSuccess) return W4_ERR_CUDA;
+    const long long nblk = (long long)K * N / 32;
+    const int grid = (int)std::min<long long>((nblk + 255) / 256, (long long)d.sms * 16);
+    q4_0_pack_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4 *>(W), nblk, blocks, d_status);
+    return launch_status();
+}
+
+size_t w4_reconstruction_workspace_bytes(void) { return (size_t)kReconMaxGrid * sizeof(double2); }
+
+w4_status w4_reconstruction_error(const w4_weights *w, const void *W, double *out, void *workspace,
+                                  size_t workspace_bytes, void *stream) {
+    w4_status s = check_weights_any(w);
+    if (s != W4_OK) return s;
+    if (!W || !out) return W4_ERR_ARG;
+    if (w->K % 32) return W4_ERR_UNSUPPORTED;
+    if (!workspace || workspace_bytes < w4_reconstruction_workspace_bytes()) return W4_ERR_WORKSPACE;
+    if (!aligned16(W) || !aligned16(out) || !aligned16(workspace)) return W4_ERR_ALIGN;
+    cudaStream_t st = as_stream(stream);
+    const long long nblk = (long long)w->K * w->N / 32;
+    const int grid = (int)std::min<long long>((nblk + 255) / 256, kReconMaxGrid);
+    recon_partial_kernel<<<grid, 256, 0, st>>>(w->fmt, w->K, nblk, w->codes, w->scales, w->global_scale,
+                                               reinterpret_cast<const uint16_t *>(W),
+                                               reinterpret_cast<double2 *>(workspace));
+    recon_final_kernel<<<1, 32, 0, st>>>(reinterpret_cast<const double2 *>(workspace), grid, out);
     return launch_status();
 }
 
