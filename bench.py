@@ -8,16 +8,19 @@ GEMV sweep -- NVFP4 weights of the 4B-class decoder shapes (K, N) = (2560,4096),
 over each of the five matrices, issued as one grouped launch
 (w4a16_gemv_grouped), six steps (one per rotating weight copy) captured in one
 CUDA graph; the same sweep as five separate launches chained with programmatic
-dependent launch is reported beside it.
-GB/s counts the packed bytes read (codes +
-scales + global scale, 4.5 bits per weight).  Six packed copies of every matrix
-rotate across steps (248 MB > the 126 MB L2), so no step finds its weights in
-L2.
+dependent launch is reported beside it.  GB/s counts the packed bytes read
+(codes + scales + global scale, 4.5 bits per weight).  Six packed copies of
+every matrix rotate across steps (248 MB > the 126 MB L2), so no step finds its
+weights in L2.
 
 The same line carries the other rows of the path, each measured in this run:
-the prefill GEMM (M=2048, K=2560, N=9728, TFLOP/s), the 36-layer weight stream
-(tokens/s at M=1, M=16 and looped), each sweep shape timed alone, and the two
-packers.  `--impl reference` times the CPU oracle on the same workload instead.
+the sweep at M = 4, 9 (speculative verify) and 16, the prefill GEMM (M=2048,
+K=2560, N=9728, TFLOP/s), the 36-layer weight stream (tokens/s at M=1, M=16
+and looped; at M=1 also with q/k/v and gate/up grouped), each sweep shape timed
+alone, the ROCmFP4 GEMV, the packers (NVFP4 abs-max and scale search, ROCmFP4
+Dual / FAST, importance-weighted, Q4_0), and the reconstruction-error quality
+report of every format.  `--impl reference` times the CPU oracle on the same
+workload instead.
 
 Multi-GPU: the path has no exchange step; `--gpus N` under torchrun runs N
 independent replicas (weak scaling) and reports the summed bytes over the
