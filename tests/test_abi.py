@@ -52,6 +52,21 @@ def test_host_validation_without_gpu(lib):
     assert lib.pack_rocmfp4(P(16), 48, 4, 32, 2, None, P(16), None, None) == 1
     assert lib.pack_rocmfp4(P(16), 64, 4, 32, 9, None, P(16), None, None) == 1
     assert lib.pack_rocmfp4(P(16), 64, 4, 32, 2, P(20), P(16), None, None) == 2
+    # the Q4_0 packer and the reconstruction report
+    assert lib.pack_q4_0(P(16), 64, 4, 16, P(16), None, None) == 1          # block must be 32
+    assert lib.pack_q4_0(P(16), 48, 4, 32, P(16), None, None) == 1          # K % 32
+    assert lib.pack_q4_0(P(16), 64, 4, 32, P(24), None, None) == 2          # alignment
+    q = W4._Weights(4, 64, 4, 16, None, None)
+    ws = lib.w4_reconstruction_workspace_bytes()
+    assert ws >= 16
+    assert lib.w4_reconstruction_error(ctypes.byref(q), None, P(16), P(16), ws, None) == 1
+    assert lib.w4_reconstruction_error(ctypes.byref(q), P(16), P(16), P(16), ws - 1, None) == 7
+    assert lib.w4_reconstruction_error(ctypes.byref(q), P(16), P(24), P(16), ws, None) == 2
+    bad_k = W4._Weights(4, 48, 4, 16, None, None)
+    assert lib.w4_reconstruction_error(ctypes.byref(bad_k), P(16), P(16), P(16), ws, None) == 1
+    # Q4_0 is scored, not multiplied
+    assert lib.w4a16_gemv(ctypes.byref(q), P(16), 1, P(16), None, 0, None) == 3
+    assert lib.w4a16_gemm(ctypes.byref(q), P(16), 64, P(16), None, None, 0, None) == 3
     w = W4._Weights(1, 256, 8, 16, 16, 16)
     assert lib.w4a16_gemv(ctypes.byref(w), P(16), 17, P(16), None, 0, None) == 1
     assert lib.w4a16_gemv(ctypes.byref(w), P(16), 0, P(16), None, 0, None) == 1
