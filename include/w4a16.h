@@ -237,8 +237,10 @@ w4_status w4a16_gemv(const w4_weights *w, const void *x, int M, float *y,
  * unpacks them to the padded 4-bit operand layout), x is split per 16-k block
  * into three exact E5M2 parts, and the E4M3 block scales are applied per row
  * after the MMA (blocks whose x cannot be split exactly are summed in
- * binary32).  Also accepted by w4a16_gemv_grouped, where it applies when every
- * problem qualifies.
+ * binary64).  Also accepted by w4a16_gemv_grouped, where it applies when every
+ * problem qualifies.  Results meet the same tolerance as the default path; on
+ * B200 it is currently slower than the default mma.sync kernel, so it is
+ * opt-in.
  */
 #define W4_LAUNCH_FP4_MMA 4u
 w4_status w4a16_gemv_ex(const w4_weights *w, const void *x, int M, float *y,
