@@ -268,6 +268,17 @@ w4_status w4a16_gemv_grouped(const w4_weights *w, const void *const *x, float *c
                              unsigned flags, void *stream);
 
 /*
+ * w4_plan_grouped -- host only (no CUDA call): the CTAs w4a16_gemv_grouped
+ * gives each problem on a GPU with `sms` SMs.  ctas[p] is proportional to
+ * problem p's packed bytes (rounded down; the spare SMs go one at a time to the
+ * problem with the most bytes per CTA), at least 1 and at most one per 16-row
+ * tile (one per 64 rows when W4_LAUNCH_FP4_MMA applies to every problem); the
+ * total is min(sms, sum of the maxima) unless G forces more.
+ *   w, G, flags  as for w4a16_gemv_grouped.  ctas  out int[G].
+ */
+w4_status w4_plan_grouped(const w4_weights *w, int G, int sms, unsigned flags, int *ctas);
+
+/*
  * w4a16_gemm -- y = x . w_hat for prefill-sized M: NVFP4 tiles are dequantised
  * to BF16 in shared memory (e2m1 * scale, exact in BF16) and multiplied on the
  * tensor cores with binary32 accumulation; the epilogue multiplies by the

@@ -24,7 +24,7 @@ import torch
 
 __all__ = [
     "W4Error", "PackedWeights", "FMT_NVFP4", "FMT_ROCMFP4_DUAL", "FMT_ROCMFP4_FAST", "FMT_Q4_0",
-    "pack_q4_0", "reconstruction_error",
+    "pack_q4_0", "reconstruction_error", "plan_grouped",
     "LAUNCH_PDL", "LAUNCH_TMEM", "LAUNCH_FP4_MMA", "pack_nvfp4", "pack_rocmfp4", "w4a16_gemv", "w4a16_gemv_grouped", "w4a16_gemm",
     "w4a16_workspace_bytes", "pack_nvfp4_workspace_bytes", "w4_encode_scalars",
     "w4_device_error", "lib", "library_path",
@@ -75,6 +75,7 @@ def lib():
             "pack_nvfp4": ([P, I, I, I, I, P, P, P, P, S, P, P], I),
             "pack_nvfp4_ex": ([P, I, I, I, I, P, P, P, P, P, S, P, P], I),
             "pack_q4_0": ([P, I, I, I, P, P, P], I),
+            "w4_plan_grouped": ([P, I, I, U, P], I),
             "w4_reconstruction_error": ([WP, P, P, P, S, P], I),
             "w4_reconstruction_workspace_bytes": ([], S),
             "pack_nvfp4_workspace_bytes": ([], S),
@@ -237,6 +238,16 @@ def w4a16_gemv(w: PackedWeights, x: torch.Tensor, *, out: Optional[torch.Tensor]
                                0 if workspace is None else workspace.numel(), flags, _stream(stream)),
            "w4a16_gemv")
     return out
+
+
+def plan_grouped(ws, sms: int, flags: int = 0):
+    """Host only: the CTAs w4a16_gemv_grouped gives each problem on `sms` SMs."""
+    G = len(ws)
+    structs = (_Weights * G)(*[w.struct() for w in ws])
+    out = (ctypes.c_int * G)()
+    _check(lib().w4_plan_grouped(ctypes.cast(structs, ctypes.c_void_p), G, sms, flags,
+                                 ctypes.cast(out, ctypes.c_void_p)), "w4_plan_grouped")
+    return list(out)
 
 
 def w4a16_gemv_grouped(ws, xs, *, outs=None, flags: int = 0, stream=None):

@@ -347,6 +347,13 @@ void share_sms(const w4_weights *w, int G, int sms, const int *max_cta, int *all
     }
 }
 
+// Most CTAs a grouped launch gives problem p: one per 16-row tile (decode
+// kernel) or one per 64 rows (the kind::f8f6f4 kernel), at least one.
+void grouped_max_cta(const w4_weights *w, int G, bool fp4, int *max_cta) {
+    for (int p = 0; p < G; p++)
+        max_cta[p] = fp4 ? std::max(1, w[p].N / 64) : (w[p].N + kTcRows - 1) / kTcRows;
+}
+
 // Several one-token NVFP4 problems in one launch (gemv_m1.cuh): the SMs are
 // shared out in proportion to each problem's packed bytes (at least one CTA
 // each, at most one per 16-row tile), and every CTA runs the single-problem
@@ -356,7 +363,7 @@ w4_status launch_gemv_grouped(const w4_weights *w, const void *const *x, float *
     DeviceInfo d;
     if (device_info(d) != W4_OK) return W4_ERR_CUDA;
     int tiles[kMaxGroup], alloc[kMaxGroup];
-    for (int p = 0; p < G; p++) tiles[p] = (w[p].N + kTcRows - 1) / kTcRows;
+    grouped_max_cta(w, G, false, tiles);
     share_sms(w, G, d.sms, tiles, alloc);
     static GroupArgs g;   // host staging of the kernel parameter (copied at launch)
     static std::mutex mu;
@@ -565,7 +572,7 @@ w4_status launch_f4_grouped(const w4_weights *w, const void *const *x, float *co
     DeviceInfo d;
     if (device_info(d) != W4_OK) return W4_ERR_CUDA;
     int max_cta[kMaxGroup], alloc[kMaxGroup];
-    for (int p = 0; p < G; p++) max_cta[p] = std::max(1, w[p].N / 64);
+    grouped_max_cta(w, G, true, max_cta);
     share_sms(w, G, d.sms, max_cta, alloc);
     int Kmax = 0;
     for (int p = 0; p < G; p++) Kmax = std::max(Kmax, w[p].K);
@@ -807,6 +814,22 @@ w4_status w4a16_gemv_ex(const w4_weights *w, const void *x, int M, float *y, voi
     case W4_FMT_ROCMFP4_FAST: return launch_gemv_fmt<W4_FMT_ROCMFP4_FAST>(w, x, M, y, workspace, p, pdl, st);
     }
     return W4_ERR_ARG;
+}
+
+w4_status w4_plan_grouped(const w4_weights *w, int G, int sms, unsigned flags, int *ctas) {
+    if (!w || !ctas || G < 1 || G > kMaxGroup || sms < 1 || (flags & ~(W4_LAUNCH_PDL | W4_LAUNCH_FP4_MMA)))
+        return W4_ERR_ARG;
+    bool f4 = (flags & W4_LAUNCH_FP4_MMA) != 0;
+    for (int p = 0; p < G; p++) {
+        const w4_status s = check_weights(&w[p]);
+        if (s != W4_OK) return s;
+        if (w[p].fmt != W4_FMT_NVFP4) return W4_ERR_UNSUPPORTED;
+        f4 = f4 && f4_applies(&w[p], 1);
+    }
+    int max_cta[kMaxGroup];
+    grouped_max_cta(w, G, f4, max_cta);
+    share_sms(w, G, sms, max_cta, ctas);
+    return W4_OK;
 }
 
 w4_status w4a16_gemv_grouped(const w4_weights *w, const void *const *x, float *const *y, int G, unsigned flags,
