@@ -81,3 +81,25 @@ def test_python_binding_refuses_cpu_tensors():
         W4.pack_nvfp4(torch.zeros(4, 64, dtype=torch.bfloat16))
     with pytest.raises(ValueError):
         W4.pack_rocmfp4(torch.zeros(4, 64, dtype=torch.bfloat16), "dual")
+
+
+def declared_parameter_counts():
+    """name -> number of parameters, from the prototypes in include/w4a16.h."""
+    text = open(os.path.join(ROOT, "include", "w4a16.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    out = {}
+    for m in re.finditer(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*([a-z_0-9]+)\s*\(([^)]*)\)\s*;", text, re.M):
+        params = " ".join(m.group(2).split())
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_signatures_match_the_header(lib):
+    """Every function the Python binding declares to ctypes takes as many
+    arguments as its prototype in the header."""
+    counts = declared_parameter_counts()
+    bound = [n for n in counts if getattr(lib, n).argtypes is not None]
+    assert {"pack_nvfp4_ex", "pack_q4_0", "w4a16_gemv_grouped", "w4_plan_grouped",
+            "w4_reconstruction_error"} <= set(bound)
+    for name in bound:
+        assert len(getattr(lib, name).argtypes) == counts[name], name
