@@ -533,21 +533,26 @@ def run_ours(args, world, rank, local):
                    "C ABI (no graph), 5 y -> pinned host, synchronize; packed weights resident"}
 
     extras = {}
+
+    def extra(name, fn):
+        # one failing side measurement is recorded, not allowed to lose the headline line
+        try:
+            extras[name] = fn()
+        except Exception as e:  # noqa: BLE001
+            extras[name] = {"error": f"{type(e).__name__}: {e}"[:300]}
+        torch.cuda.empty_cache()
+
     if not args.no_extras:
-        extras["sweep_separate_launches"] = separate_sweep(W4, mats)
-        extras["per_shape_isolated"] = per_shape(W4, mats)
-        extras["sweep_skinny"] = sweep_m_bench(W4, I, mats, pk)
-        del graphs, mats
+        extra("sweep_separate_launches", lambda: separate_sweep(W4, mats))
+        extra("per_shape_isolated", lambda: per_shape(W4, mats))
+        extra("sweep_skinny", lambda: sweep_m_bench(W4, I, mats, pk))
+        del graphs, graph_rot, mats
         torch.cuda.empty_cache()
-        extras["gemm"] = gemm_bench(W4, I, pk)
-        torch.cuda.empty_cache()
-        extras["packers"] = pack_bench(W4, I)
-        torch.cuda.empty_cache()
-        extras["quality"] = quality_report(W4, I)
-        torch.cuda.empty_cache()
-        extras["rocm_gemv"] = rocm_gemv_bench(W4, I, pk)
-        torch.cuda.empty_cache()
-        extras["stream"] = stream_bench(W4, I)
+        extra("gemm", lambda: gemm_bench(W4, I, pk))
+        extra("packers", lambda: pack_bench(W4, I))
+        extra("quality", lambda: quality_report(W4, I))
+        extra("rocm_gemv", lambda: rocm_gemv_bench(W4, I, pk))
+        extra("stream", lambda: stream_bench(W4, I))
     err = W4.w4_device_error(clear=True)
 
     cpu = None
