@@ -43,3 +43,26 @@ def test_rocm_search_is_the_minimum_and_uniform_weights_change_nothing(x, c):
     cw = np.full(x.size, np.float32(2.0) ** int(np.round(np.log2(c))), np.float32)   # a power of two: exact
     uw, ew = O.rocm_search(x, cw)
     assert uw == u and ew == e * float(cw[0])
+
+
+@settings(max_examples=60, deadline=None)
+@given(x=st.lists(finite_bf16, min_size=32, max_size=32))
+def test_q4_0_block_properties(x):
+    """Stock Q4_0 ("rocmwhy" format table; signed abs-max scale, integer steps):
+    the largest weight sits at -8, every code is the nearest integer step to its
+    weight within the clamp, and the block reconstructs within half a step."""
+    W = torch.tensor([x], dtype=torch.float32).to(torch.bfloat16)
+    blk = O.pack_q4_0(W)[0, 0]
+    d = O.fp16_decode(int(blk[0]) | int(blk[1]) << 8)
+    codes = [int(blk[2 + (j & 15)] >> (4 * (j >> 4))) & 15 for j in range(32)]
+    xs = W.float().numpy()[0]
+    jm = int(np.argmax(np.abs(xs)))
+    if d == 0.0:
+        assert all(c == 8 for c in codes)
+        return
+    assert codes[jm] == 0
+    wh = O.dequant_q4_0(O.pack_q4_0(W))[0]
+    for j in range(32):
+        q = float(xs[j]) / d
+        if -8.0 <= q <= 7.0:
+            assert abs(float(xs[j]) - wh[j]) <= abs(d) * (0.5 + 1e-6)
