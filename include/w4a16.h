@@ -203,13 +203,21 @@ size_t w4_reconstruction_workspace_bytes(void);
 /*
  * w4a16_gemv -- y[M][N] = x[M][K] . w_hat, fused dequantise-and-multiply for
  * decode-sized M ([Nanbeige] Serving: the W4A16 kernel a decode step spends its
- * weight bandwidth on).  Products and sums are binary32; the NVFP4 global scale
- * is applied once per output.  The result is deterministic (fixed summation
- * order for a given shape).
- *   w        packed weights (any format); K % 32 == 0.
+ * weight bandwidth on).  NVFP4: products on the tensor cores from f16 operands
+ * (e2m1 * scale is exact in f16; x is rescaled by powers of two into f16's range,
+ * with a binary32 CUDA-core path for x that does not convert exactly), binary32
+ * accumulation; the global scale and the power of two are applied together at
+ * the end in binary64, so the output is finite whenever the exact result is.
+ * ROCmFP4: level * scale products in binary32.  The result is deterministic (a
+ * fixed summation order for a given shape and M).
+ *   w        packed NVFP4 or ROCmFP4 weights (Q4_0: W4_ERR_UNSUPPORTED).
+ *            K % 256 == 0 (NVFP4, ROCmFP4 Dual) or K % 512 == 0 (ROCmFP4 FAST),
+ *            so that every row piece the kernels copy starts on 16 bytes;
+ *            other K return W4_ERR_UNSUPPORTED.
  *   x        [M][K] BF16, 1 <= M <= 16.
  *   y        out [M][N] float.
- *   workspace>= w4a16_workspace_bytes(w, M) bytes (may be 0 -> NULL allowed).
+ *   workspace>= w4a16_workspace_bytes(w, M) bytes (0 for most shapes: NULL
+ *            allowed then); the split-K partial sums of long K at large M.
  */
 w4_status w4a16_gemv(const w4_weights *w, const void *x, int M, float *y,
                      void *workspace, size_t workspace_bytes, void *stream);
@@ -219,30 +227,9 @@ w4_status w4a16_gemv(const w4_weights *w, const void *x, int M, float *y,
  * kernel with programmatic dependent launch: it may start streaming weights
  * while the previous kernel on the stream is still running, and reads x only
  * after that kernel has completed.  Use inside a captured CUDA graph of
- * back-to-back layers.
+ * back-to-back layers.  Any other bit returns W4_ERR_ARG.
  */
 #define W4_LAUNCH_PDL 1u
-/*
- * W4_LAUNCH_TMEM (NVFP4, M == 1, K % 512 == 0, K <= 12288; otherwise ignored)
- * selects the GEMV whose products run on tcgen05.mma with the decoded weights
- * in tensor memory (A from TMEM, x from shared memory).  Results meet the same
- * tolerance as the default path; on B200 it is currently slower than the
- * default mma.sync kernel, so it is opt-in.
- */
-#define W4_LAUNCH_TMEM 2u
-/*
- * W4_LAUNCH_FP4_MMA (NVFP4, M == 1, K % 256 == 0, N % 8 == 0, codes 32-byte
- * aligned; otherwise ignored) runs the one-token GEMV on tcgen05.mma
- * kind::f8f6f4: the packed E2M1 codes go to the tensor cores as stored (TMA
- * unpacks them to the padded 4-bit operand layout), x is split per 16-k block
- * into three exact E5M2 parts, and the E4M3 block scales are applied per row
- * after the MMA (blocks whose x cannot be split exactly are summed in
- * binary64).  Also accepted by w4a16_gemv_grouped, where it applies when every
- * problem qualifies.  Results meet the same tolerance as the default path; on
- * B200 it is currently slower than the default mma.sync kernel, so it is
- * opt-in.
- */
-#define W4_LAUNCH_FP4_MMA 4u
 w4_status w4a16_gemv_ex(const w4_weights *w, const void *x, int M, float *y,
                         void *workspace, size_t workspace_bytes, unsigned flags,
                         void *stream);
@@ -259,7 +246,7 @@ w4_status w4a16_gemv_ex(const w4_weights *w, const void *x, int M, float *y,
  *   x      array of G device pointers to [K_p] BF16 (may repeat).
  *   y      array of G device pointers to [N_p] float (must not overlap).
  *   G      1..8.
- *   flags  0, W4_LAUNCH_PDL and / or W4_LAUNCH_FP4_MMA.
+ *   flags  0 or W4_LAUNCH_PDL.
  * The arrays are read on the host before the call returns; no workspace.
  * Errors: W4_ERR_ARG (null pointers, G out of range, unknown flags),
  * W4_ERR_ALIGN, W4_ERR_UNSUPPORTED (format or K), W4_ERR_CUDA.
@@ -272,21 +259,31 @@ w4_status w4a16_gemv_grouped(const w4_weights *w, const void *const *x, float *c
  * gives each problem on a GPU with `sms` SMs.  ctas[p] is proportional to
  * problem p's packed bytes (rounded down; the spare SMs go one at a time to the
  * problem with the most bytes per CTA), at least 1 and at most one per 16-row
- * tile (one per 64 rows when W4_LAUNCH_FP4_MMA applies to every problem); the
- * total is min(sms, sum of the maxima) unless G forces more.
+ * tile; the total is min(sms, sum of the maxima) unless G forces more.
  *   w, G, flags  as for w4a16_gemv_grouped.  ctas  out int[G].
  */
 w4_status w4_plan_grouped(const w4_weights *w, int G, int sms, unsigned flags, int *ctas);
 
 /*
- * w4a16_gemm -- y = x . w_hat for prefill-sized M: NVFP4 tiles are dequantised
- * to BF16 in shared memory (e2m1 * scale, exact in BF16) and multiplied on the
- * tensor cores with binary32 accumulation; the epilogue multiplies by the
- * global scale and writes binary32 and/or BF16 (round to nearest even).
- *   w        NVFP4 weights, K % 128 == 0.
+ * w4a16_gemm -- y = x . w_hat for prefill-sized M on the 5th-generation tensor
+ * cores (tcgen05.mma kind::f16, binary32 accumulators in tensor memory).  The
+ * packed NVFP4 tiles are dequantised (e2m1 * scale, exact in f16 and in BF16)
+ * by CUDA-core warps straight into tensor memory, where they are the MMA's A
+ * operand; x tiles (the B operand) are staged in shared memory by TMA.  The
+ * epilogue applies the global scale (and the per-row power of two below) in
+ * binary64 and writes binary32 and/or BF16 (round to nearest even).
+ * Operands per 192-token tile: with a workspace, x_to_f16 first writes each
+ * token row as f16 x * 2^-sigma_m (exact for rows whose range fits f16); tiles
+ * whose rows all converted exactly run on f16 operands, any other tile (and
+ * every tile without a workspace) on BF16 operands, with g's power of two
+ * folded into the weights.
+ *   w        NVFP4 weights, K % 64 == 0 (W4_ERR_UNSUPPORTED otherwise; ROCmFP4
+ *            and Q4_0 are W4_ERR_UNSUPPORTED too).
  *   x        [M][K] BF16, M >= 1.
  *   y_f32    out [M][N] float, or NULL;  y_bf16 out [M][N] BF16, or NULL
  *            (at least one of the two).
+ *   workspace NULL, or >= w4a16_workspace_bytes(w, M) bytes: the f16 copy of x
+ *            and two ints per row (smaller or NULL: BF16 operands throughout).
  */
 w4_status w4a16_gemm(const w4_weights *w, const void *x, int M, float *y_f32,
                      void *y_bf16, void *workspace, size_t workspace_bytes,
@@ -312,7 +309,10 @@ size_t w4a16_workspace_bytes(const w4_weights *w, int M);
  * caches it; make that first call before any stream capture.  All calls on a
  * device share the array: calls whose work overlaps on the GPU race and must
  * be serialised by the caller.  Every scratch value a call reads is written
- * earlier in the same call, so no clearing is needed between calls.
+ * earlier in the same call, so no clearing is needed between calls.  The cached
+ * address belongs to the device's current context: after cudaDeviceReset (or
+ * with another primary context on that device) it is stale, so the library must
+ * not be used across a reset in one process.
  */
 #define W4_NOALLOC_SCRATCH_BYTES (8u << 20)
 w4_status w4a16_gemv_noalloc(const w4_weights *w, const void *x, int M, float *y, void *stream);
@@ -335,6 +335,20 @@ w4_status w4_encode_scalars(const float *v, size_t n, uint8_t *e4m3, uint8_t *e2
  * Synchronises the device.
  */
 w4_status w4_device_error(int *out, int clear);
+
+/*
+ * w4_set_wait_limit -- limit, in nanoseconds, of the device-side waits that
+ * gate a kernel's progress (a consumer waiting for its data, a producer for a
+ * free buffer), on the current device; 0 restores the default of 2 s.  When
+ * such a wait expires the kernel records W4_ERR_TIMEOUT in the sticky word
+ * (w4_device_error), every other wait of its CTA returns at once, and the CTA
+ * runs to its end: before exiting it still waits (up to 2 s, whatever this
+ * limit) for the copies and MMAs it has already issued, so no asynchronous
+ * write outlives it.  The outputs of a call whose wait expired are undefined.
+ * Meant for exercising that failure path (a short limit makes the first waits
+ * expire); it applies to kernels launched after it returns.  Synchronous.
+ */
+w4_status w4_set_wait_limit(unsigned long long ns);
 
 /* Human-readable name of a status code. */
 const char *w4_status_string(int status);

@@ -106,3 +106,31 @@ def test_bf16_operands_without_workspace():
     x = I.activations(M, K, 14, outlier_cols=16)
     pw, cs = packed(W)
     check(pw, cs, x, workspace=torch.empty(0, dtype=torch.uint8, device="cuda"))
+
+
+@pytest.mark.parametrize("case", ["x_2p110", "x_2p118", "x_2p125_sparse", "w_2p100_x_2pm110"])
+@pytest.mark.parametrize("with_workspace", [True, False])
+def test_huge_range_outputs(case, with_workspace):
+    """Outputs near the top and bottom of binary32's range: the epilogue applies g
+    and 2^sigma in one binary64 product, and BF16-operand tiles fold g's exponent
+    into the weights, so nothing overflows before the result does."""
+    M, N, K = 256, 384, 2560
+    W = I.matrix("student_t4", N, K, 401, 0.02, 1e-3).double()
+    x = I.activations(M, K, 402).double()
+    if case == "x_2p110":
+        x *= 2.0 ** 110
+    elif case == "x_2p118":
+        x *= 2.0 ** 118
+    elif case == "x_2p125_sparse":
+        x[:, [k for k in range(K) if k % 160]] = 0.0
+        x *= 2.0 ** 125
+    else:
+        W *= 2.0 ** 100
+        x *= 2.0 ** -110
+    W, x = I.bf16_rne(W).contiguous(), I.bf16_rne(x).contiguous()
+    pw, cs = packed(W)
+    wh = O.dequant_nvfp4(*cs)
+    yr, ar = O.matmul(x, wh)
+    assert np.all(np.abs(yr) < 3.0e38)
+    ws = None if with_workspace else torch.empty(0, dtype=torch.uint8, device="cuda")
+    check(pw, cs, x, workspace=ws)

@@ -193,46 +193,6 @@ def test_single_token_block_exponents(case, K, N):
         assert_within_tolerance(y, yr, ar)
 
 
-@pytest.mark.parametrize("K,N", [(2560, 4096), (9728, 2560), (1024, 1024), (512, 7), (2560, 333), (9728, 2),
-                                 (12288, 5), (4096, 2560)])
-def test_tensor_memory_path(K, N):
-    """The opt-in tcgen05 GEMV (decoded weights in tensor memory) meets the same bound."""
-    pw, wh = nvfp4_packed(I.sweep_weights(K, N, 4)[:N].contiguous())
-    x = I.activations(1, K, 21).double()
-    x = I.bf16_rne(x)
-    for flags in (W4.LAUNCH_TMEM, W4.LAUNCH_TMEM | W4.LAUNCH_PDL):
-        run_and_check(pw, wh, x, flags=flags)
-
-
-@pytest.mark.parametrize("case", ["zeros", "scaled_up", "scaled_down", "wide_range", "inf"])
-def test_tensor_memory_path_ranges(case):
-    """x that the tensor-memory path converts exactly to f16 after scaling, and x it
-    cannot (the binary32 path of the same kernel)."""
-    K, N = 2560, 300
-    pw, wh = nvfp4_packed(I.sweep_weights(K, N, 5)[:N].contiguous())
-    x = I.activations(1, K, 22).double()
-    if case == "zeros":
-        x[:] = 0.0
-    elif case == "scaled_up":
-        x *= 2.0 ** 100
-    elif case == "scaled_down":
-        x *= 2.0 ** -100
-    elif case == "wide_range":
-        x[:, :8] *= 2.0 ** 40
-        x[:, 8:16] *= 2.0 ** -40
-    else:
-        x[:, 700] = float("inf")
-    x = I.bf16_rne(x)
-    y = np_of(W4.w4a16_gemv(pw, x.cuda(), flags=W4.LAUNCH_TMEM))
-    yr, ar = O.matmul(x, wh)
-    if case == "inf":
-        assert np.array_equal(np.isfinite(y), np.isfinite(yr))
-        fin = np.isfinite(yr)
-        assert_within_tolerance(y[fin], yr[fin], ar[fin])
-    else:
-        assert_within_tolerance(y, yr, ar)
-
-
 def check_group(pws, whs, xs, flags=0):
     ys = W4.w4a16_gemv_grouped(pws, [x.cuda() for x in xs], flags=flags)
     for y, wh, x in zip(ys, whs, xs):
@@ -297,114 +257,58 @@ def test_grouped_argument_errors():
     with pytest.raises(W4.W4Error):
         W4.w4a16_gemv_grouped([pw] * 9, [x] * 9)
     with pytest.raises(W4.W4Error):
-        W4.w4a16_gemv_grouped([pw], [x], flags=W4.LAUNCH_TMEM)
+        W4.w4a16_gemv_grouped([pw], [x], flags=2)
     pr = W4.pack_rocmfp4(I.matrix("laplace", 16, 256, 82, 0.015, 0.0, device="cuda"), "dual")
     with pytest.raises(W4.W4Error):
         W4.w4a16_gemv_grouped([pr], [x])
 
 
-@pytest.mark.parametrize("K,N", [(2560, 4096), (2560, 1024), (4096, 2560), (2560, 9728), (9728, 2560), (256, 8),
-                                 (512, 72), (1024, 136), (2560, 1000), (12288, 64), (2560, 333)])
-def test_fp4_mma_path(K, N):
-    """The one-token GEMV on kind::f8f6f4 (E2M1 codes unpacked by TMA, x in three
-    E5M2 parts per block) meets the bound; N % 8 != 0 takes the other kernel."""
-    pw, wh = nvfp4_packed(I.sweep_weights(K, N, 6)[:N].contiguous())
-    x = I.bf16_rne(I.activations(1, K, 23).double())
-    for flags in (W4.LAUNCH_FP4_MMA, W4.LAUNCH_FP4_MMA | W4.LAUNCH_PDL):
-        run_and_check(pw, wh, x, flags=flags)
+def huge_range_case(case, M, K, seed):
+    """x (and W) scaled so that the binary64 y is finite in binary32 while the
+    kernels' internal sums, taken without the global scale g, would not be:
+    rows of x at 2^110..2^125, or weights near 2^100 against x near 2^-110."""
+    W = I.sweep_weights(K, 512, 1)[:512].double()
+    x = I.activations(M, K, seed).double()
+    if case == "x_2p110":
+        x *= 2.0 ** 110
+    elif case == "x_2p118":
+        x *= 2.0 ** 118
+    elif case == "x_2p125_sparse":          # few nonzero x so that y stays below 2^128
+        keep = torch.zeros(K, dtype=torch.bool)
+        keep[::160] = True
+        x[:, ~keep] = 0.0
+        x *= 2.0 ** 125
+    elif case == "w_2p100_x_2pm110":
+        W *= 2.0 ** 100
+        x *= 2.0 ** -110
+    return I.bf16_rne(W), I.bf16_rne(x)
 
 
-@pytest.mark.parametrize("case", ["zeros", "one_block", "scaled_up", "scaled_down", "range_2p20", "wide_range",
-                                  "subnormal", "far_blocks", "inf", "nan"])
-def test_fp4_mma_ranges(case):
-    """Blocks split exactly into E5M2 parts, and blocks that are not (spread over
-    more than 2^23, a factor outside binary32's normal range, Inf / NaN), which
-    the epilogue sums in binary32."""
-    K, N = 2560, 392
-    pw, wh = nvfp4_packed(I.sweep_weights(K, N, 7)[:N].contiguous())
-    x = I.activations(1, K, 24).double()
-    if case == "zeros":
-        x[:] = 0.0
-    elif case == "one_block":
-        x[:] = 0.0
-        x[:, 16 * 19:16 * 20] = I.activations(1, 16, 25).double()
-    elif case == "scaled_up":
-        x *= 2.0 ** 100
-    elif case == "scaled_down":
-        x *= 2.0 ** -100
-    elif case == "range_2p20":        # inside one block, still exact
-        x[:, 16:24] *= 2.0 ** 10
-        x[:, 24:32] *= 2.0 ** -10
-    elif case == "wide_range":        # 2^80 inside one block: that block falls back
-        x[:, :8] *= 2.0 ** 40
-        x[:, 8:16] *= 2.0 ** -40
-    elif case == "subnormal":
-        x[:, ::3] = 2.0 ** -130
-    elif case == "far_blocks":        # one block 2^240 below the largest: its factor underflows
-        x[:, 32:48] *= 2.0 ** -120
-        x[:, :16] *= 2.0 ** 120
-    elif case == "inf":
-        x[:, 700] = float("inf")
-    else:
-        x[:, 1234] = float("nan")
-    x = I.bf16_rne(x)
-    y = np_of(W4.w4a16_gemv(pw, x.cuda(), flags=W4.LAUNCH_FP4_MMA))
-    yr, ar = O.matmul(x, wh)
-    if case in ("inf", "nan"):
-        assert np.array_equal(np.isfinite(y), np.isfinite(yr))
-        fin = np.isfinite(yr)
-        assert_within_tolerance(y[fin], yr[fin], ar[fin])
-    else:
-        assert_within_tolerance(y, yr, ar)
+HUGE_CASES = ["x_2p110", "x_2p118", "x_2p125_sparse", "w_2p100_x_2pm110"]
 
 
-def test_fp4_mma_grouped():
-    """Grouped launches on kind::f8f6f4: the sweep, q/k/v sharing x, and a group
-    with a ragged N (which takes the decode kernel for the whole group)."""
+@pytest.mark.parametrize("case", HUGE_CASES)
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_huge_range_outputs(case, M):
+    """The global scale is applied together with the power of two that undoes x's
+    rescaling, so outputs near the top (and bottom) of binary32's range are finite
+    and within the bound (M = 1, the skinny kernel, and split-K at M = 16)."""
+    for K in (2560, 9728):
+        W, x = huge_range_case(case, M, K, 300 + M)
+        pw, wh = nvfp4_packed(W.contiguous())
+        yr, ar = O.matmul(x, wh)
+        assert np.all(np.abs(yr) < 3.0e38) and np.all(np.isfinite(ar))
+        if case == "x_2p118":
+            # without g the sums reach y / g: above binary32's range here
+            assert float(np.max(np.abs(yr))) / float(pw.global_scale.item()) > 3.5e38
+        run_and_check(pw, wh, x)
+
+
+@pytest.mark.parametrize("case", HUGE_CASES)
+def test_huge_range_grouped(case):
     pws, whs, xs = [], [], []
-    for idx, (K, N) in enumerate(I.SWEEP_SHAPES):
-        pw, wh = nvfp4_packed(I.sweep_weights(K, N, idx))
-        pws.append(pw); whs.append(wh); xs.append(I.sweep_x(1, K, idx))
-    check_group(pws, whs, xs, flags=W4.LAUNCH_FP4_MMA)
-    check_group(pws, whs, xs, flags=W4.LAUNCH_FP4_MMA | W4.LAUNCH_PDL)
-    K = 2560
-    mats = [nvfp4_packed(I.sweep_weights(K, N, 90 + i)[:N].contiguous()) for i, N in enumerate((4096, 1024, 1024))]
-    x = I.activations(1, K, 91)
-    check_group([m[0] for m in mats], [m[1] for m in mats], [x, x, x], flags=W4.LAUNCH_FP4_MMA)
-    shapes = [(256, 8), (1024, 152), (2560, 333), (9728, 16), (512, 8), (4096, 4096)]
-    pws, whs, xs = [], [], []
-    for i, (K, N) in enumerate(shapes):
-        pw, wh = nvfp4_packed(I.sweep_weights(K, N, 100 + i)[:N].contiguous())
-        pws.append(pw); whs.append(wh); xs.append(I.activations(1, K, 110 + i))
-    check_group(pws, whs, xs, flags=W4.LAUNCH_FP4_MMA)
-    check_group(pws[:2] + pws[3:], whs[:2] + whs[3:], xs[:2] + xs[3:], flags=W4.LAUNCH_FP4_MMA)
-
-
-def test_fp4_mma_graph_deterministic():
-    """Replayed in a CUDA graph with PDL the kernel gives the same bits every time."""
-    shapes = [(2560, 1024), (4096, 512), (9728, 256)]
-    pws, whs, xs = [], [], []
-    for i, (K, N) in enumerate(shapes):
-        pw, wh = nvfp4_packed(I.sweep_weights(K, N, 120 + i)[:N].contiguous())
-        pws.append(pw); whs.append(wh); xs.append(I.activations(1, K, 130 + i))
-    fl = W4.LAUNCH_FP4_MMA | W4.LAUNCH_PDL
-    ref = [y.clone() for y in check_group(pws, whs, xs, flags=fl)]
-    xd = [x.cuda() for x in xs]
-    outs = [torch.empty(1, w.N, device="cuda") for w in pws]
-    s = torch.cuda.Stream()
-    s.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(s):
-        W4.w4a16_gemv_grouped(pws, xd, outs=outs, flags=fl)
-    torch.cuda.current_stream().wait_stream(s)
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        W4.w4a16_gemv_grouped(pws, xd, outs=outs, flags=fl)
-    for _ in range(3):
-        g.replay()
-    torch.cuda.synchronize()
-    for a, b in zip(ref, outs):
-        assert torch.equal(a, b)
-    single = [W4.w4a16_gemv(p, x, flags=fl) for p, x in zip(pws, xd)]
-    for a, b in zip(ref, single):
-        assert torch.equal(a, b)
+    for i, K in enumerate((2560, 4096, 9728)):
+        W, x = huge_range_case(case, 1, K, 320 + i)
+        pw, wh = nvfp4_packed(W.contiguous())
+        pws.append(pw); whs.append(wh); xs.append(x)
+    check_group(pws, whs, xs)

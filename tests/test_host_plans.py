@@ -45,8 +45,6 @@ def test_caps_and_small_problems():
     ctas = W4.plan_grouped(ws, 148)
     assert ctas[0] == 1 and ctas[1] == 1                 # one 16-row tile each
     assert ctas[2] == 146                                # the rest, under its 160-tile cap
-    f4 = W4.plan_grouped(ws, 148, W4.LAUNCH_FP4_MMA)
-    assert f4[2] == 2560 // 64                           # one CTA per 64 rows on the f8f6f4 kernel
     assert sum(W4.plan_grouped([FakeNvfp4(512, 32)] * 3, 148)) == 3 * 2   # total capped by the tiles
 
 
@@ -62,6 +60,6 @@ def test_plan_argument_errors():
     with pytest.raises(W4.W4Error):
         W4.plan_grouped([w], 0)
     with pytest.raises(W4.W4Error):
-        W4.plan_grouped([w], 148, W4.LAUNCH_TMEM)
+        W4.plan_grouped([w], 148, 2)                     # unknown flag
     with pytest.raises(W4.W4Error):
         W4.plan_grouped([FakeNvfp4(512, 64, W4.FMT_ROCMFP4_DUAL)], 148)

@@ -25,7 +25,7 @@ import torch
 __all__ = [
     "W4Error", "PackedWeights", "FMT_NVFP4", "FMT_ROCMFP4_DUAL", "FMT_ROCMFP4_FAST", "FMT_Q4_0",
     "pack_q4_0", "reconstruction_error", "plan_grouped",
-    "LAUNCH_PDL", "LAUNCH_TMEM", "LAUNCH_FP4_MMA", "pack_nvfp4", "pack_rocmfp4", "w4a16_gemv", "w4a16_gemv_grouped", "w4a16_gemm",
+    "LAUNCH_PDL", "set_wait_limit", "pack_nvfp4", "pack_rocmfp4", "w4a16_gemv", "w4a16_gemv_grouped", "w4a16_gemm",
     "w4a16_workspace_bytes", "pack_nvfp4_workspace_bytes", "w4_encode_scalars",
     "w4_device_error", "lib", "library_path",
 ]
@@ -33,8 +33,6 @@ __all__ = [
 FMT_NVFP4, FMT_ROCMFP4_DUAL, FMT_ROCMFP4_FAST, FMT_Q4_0 = 1, 2, 3, 4
 SCALE_ABSMAX, SCALE_MSE = 0, 1
 LAUNCH_PDL = 1
-LAUNCH_TMEM = 2   # opt-in tcgen05 GEMV for one token (see include/w4a16.h)
-LAUNCH_FP4_MMA = 4   # one token on tcgen05 kind::f8f6f4, codes unpacked by TMA (see include/w4a16.h)
 BLOCK_BYTES = {FMT_ROCMFP4_DUAL: 18, FMT_ROCMFP4_FAST: 17}
 _FMT_NAMES = {"nvfp4": FMT_NVFP4, "dual": FMT_ROCMFP4_DUAL, "fast": FMT_ROCMFP4_FAST}
 
@@ -87,6 +85,7 @@ def lib():
             "w4a16_workspace_bytes": ([WP, I], S),
             "w4_encode_scalars": ([P, S, P, P, P], I),
             "w4_device_error": ([ctypes.POINTER(ctypes.c_int), I], I),
+            "w4_set_wait_limit": ([ctypes.c_ulonglong], I),
             "w4_status_string": ([I], ctypes.c_char_p),
             "w4_version": ([], ctypes.c_char_p),
         }
@@ -294,6 +293,12 @@ def w4_encode_scalars(v: torch.Tensor, stream=None):
     _check(lib().w4_encode_scalars(_ptr(v), v.numel(), _ptr(e4), _ptr(e2), _stream(stream)),
            "w4_encode_scalars")
     return e4, e2
+
+
+def set_wait_limit(ns: int = 0):
+    """Limit (ns) of the device-side waits that gate progress, on the current
+    device; 0 restores the default (2 s).  For exercising failure detection."""
+    _check(lib().w4_set_wait_limit(ns), "w4_set_wait_limit")
 
 
 def w4_device_error(clear: bool = True) -> int:

@@ -9,6 +9,10 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include <map>
+#include <mutex>
+#include <utility>
+
 #include "../../include/w4a16.h"
 
 namespace w4 {
@@ -19,6 +23,12 @@ __device__ int g_device_error;
 // A wait on an mbarrier that takes longer than this is treated as a failure:
 // the kernel records W4_ERR_TIMEOUT and returns instead of spinning forever.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+
+// Limit of the waits that gate progress (mbar_wait), per device; settable from
+// the host (w4_set_wait_limit) so that failure detection can be exercised.  The
+// waits that drain a CTA's own copies and MMAs before it exits (mbar_wait_bounded)
+// keep the fixed kWaitLimitNs.
+__device__ unsigned long long g_wait_limit_ns = kWaitLimitNs;
 
 __device__ __forceinline__ void record_error(int status) {
     atomicCAS(&g_device_error, 0, status);
@@ -110,10 +120,10 @@ __device__ __forceinline__ unsigned long long global_ns() {
 // records W4_ERR_TIMEOUT.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
     if (mbar_try_wait(bar, parity)) return true;
-    const unsigned long long t0 = global_ns();
+    const unsigned long long t0 = global_ns(), limit = g_wait_limit_ns;
     while (!mbar_try_wait(bar, parity)) {
         if (*abort) return false;
-        if (global_ns() - t0 > kWaitLimitNs) {
+        if (global_ns() - t0 > limit) {
             *abort = 1;
             record_error(W4_ERR_TIMEOUT);
             return false;
@@ -172,8 +182,9 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
-// Wait as mbar_wait, but ignoring the CTA's abort flag (still bounded in time):
-// for the last completion a thread must see before tensor memory is released.
+// Wait as mbar_wait, but ignoring the CTA's abort flag and the settable limit
+// (still bounded, by kWaitLimitNs): for the completions a CTA must see before it
+// releases tensor memory or exits -- its own bulk copies and MMAs in flight.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
@@ -184,6 +195,33 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
         }
     }
     return true;
+}
+
+// Raise a kernel's dynamic shared-memory limit to at least `bytes` on the
+// current device.  The attribute belongs to the device's context, so the sizes
+// already set are kept per (kernel, device), under a lock shared by all host
+// threads.
+inline bool set_smem_limit(const void *kernel, size_t bytes) {
+    static std::mutex mu;
+    static std::map<std::pair<const void *, int>, size_t> done;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    std::lock_guard<std::mutex> lk(mu);
+    size_t &cur = done[{kernel, dev}];
+    if (bytes <= cur) return true;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
+        return false;
+    cur = bytes;
+    return true;
+}
+
+// Before a producer lane returns: wait for the copies it issued into a ring of
+// `ns` stages whose fill count is `issued` (stage i went to slot i % ns with
+// phase (i / ns) & 1), so that no copy is still writing shared memory when the
+// CTA exits -- on the normal path these phases have long completed; after an
+// aborted run the copies issued before the abort still land.
+__device__ __forceinline__ void drain_ring(uint64_t *full, int ns, int issued) {
+    for (int i = max(0, issued - ns); i < issued; i++) mbar_wait_bounded(full + (i % ns), (uint32_t)((i / ns) & 1));
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).

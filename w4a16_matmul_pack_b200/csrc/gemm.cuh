@@ -84,6 +84,7 @@ struct SharedStorage {
     uint64_t x_full[STAGES], x_empty[STAGES];
     uint64_t a_full[STAGES], a_empty[STAGES];
     uint64_t acc_full[2], acc_empty[2];
+    uint64_t mma_done;                  // the issuer's last commit: every MMA has finished
     uint32_t tmem_base;
     int abort;
     int f16_tile[kMaxTilesM];   // token tile mt runs with f16 operands (else BF16)
@@ -182,6 +183,16 @@ __device__ __forceinline__ uint4 dequant8_f16(uint32_t cw, uint32_t s2) {
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// The power of two a BF16-operand tile folds into its weights: the exponent of
+// g, clamped so that e2m1 * scale * 2^fold stays an exact BF16 value (e2m1 *
+// scale lies in [2^-10, 2688] with at most 6 significant bits).  The products
+// x * A then have the size of the true x * w_hat, so the accumulator overflows
+// only if the result itself does; the epilogue multiplies by g * 2^-fold.
+__device__ __forceinline__ int bf16_fold(float g) {
+    const int eg = (int)((__float_as_uint(g) >> 23) & 0xFF) - 127;
+    return max(-123, min(116, eg));
+}
+
 // Row m of x -> f16 as x * 2^-sigma_m, sigma_m chosen so that the row's largest
 // |x * 2^-sigma_m| lies in [2^14, 2^15); bad[m] = 1 when some nonzero value
 // lands below 2^-17 (then it may be inexact in f16) or the row holds Inf / NaN.
@@ -269,6 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             mbar_init(&sh.acc_full[i], 1);
             mbar_init(&sh.acc_empty[i], kEpiThreads / 32);
         }
+        mbar_init(&sh.mma_done, 1);
         fence_mbar_init();
     }
     const bool use_f16 = p.bad != nullptr && p.tiles_m <= kMaxTilesM;
@@ -313,6 +325,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                 }
                 if (*abort) break;
             }
+            // every issued copy has landed before the CTA can exit (after an abort
+            // the loop above stops early, with copies possibly in flight)
+            drain_ring(sh.w_full, WSTAGES, wit);
+            drain_ring(sh.x_full, STAGES, it);
         }
         __syncwarp();   // the whole warp reaches the final barrier together (it is .aligned)
     } else if (warp == 1) {
@@ -344,6 +360,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                 __syncwarp();
             }
         }
+        // tensor memory is released after the final barrier: every MMA this
+        // thread issued must have completed by then (also after an abort)
+        if (lane == 0) {
+            mma_commit(&sh.mma_done);
+            mbar_wait_bounded(&sh.mma_done, 0);
+        }
+        __syncwarp();
     } else if (warp == kWaitWarp) {
         // ------------------------- waits on behalf of the MMA issuer -------------------------
         int it = 0, lt = 0;
@@ -363,6 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         // -------------------------------- epilogue --------------------------------
         const int q = warp & 3;                 // TMEM lane quadrant of this warp
         const float g = __ldg(p.gscale);
+        const int fold = bf16_fold(g);
         int lt = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, lt++) {
             const int b = lt & 1;
@@ -384,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                     const int m = m0 + c * 32 + j;
                     if (n < p.N) {
                         if (m < p.M) {
-                            const float val = g * (f16 ? mul_pow2(__uint_as_float(v[j]), sg) : __uint_as_float(v[j]));
+                            const float val = scale_out(__uint_as_float(v[j]), g, f16 ? sg : -fold);
                             if (p.y32) p.y32[(size_t)m * p.N + n] = val;
                             if (p.y16) p.y16[(size_t)m * p.N + n] = __float2bfloat16_rn(val);
                         }
@@ -403,6 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         // warp w writes TMEM lanes 32*(w%4) .. +31 (the lanes it may access): row r,
         // k-half h of each 64-k stage
         const int r = 32 * (warp & 3) + lane, h = (warp - 6) >> 2;
+        const int fold = bf16_fold(__ldg(p.gscale));
         const uint32_t a_lane = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
         constexpr int KQ = WK / BK;             // k-steps per codes stage
         int it = 0, wit = 0;
@@ -452,7 +477,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                                 av[j][4 * cc] = o.x, av[j][4 * cc + 1] = o.y, av[j][4 * cc + 2] = o.z, av[j][4 * cc + 3] = o.w;
                             }
                         } else {
-                            const float s0 = e4m3_to_f32(sw & 0xFFu), s1 = e4m3_to_f32((sw >> 8) & 0xFFu);
+                            const float s0 = mul_pow2(e4m3_to_f32(sw & 0xFFu), fold),
+                                        s1 = mul_pow2(e4m3_to_f32((sw >> 8) & 0xFFu), fold);
 #pragma unroll
                             for (int cc = 0; cc < 4; cc++) {
                                 const uint4 o = valid ? dequant8(cws[cc], cc < 2 ? s0 : s1) : make_uint4(0, 0, 0, 0);
@@ -541,13 +567,8 @@ inline w4_status gemm_launch(const w4_weights *w, const void *x, int M, float *y
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev))
         return W4_ERR_CUDA;
-    static bool configured = false;
     const size_t smem = gemm_smem_bytes();
-    if (!configured) {
-        if (cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-            return W4_ERR_CUDA;
-        configured = true;
-    }
+    if (!set_smem_limit(reinterpret_cast<const void *>(gemm_kernel), smem)) return W4_ERR_CUDA;
     Params p;
     p.codes = w->codes;
     p.scales = w->scales;

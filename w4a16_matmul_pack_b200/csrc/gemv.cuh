@@ -168,9 +168,11 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvArgs a)
         // ------------------------------ producer ------------------------------
         if (lane == 0) {
             const uint64_t pol = policy_evict_first();
+            int issued = 0;
             for (int t = 0; t < ntiles; t++) {
                 const int st = t % NS;
                 if (t >= NS && !mbar_wait(empty + st, ((t / NS) - 1) & 1, abort)) break;
+                issued++;
                 const long long rt = r0 + (long long)t * TR;
                 const int rows = (int)min((long long)TR, r1 - rt);
                 uint8_t *dst = stages + (size_t)st * a.tile_bytes;
@@ -199,6 +201,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvArgs a)
                     }
                 }
             }
+            // no copy may still be landing in shared memory when the CTA exits
+            drain_ring(full, NS, issued);
         }
         return;
     }

@@ -202,7 +202,10 @@ __device__ __forceinline__ void m1_body(const CUtensorMap &cmap, const CUtensorM
         __syncwarp();
     }
     const bool fast = !__any_sync(0xFFFFFFFFu, bad);
-    if (!fast) sref = 0;   // binary32 path: partial sums in units of x itself
+    // binary32 path: partial sums in units of x * 2^fold (the largest block of
+    // this warp has |x| in [2^(sref+14), 2^(sref+15)))
+    const int fold = fast ? 0 : fallback_fold(gs, sref + 14 >= 100);
+    if (!fast) sref = -fold;
 
     // MMA operands.  Lane (g, t) holds rows g, g+8 of the codes of k = 32t .. 32t+31
     // (blocks 2t, 2t+1) and B column g.  Column g is block g: it is nonzero only for
@@ -280,6 +283,7 @@ __device__ __forceinline__ void m1_body(const CUtensorMap &cmap, const CUtensorM
                         const uint2 c = *reinterpret_cast<const uint2 *>(cp + 8 * q);
                         float2 w[8], xv[8];
                         decode_nvfp4(c, w);
+                        scale_pairs(w, fold);
                         const uint4 u0 = __ldg(xg + 2 * q), u1 = __ldg(xg + 2 * q + 1);
                         const uint32_t wv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
@@ -301,12 +305,12 @@ __device__ __forceinline__ void m1_body(const CUtensorMap &cmap, const CUtensorM
             accB += __shfl_xor_sync(0xFFFFFFFFu, accB, 1);
             accB += __shfl_xor_sync(0xFFFFFFFFu, accB, 2);
             if (t4 == 0) {
-                rb[warp * kTcRows + g] = mul_pow2(accA, sref);
-                rb[warp * kTcRows + g + 8] = mul_pow2(accB, sref);
+                rb[warp * kTcRows + g] = scale_out(accA, gs, sref);
+                rb[warp * kTcRows + g + 8] = scale_out(accB, gs, sref);
             }
         } else {
             accA += __shfl_xor_sync(0xFFFFFFFFu, accA, 1);
-            if ((lane & 1) == 0) rb[warp * kTcRows + (lane >> 1)] = accA;
+            if ((lane & 1) == 0) rb[warp * kTcRows + (lane >> 1)] = scale_out(accA, gs, sref);
         }
         if (!all_at_end) {
             named_barrier_sync(1, kTcWarps * 32);
@@ -317,7 +321,7 @@ __device__ __forceinline__ void m1_body(const CUtensorMap &cmap, const CUtensorM
                 for (int q = 0; q < kTcParts; q++) s += rb[q * kTcRows + threadIdx.x];
                 const long long n = rt + threadIdx.x;
                 if (nslices == 1)
-                    a.y[n] = gs * s;
+                    a.y[n] = s;
                 else
                     a.partial[(size_t)slice * N + n] = s;
             }
@@ -333,7 +337,7 @@ __device__ __forceinline__ void m1_body(const CUtensorMap &cmap, const CUtensorM
             float s = 0.0f;
             for (int q = 0; q < kTcParts; q++) s += rb[q * kTcRows];
             if (nslices == 1)
-                a.y[n] = gs * s;
+                a.y[n] = s;
             else
                 a.partial[(size_t)slice * N + n] = s;
         }

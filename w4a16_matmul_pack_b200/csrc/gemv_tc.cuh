@@ -64,6 +64,36 @@ __device__ __forceinline__ float mul_pow2(float v, int e) {
     return (v * __int_as_float((127 + h) << 23)) * __int_as_float((127 + h2) << 23);
 }
 
+// v * g * 2^e rounded once to binary32.  The kernels accumulate in units of
+// x * 2^-e (x rescaled into f16's range) with the weights' global scale g left
+// out; the output is the product of all three.  In binary64 the product v * g of
+// two binary32 values is exact and 2^e (|e| <= 400 here) is in range, so no
+// intermediate overflows or underflows: the result is finite whenever the true
+// product is below binary32's largest value.
+__device__ __forceinline__ float scale_out(float v, float g, int e) {
+    const double p2 = __longlong_as_double((long long)(1023 + e) << 52);
+    return (float)((double)v * (double)g * p2);
+}
+
+// Power of two folded into the decoded weights of the binary32 fallback paths:
+// the exponent of g, clamped to [-100, 0], when x reaches 2^100 (else 0).  Sums
+// of x * e2m1 * 2^fold (and their products with the block scale) then stay near
+// the size of the true x * w_hat, so a finite result cannot overflow inside the
+// accumulator.
+__device__ __forceinline__ int fallback_fold(float g, bool x_huge) {
+    if (!x_huge) return 0;
+    const int eg = (int)((__float_as_uint(g) >> 23) & 0xFF) - 127;
+    return max(-100, min(0, eg));
+}
+
+// w[p] *= 2^e (exact for the E2M1 values of a fallback block, e in [-100, 0]).
+template <int NP>
+__device__ __forceinline__ void scale_pairs(float2 (&w)[NP], int e) {
+    const float f = __int_as_float((127 + e) << 23);
+#pragma unroll
+    for (int p = 0; p < NP; p++) w[p] = __fmul2_rn(w[p], make_float2(f, f));
+}
+
 constexpr int kTcRows = 16;                    // rows per tile (one MMA M)
 constexpr int kTcWarps = 8;                    // consumer warps, each a contiguous share of a tile's k
 constexpr int kTcParts = kTcWarps;
@@ -111,10 +141,11 @@ __device__ __forceinline__ void reduce_tile(const GemvTcArgs &a, const float *rb
         float s = 0.0f;
         for (int q = 0; q < nparts; q++) s += rb[(q * kTcRows + row) * M + m];
         const long long n = rt + row;
+        const float v = scale_out(s, gs, yexp);
         if (gridDim.y == 1)
-            a.y[(size_t)m * a.N + n] = gs * mul_pow2(s, yexp);
+            a.y[(size_t)m * a.N + n] = v;
         else
-            a.partial[((size_t)slice * M + m) * a.N + n] = mul_pow2(s, yexp);
+            a.partial[((size_t)slice * M + m) * a.N + n] = v;
     }
 }
 
@@ -130,17 +161,21 @@ __device__ __forceinline__ void tc_produce(const CUtensorMap &cmap, const CUtens
     const int CS = KP / 2, SS = KP / 16;
     const uint64_t pol = policy_evict_first();
     const int before = a.pdl ? min(NS, nstages) : 0;
+    int issued = 0;        // weight stages issued
+    bool x_issued = false;
     for (int t = 0; t < nstages + 1; t++) {
         if (t == before) {
             pdl_wait_prior_grid();
             mbar_arrive_expect_tx(xfull, (uint32_t)(M * kcs * 2));
             for (int m = 0; m < M; m++)
                 bulk_g2s(xs + (size_t)m * XS, a.x + (size_t)m * K + k0, (uint32_t)(kcs * 2), xfull, pol);
+            x_issued = true;
             continue;
         }
         const int tt = t > before ? t - 1 : t;   // weight stage index
         const int st = tt % NS;
         if (tt >= NS && !mbar_wait(empty + st, ((tt / NS) - 1) & 1, abort)) break;
+        issued++;
         const long long rt = r0 + (long long)(tt / npieces) * kTcRows;
         const int rows = (int)min((long long)kTcRows, r1 - rt);
         const int kpos = k0 + (tt % npieces) * KP;
@@ -162,6 +197,9 @@ __device__ __forceinline__ void tc_produce(const CUtensorMap &cmap, const CUtens
             }
         }
     }
+    // no copy may still be landing in shared memory when the CTA exits
+    drain_ring(full, NS, issued);
+    if (x_issued) mbar_wait_bounded(xfull, 0);
 }
 
 template <int M>
@@ -283,7 +321,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         named_barrier_sync(1, kTcWarps * 32);
     }
-    const int yexp = fast ? sigma : 0;   // undo the x scaling
+    // undo the x scaling (f16 path); the binary32 path folds a power of two into
+    // the decoded weights instead when x is huge (fallback_fold)
+    const int fold = fast ? 0 : fallback_fold(gs, mx >= ((127u + 100u) << 7));   // largest |x| >= 2^100
+    const int yexp = fast ? sigma : -fold;
 
     const int g = lane >> 2, t4 = lane & 3;
     int st_idx = 0;
@@ -351,6 +392,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             const float sv = e4m3_to_f32(tp[kTcRows * CS + row * SS + q]);
                             float2 w[8];
                             decode_nvfp4(c, w);
+                            scale_pairs(w, fold);
 #pragma unroll
                             for (int m = 0; m < M; m++) {
                                 float2 xv[8];
@@ -409,10 +451,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const float *rb = red + (size_t)tile * kTcParts * kTcRows * M;
             float s = 0.0f;
             for (int q = 0; q < nparts; q++) s += rb[(q * kTcRows + row) * M + m];
+            const float v = scale_out(s, gs, yexp);
             if (gridDim.y == 1)
-                a.y[(size_t)m * N + n] = gs * mul_pow2(s, yexp);
+                a.y[(size_t)m * N + n] = v;
             else
-                a.partial[((size_t)slice * M + m) * N + n] = mul_pow2(s, yexp);
+                a.partial[((size_t)slice * M + m) * N + n] = v;
         }
     }
 }

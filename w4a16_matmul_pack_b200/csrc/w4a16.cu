@@ -10,8 +10,6 @@
 #include "gemv.cuh"
 #include "gemv_tc.cuh"
 #include "gemv_m1.cuh"
-#include "gemv_umma.cuh"
-#include "gemv_f4.cuh"
 #include "gemm.cuh"
 
 using namespace w4;
@@ -108,12 +106,7 @@ w4_status launch_gemv_m(const w4_weights *w, const void *x, float *y, void *ws, 
                         cudaStream_t st) {
     constexpr int R = M <= 2 ? 4 : (M <= 4 ? 2 : 1);
     auto kern = gemv_kernel<FMT, M, R>;
-    static size_t configured = 0;  // largest dynamic smem size set so far for this instantiation
-    if (p.smem > configured) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem) != cudaSuccess)
-            return W4_ERR_CUDA;
-        configured = p.smem;
-    }
+    if (!set_smem_limit(reinterpret_cast<const void *>(kern), p.smem)) return W4_ERR_CUDA;
     GemvArgs a;
     a.codes = w->codes;
     a.scales = w->scales;
@@ -287,12 +280,7 @@ w4_status launch_gemv_tc_m(const w4_weights *w, const void *x, float *y, void *w
                            cudaStream_t st) {
     // one token: block scales applied after the MMA (gemv_m1.cuh)
     auto kern = M == 1 ? gemv_nvfp4_m1_kernel : gemv_nvfp4_tc_kernel<M>;
-    static size_t configured = 0;
-    if (p.smem > configured) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem) != cudaSuccess)
-            return W4_ERR_CUDA;
-        configured = p.smem;
-    }
+    if (!set_smem_limit(reinterpret_cast<const void *>(kern), p.smem)) return W4_ERR_CUDA;
     const int N = w->N;
     CUtensorMap cmap, smap;
     GemvTcArgs a;
@@ -311,7 +299,8 @@ w4_status launch_gemv_tc_m(const w4_weights *w, const void *x, float *y, void *w
     if (cudaLaunchKernelEx(&cfg, kern, cmap, smap, a) != cudaSuccess) return W4_ERR_CUDA;
     if (p.S > 1) {
         const int MN = M * N;
-        gemv_finalize_kernel<<<std::min((MN + 255) / 256, 1024), 256, 0, st>>>(a.partial, p.S, MN, w->global_scale, y);
+        // the slice partials already carry the global scale (scale_out)
+        gemv_finalize_kernel<<<std::min((MN + 255) / 256, 1024), 256, 0, st>>>(a.partial, p.S, MN, nullptr, y);
     }
     return launch_status();
 }
@@ -347,11 +336,9 @@ void share_sms(const w4_weights *w, int G, int sms, const int *max_cta, int *all
     }
 }
 
-// Most CTAs a grouped launch gives problem p: one per 16-row tile (decode
-// kernel) or one per 64 rows (the kind::f8f6f4 kernel), at least one.
-void grouped_max_cta(const w4_weights *w, int G, bool fp4, int *max_cta) {
-    for (int p = 0; p < G; p++)
-        max_cta[p] = fp4 ? std::max(1, w[p].N / 64) : (w[p].N + kTcRows - 1) / kTcRows;
+// Most CTAs a grouped launch gives problem p: one per 16-row tile, at least one.
+void grouped_max_cta(const w4_weights *w, int G, int *max_cta) {
+    for (int p = 0; p < G; p++) max_cta[p] = (w[p].N + kTcRows - 1) / kTcRows;
 }
 
 // Several one-token NVFP4 problems in one launch (gemv_m1.cuh): the SMs are
@@ -363,7 +350,7 @@ w4_status launch_gemv_grouped(const w4_weights *w, const void *const *x, float *
     DeviceInfo d;
     if (device_info(d) != W4_OK) return W4_ERR_CUDA;
     int tiles[kMaxGroup], alloc[kMaxGroup];
-    grouped_max_cta(w, G, false, tiles);
+    grouped_max_cta(w, G, tiles);
     share_sms(w, G, d.sms, tiles, alloc);
     static GroupArgs g;   // host staging of the kernel parameter (copied at launch)
     static std::mutex mu;
@@ -381,13 +368,7 @@ w4_status launch_gemv_grouped(const w4_weights *w, const void *const *x, float *
         g.cta0[p + 1] = g.cta0[p] + plan.grid;
         smem = std::max(smem, plan.smem);
     }
-    static size_t configured = 0;
-    if (smem > configured) {
-        if (cudaFuncSetAttribute(gemv_nvfp4_m1_grouped_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem) != cudaSuccess)
-            return W4_ERR_CUDA;
-        configured = smem;
-    }
+    if (!set_smem_limit(reinterpret_cast<const void *>(gemv_nvfp4_m1_grouped_kernel), smem)) return W4_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(g.cta0[G], 1, 1);
     cfg.blockDim = dim3(kTcThreads, 1, 1);
@@ -399,213 +380,6 @@ w4_status launch_gemv_grouped(const w4_weights *w, const void *const *x, float *
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
     if (cudaLaunchKernelEx(&cfg, gemv_nvfp4_m1_grouped_kernel, g) != cudaSuccess) return W4_ERR_CUDA;
-    return launch_status();
-}
-
-// One token on tcgen05 (gemv_umma.cuh, opt-in with W4_LAUNCH_TMEM): K a
-// multiple of 512 and small enough that x (twice) and two weight stages fit
-// next to a co-resident CTA.
-constexpr int kUmmaMaxK = 12288;
-
-struct UmmaPlan {
-    int TB = 1, NS = 2, grid = 0;
-    size_t smem = 0;
-};
-
-bool umma_applies(int K, int M) { return M == 1 && K % um::kStepK == 0 && K <= kUmmaMaxK; }
-
-w4_status plan_umma(int K, int N, bool pdl, UmmaPlan &p) {
-    DeviceInfo d;
-    if (device_info(d) != W4_OK) return W4_ERR_CUDA;
-    const int T = (N + um::kTileRows - 1) / um::kTileRows;
-    p.grid = std::min(d.sms, T);
-    const double tile_bytes = um::kTileRows * (K / 2.0 + K / 16.0);
-    // stages of about 16-24 KB (bulk copies below that lose bandwidth), at most
-    // the CTA's own tile count
-    const int tiles_per_cta = (T + p.grid - 1) / p.grid;
-    p.TB = std::max(1, std::min({8, tiles_per_cta, (int)(20480.0 / tile_bytes + 0.5)}));
-    const size_t budget = std::min<size_t>(pdl ? 110 * 1024 : 200 * 1024, (size_t)d.smem_optin);
-    p.NS = 8;
-    while (p.NS > 2 && um::layout(K, p.TB, p.NS).total > budget) p.NS--;
-    p.smem = um::layout(K, p.TB, p.NS).total;
-    if (p.smem > (size_t)d.smem_optin) return W4_ERR_UNSUPPORTED;
-    return W4_OK;
-}
-
-w4_status launch_umma(const w4_weights *w, const void *x, float *y, const UmmaPlan &p, bool pdl, cudaStream_t st) {
-    static size_t configured = 0;
-    if (p.smem > configured) {
-        if (cudaFuncSetAttribute(um::gemv_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem) !=
-            cudaSuccess)
-            return W4_ERR_CUDA;
-        configured = p.smem;
-    }
-    PFN_encodeTiled enc = get_encode_tiled();
-    if (!enc) return W4_ERR_CUDA;
-    const int K = w->K, N = w->N;
-    // codes as [N][K/512][32 x 8 bytes], scales as [N][K/512][32 bytes]; boxes of
-    // 4*TB rows (full stages) and 4 rows (a CTA's last, partial stage)
-    CUtensorMap cmap, smap, cmap1, smap1;
-    const cuuint64_t cdims[3] = {32, (cuuint64_t)K / 512, (cuuint64_t)N};
-    const cuuint64_t cstr[2] = {256, (cuuint64_t)K / 2};
-    const cuuint64_t sdims[3] = {32, (cuuint64_t)K / 512, (cuuint64_t)N};
-    const cuuint64_t sstr[2] = {32, (cuuint64_t)K / 16};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    auto encode = [&](CUtensorMap *m, CUtensorMapDataType dt, const void *base, const cuuint64_t *dims,
-                      const cuuint64_t *str, int rows) {
-        const cuuint32_t box[3] = {32, (cuuint32_t)K / 512, (cuuint32_t)rows};
-        return enc(m, dt, 3, const_cast<void *>(base), dims, str, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-    };
-    if (!encode(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT64, w->codes, cdims, cstr, um::kTileRows * p.TB) ||
-        !encode(&smap, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->scales, sdims, sstr, um::kTileRows * p.TB) ||
-        !encode(&cmap1, CU_TENSOR_MAP_DATA_TYPE_UINT64, w->codes, cdims, cstr, um::kTileRows) ||
-        !encode(&smap1, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->scales, sdims, sstr, um::kTileRows))
-        return W4_ERR_CUDA;
-    um::Args a;
-    a.codes = w->codes;
-    a.scales = w->scales;
-    a.gscale = w->global_scale;
-    a.x = reinterpret_cast<const uint16_t *>(x);
-    a.y = y;
-    a.K = K;
-    a.N = N;
-    a.TB = p.TB;
-    a.NS = p.NS;
-    a.pdl = pdl ? 1 : 0;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.grid, 1, 1);
-    cfg.blockDim = dim3(um::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = p.smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
-    if (cudaLaunchKernelEx(&cfg, um::gemv_umma_kernel, cmap, smap, cmap1, smap1, a) != cudaSuccess)
-        return W4_ERR_CUDA;
-    return launch_status();
-}
-
-// One token with the codes fed to tcgen05 kind::f8f6f4 (gemv_f4.cuh): NVFP4,
-// K a multiple of 256, N of 8, codes 32-byte aligned (the unpacking TMA type).
-constexpr int kF4MaxK = 32768;   // x (64 KB) and two stages fit in shared memory
-bool f4_applies(const w4_weights *w, int M) {
-    return M == 1 && w->fmt == W4_FMT_NVFP4 && w->K % f4::kStageK == 0 && w->K <= kF4MaxK && w->N % 8 == 0 &&
-           (reinterpret_cast<uintptr_t>(w->codes) & 31u) == 0;
-}
-
-// Stages that fit with x of length K (at most kMaxStages, at least 2).
-int f4_stages(const DeviceInfo &d, int K) {
-    int NS = f4::kMaxStages;
-    while (NS > 2 && f4::smem_bytes(NS, K) > (size_t)d.smem_optin) NS--;
-    return NS;
-}
-
-// CTAs of a single problem: at least 64 rows each (a 128-row MMA tile at least
-// half used), at most one per SM.
-int f4_grid(int N, int sms) { return std::max(1, std::min(sms, N / 64)); }
-
-w4_status f4_setup(const w4_weights *w, const void *x, float *y, int NS, CUtensorMap &amap, CUtensorMap &smap,
-                   f4::Args &a) {
-    PFN_encodeTiled enc = get_encode_tiled();
-    if (!enc) return W4_ERR_CUDA;
-    const int K = w->K, N = w->N;
-    const cuuint64_t adims[2] = {(cuuint64_t)K, (cuuint64_t)N};   // 4-bit elements
-    const cuuint64_t astr[1] = {(cuuint64_t)K / 2};
-    const cuuint32_t abox[2] = {128, (cuuint32_t)f4::kRows};
-    const cuuint64_t sdims[2] = {(cuuint64_t)K / 16, (cuuint64_t)N};
-    const cuuint64_t sstr[1] = {(cuuint64_t)K / 16};
-    const cuuint32_t sbox[2] = {(cuuint32_t)(f4::kStageK / 16), (cuuint32_t)f4::kRows};
-    const cuuint32_t estr[2] = {1, 1};
-    if (enc(&amap, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<uint8_t *>(w->codes), adims, astr, abox, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return W4_ERR_CUDA;
-    if (enc(&smap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(w->scales), sdims, sstr, sbox, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return W4_ERR_CUDA;
-    a.x = reinterpret_cast<const uint16_t *>(x);
-    a.y = y;
-    a.gscale = w->global_scale;
-    a.K = K;
-    a.N = N;
-    a.NS = NS;
-    return W4_OK;
-}
-
-w4_status launch_f4(const w4_weights *w, const void *x, float *y, bool pdl, cudaStream_t st) {
-    DeviceInfo d;
-    if (device_info(d) != W4_OK) return W4_ERR_CUDA;
-    const int NS = f4_stages(d, w->K);
-    const size_t smem = f4::smem_bytes(NS, w->K);
-    static size_t configured = 0;
-    if (smem > configured) {
-        if (cudaFuncSetAttribute(f4::gemv_nvfp4_f4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-            cudaSuccess)
-            return W4_ERR_CUDA;
-        configured = smem;
-    }
-    CUtensorMap amap, smap;
-    f4::Args a;
-    w4_status s = f4_setup(w, x, y, NS, amap, smap, a);
-    if (s != W4_OK) return s;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(f4_grid(w->N, d.sms), 1, 1);
-    cfg.blockDim = dim3(f4::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
-    if (cudaLaunchKernelEx(&cfg, f4::gemv_nvfp4_f4_kernel, amap, smap, a) != cudaSuccess) return W4_ERR_CUDA;
-    return launch_status();
-}
-
-w4_status launch_f4_grouped(const w4_weights *w, const void *const *x, float *const *y, int G, bool pdl,
-                            cudaStream_t st) {
-    DeviceInfo d;
-    if (device_info(d) != W4_OK) return W4_ERR_CUDA;
-    int max_cta[kMaxGroup], alloc[kMaxGroup];
-    grouped_max_cta(w, G, true, max_cta);
-    share_sms(w, G, d.sms, max_cta, alloc);
-    int Kmax = 0;
-    for (int p = 0; p < G; p++) Kmax = std::max(Kmax, w[p].K);
-    const int NS = f4_stages(d, Kmax);
-    const size_t smem = f4::smem_bytes(NS, Kmax);
-    static f4::GroupArgs g;   // host staging of the kernel parameter (copied at launch)
-    static std::mutex mu;
-    std::lock_guard<std::mutex> lk(mu);
-    g.G = G;
-    g.cta0[0] = 0;
-    for (int p = 0; p < G; p++) {
-        const w4_status s = f4_setup(&w[p], x[p], y[p], NS, g.amap[p], g.smap[p], g.a[p]);
-        if (s != W4_OK) return s;
-        g.cta0[p + 1] = g.cta0[p] + alloc[p];
-    }
-    static size_t configured = 0;
-    if (smem > configured) {
-        if (cudaFuncSetAttribute(f4::gemv_nvfp4_f4_grouped_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem) != cudaSuccess)
-            return W4_ERR_CUDA;
-        configured = smem;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(g.cta0[G], 1, 1);
-    cfg.blockDim = dim3(f4::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
-    if (cudaLaunchKernelEx(&cfg, f4::gemv_nvfp4_f4_grouped_kernel, g) != cudaSuccess) return W4_ERR_CUDA;
     return launch_status();
 }
 
@@ -788,19 +562,12 @@ w4_status w4a16_gemv_ex(const w4_weights *w, const void *x, int M, float *y, voi
                         size_t workspace_bytes, unsigned flags, void *stream) {
     w4_status s = check_weights(w);
     if (s != W4_OK) return s;
-    if (!x || !y || M < 1 || M > 16 || (flags & ~(W4_LAUNCH_PDL | W4_LAUNCH_TMEM | W4_LAUNCH_FP4_MMA)))
-        return W4_ERR_ARG;
+    if (!x || !y || M < 1 || M > 16 || (flags & ~W4_LAUNCH_PDL)) return W4_ERR_ARG;
     if (!aligned16(x) || !aligned16(y) || (workspace && !aligned16(workspace))) return W4_ERR_ALIGN;
     if (w->K % k_unit(w->fmt)) return W4_ERR_UNSUPPORTED;
     const bool pdl = (flags & W4_LAUNCH_PDL) != 0;
     cudaStream_t st = as_stream(stream);
     if (w->fmt == W4_FMT_NVFP4) {
-        if ((flags & W4_LAUNCH_FP4_MMA) && f4_applies(w, M)) return launch_f4(w, x, y, pdl, st);
-        if ((flags & W4_LAUNCH_TMEM) && umma_applies(w->K, M)) {
-            UmmaPlan u;
-            if ((s = plan_umma(w->K, w->N, pdl, u)) != W4_OK) return s;
-            return launch_umma(w, x, y, u, pdl, st);
-        }
         GemvTcPlan p;
         if ((s = plan_gemv_tc(w->K, w->N, M, pdl, p)) != W4_OK) return s;
         if (p.ws_bytes && (!workspace || workspace_bytes < p.ws_bytes)) return W4_ERR_WORKSPACE;
@@ -817,24 +584,21 @@ w4_status w4a16_gemv_ex(const w4_weights *w, const void *x, int M, float *y, voi
 }
 
 w4_status w4_plan_grouped(const w4_weights *w, int G, int sms, unsigned flags, int *ctas) {
-    if (!w || !ctas || G < 1 || G > kMaxGroup || sms < 1 || (flags & ~(W4_LAUNCH_PDL | W4_LAUNCH_FP4_MMA)))
-        return W4_ERR_ARG;
-    bool f4 = (flags & W4_LAUNCH_FP4_MMA) != 0;
+    if (!w || !ctas || G < 1 || G > kMaxGroup || sms < 1 || (flags & ~W4_LAUNCH_PDL)) return W4_ERR_ARG;
     for (int p = 0; p < G; p++) {
         const w4_status s = check_weights(&w[p]);
         if (s != W4_OK) return s;
         if (w[p].fmt != W4_FMT_NVFP4) return W4_ERR_UNSUPPORTED;
-        f4 = f4 && f4_applies(&w[p], 1);
     }
     int max_cta[kMaxGroup];
-    grouped_max_cta(w, G, f4, max_cta);
+    grouped_max_cta(w, G, max_cta);
     share_sms(w, G, sms, max_cta, ctas);
     return W4_OK;
 }
 
 w4_status w4a16_gemv_grouped(const w4_weights *w, const void *const *x, float *const *y, int G, unsigned flags,
                              void *stream) {
-    if (!w || !x || !y || G < 1 || G > kMaxGroup || (flags & ~(W4_LAUNCH_PDL | W4_LAUNCH_FP4_MMA))) return W4_ERR_ARG;
+    if (!w || !x || !y || G < 1 || G > kMaxGroup || (flags & ~W4_LAUNCH_PDL)) return W4_ERR_ARG;
     for (int p = 0; p < G; p++) {
         const w4_status s = check_weights(&w[p]);
         if (s != W4_OK) return s;
@@ -843,11 +607,7 @@ w4_status w4a16_gemv_grouped(const w4_weights *w, const void *const *x, float *c
         if (!aligned16(x[p]) || !aligned16(y[p])) return W4_ERR_ALIGN;
         if (w[p].K % 256) return W4_ERR_UNSUPPORTED;
     }
-    const bool pdl = (flags & W4_LAUNCH_PDL) != 0;
-    bool f4 = (flags & W4_LAUNCH_FP4_MMA) != 0;
-    for (int p = 0; p < G; p++) f4 = f4 && f4_applies(&w[p], 1);
-    if (f4) return launch_f4_grouped(w, x, y, G, pdl, as_stream(stream));
-    return launch_gemv_grouped(w, x, y, G, pdl, as_stream(stream));
+    return launch_gemv_grouped(w, x, y, G, (flags & W4_LAUNCH_PDL) != 0, as_stream(stream));
 }
 
 w4_status w4a16_gemv(const w4_weights *w, const void *x, int M, float *y, void *workspace, size_t workspace_bytes,
@@ -899,6 +659,12 @@ const char *w4_status_string(int status) {
     return "unknown w4_status";
 }
 
-const char *w4_version(void) { return "w4a16 0.1.0 (sm_100a)"; }
+w4_status w4_set_wait_limit(unsigned long long ns) {
+    const unsigned long long v = ns ? ns : kWaitLimitNs;
+    if (cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)) != cudaSuccess) return W4_ERR_CUDA;
+    return W4_OK;
+}
+
+const char *w4_version(void) { return "w4a16 0.2.0 (sm_100a)"; }
 
 }  // extern "C"
