@@ -6,21 +6,21 @@ GEMV sweep -- NVFP4 weights of the 4B-class decoder shapes (K, N) = (2560,4096),
 (2560,1024), (4096,2560), (2560,9728), (9728,2560), Student-t(4) weights of std
 0.02 with 0.01% of entries x20, BF16 activations N(0,1).  One step = one GEMV
 over each of the five matrices, issued as one grouped launch
-(w4a16_gemv_grouped), six steps (one per rotating weight copy) captured in one
-CUDA graph; the same sweep as five separate launches chained with programmatic
-dependent launch is reported beside it.  GB/s counts the packed bytes read
-(codes + scales + global scale, 4.5 bits per weight).  Six packed copies of
-every matrix rotate across steps (248 MB > the 126 MB L2), so no step finds its
-weights in L2.
+(w4a16_gemv_grouped); the steps of one rotation over the packed copies are
+captured in one CUDA graph.  GB/s counts the packed bytes read (codes + scales
++ global scale, 4.5 bits per weight).  Every weight matrix has enough packed
+copies that one rotation reads more than four times the 126 MB L2, so no step
+finds its weights in L2.
 
-The same line carries the other rows of the path, each measured in this run:
-the sweep at M = 4, 9 (speculative verify) and 16, the prefill GEMM (M=2048,
-K=2560, N=9728, TFLOP/s), the 36-layer weight stream (tokens/s at M=1, M=16
-and looped; at M=1 also with q/k/v and gate/up grouped), each sweep shape timed
-alone, the ROCmFP4 GEMV, the packers (NVFP4 abs-max and scale search, ROCmFP4
-Dual / FAST, importance-weighted, Q4_0), and the reconstruction-error quality
-report of every format.  `--impl reference` times the CPU oracle on the same
-workload instead.
+The same line carries the other rows of the path, each measured in this run
+with the same rotation rule and reported as the median of at least 50 timed
+repeats with their min and max: the sweep as separate launches, each sweep
+shape alone, the sweep at M = 4, 9 (speculative verify) and 16, the prefill
+GEMM (M=2048, K=2560, N=9728, TFLOP/s), the 36-layer weight stream (tokens/s at
+M=1, M=16 and looped; at M=1 also with q/k/v and gate/up grouped), the ROCmFP4
+GEMV, the packers (NVFP4 abs-max and scale search, ROCmFP4 Dual / FAST,
+importance-weighted, Q4_0), and the reconstruction-error quality report of
+every format.  `--impl reference` times the CPU oracle on the same workload.
 
 Multi-GPU: the path has no exchange step; `--gpus N` under torchrun runs N
 independent replicas (weak scaling) and reports the summed bytes over the
@@ -45,7 +45,29 @@ sys.path.insert(0, ROOT)
 METRIC = "W4A16 GEMV HBM GB/s (M=1), GEMM TFLOP/s (M=2048), % of roofline"
 WORKLOAD = ("decode GEMV sweep, NVFP4 W4A16, M=1, (K,N) in {(2560,4096),(2560,1024),(4096,2560),"
             "(2560,9728),(9728,2560)}, Student-t(4) std 0.02 weights with 0.01% x20, BF16 x ~ N(0,1)")
-ROTATE = 6
+L2_BYTES = 126 * 1024 * 1024
+ROTATE_BYTES = 4 * L2_BYTES + 1     # one rotation over the copies reads more than 4x L2
+REPEATS = 60                        # individually timed repeats behind every median
+
+
+def n_copies(nbytes: int) -> int:
+    """Packed copies of an operand so that one rotation reads more than 4x L2."""
+    return max(2, -(-ROTATE_BYTES // int(nbytes)))
+
+
+def sweep_step_bytes() -> int:
+    import w4a16_inputs as I
+    return sum(N * (K // 2 + K // 16) + 4 for K, N in I.SWEEP_SHAPES)
+
+
+def headline_config(world: int) -> dict:
+    """The config both arms report (the same keys and values)."""
+    nb = sweep_step_bytes()
+    return {"workload": WORKLOAD, "M": 1,
+            "step": "5 GEMVs in one grouped launch; one rotation of steps per CUDA graph",
+            "l2": f"{n_copies(nb)} rotating packed copies per matrix ({n_copies(nb) * nb / 1e6:.0f} MB > 4x the "
+                  f"126 MB L2)",
+            "bytes_per_step": nb, "parallelism": f"replicas x{world}"}
 
 
 # ----------------------------------------------------------------------------- util
@@ -56,7 +78,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extras", action="store_true", help="headline only (skip GEMM/stream/packers)")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle sample length")
+    ap.add_argument("--cpu-seconds", type=float, default=8.0, help="CPU oracle sample length")
     return ap.parse_args()
 
 
@@ -150,14 +172,22 @@ def replica_value(world: int, step_bytes: float, ms_total: float, steps: int) ->
 
 
 # ------------------------------------------------------------------ workloads (GPU)
+def clone_packed(W4, base):
+    return W4.PackedWeights(base.fmt, base.K, base.N, base.codes.clone(),
+                            None if base.scales is None else base.scales.clone(),
+                            None if base.global_scale is None else base.global_scale.clone())
+
+
 def sweep_setup(W4, I, M=1):
+    """The five sweep matrices, each with enough packed copies that one rotation
+    over them reads more than 4x L2."""
+    R = n_copies(sweep_step_bytes())
     mats = []
     for idx, (K, N) in enumerate(I.SWEEP_SHAPES):
         W = I.sweep_weights(K, N, idx, device="cuda")
         base = W4.pack_nvfp4(W)
         del W
-        copies = [base] + [W4.PackedWeights(base.fmt, K, N, base.codes.clone(), base.scales.clone(),
-                                            base.global_scale.clone()) for _ in range(ROTATE - 1)]
+        copies = [base] + [clone_packed(W4, base) for _ in range(R - 1)]
         x = I.sweep_x(M, K, idx, device="cuda")
         y = torch.empty(M, N, dtype=torch.float32, device="cuda")
         mats.append({"K": K, "N": N, "copies": copies, "x": x, "y": y, "bytes": base.nbytes + 4})
@@ -178,65 +208,86 @@ def capture(fn):
     return g
 
 
-def time_graphs(graphs, steps, warmup):
-    for i in range(warmup):
-        graphs[i % len(graphs)].replay()
+def time_replays(graph, reps=REPEATS, warmup=3):
+    """Milliseconds of each of `reps` replays, timed one by one with CUDA events
+    on the replaying stream (after `warmup` untimed replays)."""
+    for _ in range(warmup):
+        graph.replay()
     torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for i in range(steps):
-        graphs[i % len(graphs)].replay()
-    b.record()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+    ev[0].record()
+    for i in range(reps):
+        graph.replay()
+        ev[i + 1].record()
     torch.cuda.synchronize()
-    return a.elapsed_time(b) / steps  # ms per replay
+    return [ev[i].elapsed_time(ev[i + 1]) for i in range(reps)]
 
 
-def separate_sweep(W4, mats, reps=120):
-    """The sweep as five w4a16_gemv launches per step (CUDA graph, PDL-chained)."""
-    def step_fn(r):
-        def run():
+def summary(ms_list, per: int = 1):
+    """Median / min / max of repeat times, in us per unit (`per` units per repeat)."""
+    v = sorted(m * 1e3 / per for m in ms_list)
+    return {"median_us": round(statistics.median(v), 3), "min_us": round(v[0], 3), "max_us": round(v[-1], 3),
+            "repeats": len(v)}
+
+
+def rate(nbytes: float, st: dict, peak: float):
+    gbs = nbytes / st["median_us"] / 1e3
+    return {"GB/s": round(gbs, 1), "frac": round(gbs / peak, 4)}
+
+
+def separate_sweep(W4, mats, pk):
+    """The sweep as five w4a16_gemv launches per step (PDL-chained), one rotation per graph."""
+    R = len(mats[0]["copies"])
+
+    def run():
+        for r in range(R):
             for m in mats:
                 W4.w4a16_gemv(m["copies"][r], m["x"], out=m["y"], flags=W4.LAUNCH_PDL)
-        return run
-    graphs = [capture(step_fn(r)) for r in range(ROTATE)]
-    ms = time_graphs(graphs, reps, 2 * ROTATE)
+    g = capture(run)
+    st = summary(time_replays(g, REPEATS), R)
     step_bytes = sum(m["bytes"] for m in mats)
-    return {"us_per_step": round(ms * 1e3, 2), "GB/s": round(step_bytes / ms / 1e6, 1), "launches_per_step": 5}
+    return {**st, **rate(step_bytes, st, pk["hbm_gbs"]), "launches_per_step": 5}
 
 
-def per_shape(W4, mats, reps=40):
+def per_shape(W4, mats, pk):
+    """Each sweep shape alone: back-to-back launches over enough copies of that
+    matrix to read more than 4x L2 per rotation."""
     out = {}
     for m in mats:
-        def run(m=m):
-            for c in m["copies"]:
+        R = n_copies(m["bytes"])
+        copies = [m["copies"][i] if i < len(m["copies"]) else clone_packed(W4, m["copies"][0]) for i in range(R)]
+
+        def run(copies=copies, m=m):
+            for c in copies:
                 W4.w4a16_gemv(c, m["x"], out=m["y"])
         g = capture(run)
-        ms = time_graphs([g], reps, 5) / ROTATE
-        out[f"{m['K']}x{m['N']}"] = {"us": round(ms * 1e3, 3), "GB/s": round(m["bytes"] / ms / 1e6, 1)}
+        st = summary(time_replays(g, REPEATS), R)
+        out[f"{m['K']}x{m['N']}"] = {**st, **rate(m["bytes"], st, pk["hbm_gbs"]), "copies": R}
+        del g, copies
+        torch.cuda.empty_cache()
     return out
 
 
 def sweep_m_bench(W4, I, mats, pk):
     """The decode sweep at M = 4, 9 (a speculative-verify step: one token plus
-    eight drafted ones) and 16 (same packed copies, PDL graph per step)."""
+    eight drafted ones) and 16 (same packed copies, PDL graph per rotation)."""
     out = {}
+    R = len(mats[0]["copies"])
     for M in (4, 9, 16):
         xs = [I.sweep_x(M, m["K"], idx, device="cuda") for idx, m in enumerate(mats)]
         ys = [torch.empty(M, m["N"], dtype=torch.float32, device="cuda") for m in mats]
         ws = torch.empty(max(W4.w4a16_workspace_bytes(m["copies"][0], M) for m in mats) + 16,
                          dtype=torch.uint8, device="cuda")
 
-        def step(r):
-            def run():
+        def run():
+            for r in range(R):
                 for m, x, y in zip(mats, xs, ys):
                     W4.w4a16_gemv(m["copies"][r], x, out=y, workspace=ws, flags=W4.LAUNCH_PDL)
-            return run
-        graphs = [capture(step(r)) for r in range(ROTATE)]
-        ms = time_graphs(graphs, 60, 6)
+        g = capture(run)
+        st = summary(time_replays(g, REPEATS), R)
         nb = sum(m["bytes"] for m in mats)
-        out[f"M{M}"] = {"GB/s": round(nb / ms / 1e6, 1), "frac": round(nb / ms / 1e6 / pk["hbm_gbs"], 4),
-                        "us_per_step": round(ms * 1e3, 2)}
-        del graphs
+        out[f"M{M}"] = {**st, **rate(nb, st, pk["hbm_gbs"])}
+        del g
     return out
 
 
@@ -246,8 +297,9 @@ def rocm_gemv_bench(W4, I, pk):
     L = I.rocm_weights(device="cuda")
     for fmt in ("dual", "fast"):
         base = W4.pack_rocmfp4(L, fmt)
-        copies = [base] + [W4.PackedWeights(base.fmt, base.K, base.N, base.codes.clone()) for _ in range(ROTATE - 1)]
         nb = base.nbytes
+        R = n_copies(nb)
+        copies = [base] + [clone_packed(W4, base) for _ in range(R - 1)]
         for M in (1, 8):
             x = I.rocm_x(M, device="cuda")
             y = torch.empty(M, base.N, dtype=torch.float32, device="cuda")
@@ -257,10 +309,11 @@ def rocm_gemv_bench(W4, I, pk):
                 for c in copies:
                     W4.w4a16_gemv(c, x, out=y, workspace=ws)
             g = capture(run)
-            ms = time_graphs([g], 20, 3) / ROTATE
-            out[f"{fmt}_M{M}"] = {"us": round(ms * 1e3, 2), "GB/s": round(nb / ms / 1e6, 1),
-                                  "frac": round(nb / ms / 1e6 / pk["hbm_gbs"], 4), "bytes": nb}
+            st = summary(time_replays(g, REPEATS), R)
+            out[f"{fmt}_M{M}"] = {**st, **rate(nb, st, pk["hbm_gbs"]), "bytes": nb, "copies": R}
+            del g
         del copies
+        torch.cuda.empty_cache()
     return out
 
 
@@ -268,25 +321,27 @@ def gemm_bench(W4, I, pk):
     W, x = I.prefill(device="cuda")
     pw = W4.pack_nvfp4(W)
     del W
-    ws = [pw] + [W4.PackedWeights(pw.fmt, pw.K, pw.N, pw.codes.clone(), pw.scales.clone(),
-                                  pw.global_scale.clone()) for _ in range(ROTATE - 1)]
-    xs = [x] + [x.clone() for _ in range(ROTATE - 1)]
     M, K, N = 2048, 2560, 9728
+    R = n_copies(pw.nbytes + x.numel() * 2)
+    ws = [pw] + [clone_packed(W4, pw) for _ in range(R - 1)]
+    xs = [x] + [x.clone() for _ in range(R - 1)]
     y32 = torch.empty(M, N, dtype=torch.float32, device="cuda")
     y16 = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    wsp = torch.empty(W4.w4a16_workspace_bytes(pw, M), dtype=torch.uint8, device="cuda")
 
     def run():
         for w_, x_ in zip(ws, xs):
-            W4.w4a16_gemm(w_, x_, out_f32=y32, out_bf16=y16)
+            W4.w4a16_gemm(w_, x_, out_f32=y32, out_bf16=y16, workspace=wsp)
     g = capture(run)
-    ms = time_graphs([g], 10, 2) / ROTATE
+    st = summary(time_replays(g, REPEATS, warmup=2), R)
     flops = 2.0 * M * N * K
-    tf = flops / ms / 1e9
-    return {"config": "M=2048 K=2560 N=9728, NVFP4 Student-t weights, x N(0,1) with 16 columns x30, "
-                      "out fp32+bf16, 6 rotating input copies",
-            "us": round(ms * 1e3, 2), "TFLOP/s": round(tf, 1),
-            "frac": round(tf / pk["bf16_tflops"], 4), "peak": pk["bf16_tflops"],
-            "peak_unit": "TFLOP/s (measured cuBLAS bf16 burst)"}
+    tf = flops / st["median_us"] / 1e6
+    out = {"config": f"M=2048 K=2560 N=9728, NVFP4 Student-t weights, x N(0,1) with 16 columns x30, out fp32+bf16, "
+                     f"{R} rotating weight+x copies (> 4x L2); time per GEMM includes its x -> f16 pass",
+           **st, "TFLOP/s": round(tf, 1), "frac": round(tf / pk["bf16_tflops"], 4), "peak": pk["bf16_tflops"],
+           "peak_unit": f"TFLOP/s ({pk['source']} cuBLAS bf16 burst)"}
+    del g, ws, xs
+    return out
 
 
 def stream_bench(W4, I):
@@ -313,10 +368,11 @@ def stream_bench(W4, I):
                         for p in row:
                             W4.w4a16_gemv(p, xs[p.K], out=ys[p.N], workspace=ws, flags=W4.LAUNCH_PDL)
             g = capture(run)
-            ms = time_graphs([g], 5, 2)
+            st = summary(time_replays(g, 20, warmup=2))
             key = f"M{M}" + ("_looped" if loops == 2 else "")
+            ms = st["median_us"] / 1e3
             res[key] = {"tokens/s": round(M * 1e3 / ms, 1), "ms_per_token_pass": round(ms, 4),
-                        "GB/s": round(loops * nbytes / ms / 1e6, 1)}
+                        "GB/s": round(loops * nbytes / ms / 1e6, 1), **st}
             del g
     # one token with the projections that share an input issued together:
     # {q,k,v} and {gate,up} as grouped launches, o and down alone (4 launches per layer)
@@ -333,16 +389,18 @@ def stream_bench(W4, I):
                             W4.w4a16_gemv(p, x1[p.K], out=y1[grp[0]], flags=W4.LAUNCH_PDL)
                         else:
                             W4.w4a16_gemv_grouped([row[j] for j in grp], [x1[row[j].K] for j in grp],
-                                                  outs=[y1[j] for j in grp])
+                                                  outs=[y1[j] for j in grp], flags=W4.LAUNCH_PDL)
         g = capture(run)
-        ms = time_graphs([g], 5, 2)
+        st = summary(time_replays(g, 20, warmup=2))
+        ms = st["median_us"] / 1e3
         key = "M1_grouped" + ("_looped" if loops == 2 else "")
         res[key] = {"tokens/s": round(1e3 / ms, 1), "ms_per_token_pass": round(ms, 4),
-                    "GB/s": round(loops * nbytes / ms / 1e6, 1)}
+                    "GB/s": round(loops * nbytes / ms / 1e6, 1), **st}
         del g
     res["packed_bytes_per_pass"] = nbytes
-    res["config"] = ("36 layers x {q,k,v,o,gate,up,down}, NVFP4, one CUDA graph per token; M1/M16: 7 launches "
-                     "per layer with PDL; M1_grouped: {q,k,v} and {gate,up} grouped, 4 launches per layer")
+    res["config"] = ("36 layers x {q,k,v,o,gate,up,down}, NVFP4, one CUDA graph per token pass (2.04 GB > L2), "
+                     "median of 20 passes; M1/M16: 7 launches per layer with PDL; M1_grouped: {q,k,v} and "
+                     "{gate,up} grouped, 4 launches per layer")
     return res
 
 
@@ -366,53 +424,56 @@ def quality_report(W4, I):
     return out
 
 
+def time_calls(fn, reps=11, warmup=2):
+    """Milliseconds of each of `reps` calls of fn (CUDA events around each)."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+    ev[0].record()
+    for i in range(reps):
+        fn()
+        ev[i + 1].record()
+    torch.cuda.synchronize()
+    return [ev[i].elapsed_time(ev[i + 1]) for i in range(reps)]
+
+
 def pack_bench(W4, I):
+    """Each packer on a 2560 x 9728 matrix (the sweep's Student-t matrix for
+    NVFP4, the Laplace matrix for ROCmFP4 and Q4_0); median of 11 calls.  For
+    the HBM-bound packers GB/s counts bf16 read + packed bytes written."""
     out = {}
     W = I.sweep_weights(2560, 9728, 3, device="cuda")
-    Ws = [W] + [W.clone() for _ in range(2)]
-    g = capture(lambda: [W4.pack_nvfp4(w) for w in Ws])
-    ms = time_graphs([g], 10, 2) / len(Ws)
-    out["pack_nvfp4"] = {"shape": "K=2560 N=9728", "us": round(ms * 1e3, 2),
-                         "GB/s": round((W.numel() * 2 + W.numel() * 0.5625) / ms / 1e6, 1)}
     L = I.rocm_weights(device="cuda")
-    for fmt in ("dual", "fast"):
-        W4.pack_rocmfp4(L, fmt)
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        W4.pack_rocmfp4(L, fmt)
-        b.record()
-        torch.cuda.synchronize()
-        ms = a.elapsed_time(b)
-        out[f"pack_rocmfp4_{fmt}"] = {"shape": "K=2560 N=9728 Laplace", "ms": round(ms, 3),
-                                      "candidate_evals/s": round(127 * L.numel() / ms / 1e3, 1)}
-    W4.pack_q4_0(L)
-    torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    W4.pack_q4_0(L)
-    b.record()
-    torch.cuda.synchronize()
-    ms = a.elapsed_time(b)
-    out["pack_q4_0"] = {"shape": "K=2560 N=9728 Laplace", "us": round(ms * 1e3, 2),
-                        "GB/s": round((L.numel() * 2 + L.numel() * 0.5625) / ms / 1e6, 1)}
+    n = W.numel()
     imp = torch.rand(L.shape[1], generator=torch.Generator().manual_seed(5)).cuda() * 2.0
-    W4.pack_rocmfp4(L, "dual", importance=imp)
-    W4.pack_nvfp4(W, scale_search=W4.SCALE_MSE)
-    W4.pack_nvfp4(W, scale_search=W4.SCALE_MSE, importance=imp)
-    torch.cuda.synchronize()
-    for name, fn in (("pack_rocmfp4_dual_weighted", lambda: W4.pack_rocmfp4(L, "dual", importance=imp)),
-                     ("pack_nvfp4_scale_search", lambda: W4.pack_nvfp4(W, scale_search=W4.SCALE_MSE)),
-                     ("pack_nvfp4_scale_search_weighted",
-                      lambda: W4.pack_nvfp4(W, scale_search=W4.SCALE_MSE, importance=imp))):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        fn()
-        b.record()
-        torch.cuda.synchronize()
-        ms = a.elapsed_time(b)
-        out[name] = {"shape": "K=2560 N=9728", "ms": round(ms, 3),
-                     "candidate_evals/s": round(127 * W.numel() / ms / 1e3, 1)}
+    # preallocated outputs: the timed calls launch only the packer kernels
+    cd = torch.empty(9728, 1280, dtype=torch.uint8, device="cuda")
+    sc = torch.empty(9728, 160, dtype=torch.uint8, device="cuda")
+    gs = torch.empty(1, dtype=torch.float32, device="cuda")
+    wsp = torch.empty(W4.pack_nvfp4_workspace_bytes(), dtype=torch.uint8, device="cuda")
+    nv = W4.PackedWeights(W4.FMT_NVFP4, 2560, 9728, cd, sc, gs)
+    blk18 = torch.empty(9728, 80, 18, dtype=torch.uint8, device="cuda")
+    blk17 = torch.empty(9728, 80, 17, dtype=torch.uint8, device="cuda")
+    legs = [
+        ("pack_nvfp4", lambda: W4.pack_nvfp4(W, out=nv, workspace=wsp), "hbm", 2 + 0.5625),
+        ("pack_q4_0", lambda: W4.pack_q4_0(L, out=blk18), "hbm", 2 + 0.5625),
+        ("pack_rocmfp4_dual", lambda: W4.pack_rocmfp4(L, "dual", out=blk18), "search", None),
+        ("pack_rocmfp4_fast", lambda: W4.pack_rocmfp4(L, "fast", out=blk17), "search", None),
+        ("pack_rocmfp4_dual_weighted", lambda: W4.pack_rocmfp4(L, "dual", importance=imp, out=blk18), "search", None),
+        ("pack_nvfp4_scale_search", lambda: W4.pack_nvfp4(W, scale_search=W4.SCALE_MSE, out=nv, workspace=wsp),
+         "search", None),
+        ("pack_nvfp4_scale_search_weighted",
+         lambda: W4.pack_nvfp4(W, scale_search=W4.SCALE_MSE, importance=imp, out=nv, workspace=wsp), "search", None),
+    ]
+    for name, fn, kind, bpw in legs:
+        st = summary(time_calls(fn))
+        row = {"shape": "K=2560 N=9728", **st}
+        if kind == "hbm":
+            row["GB/s"] = round(n * bpw / st["median_us"] / 1e3, 1)
+        else:
+            row["candidate_evals/s"] = round(127 * n / st["median_us"] * 1e6, 1)
+        out[name] = row
     return out
 
 
@@ -443,6 +504,53 @@ def oracle_gemv_sample(mats, seconds: float):
     return done_bytes / el / 1e9, n, el, O.max_threads()
 
 
+def oracle_legs(I, seconds: float, mats):
+    """The oracle's other CPU legs, each a bounded sample (about `seconds` of work)
+    of the same workloads: the GEMV on one thread, the NVFP4 abs-max packer, the
+    ROCmFP4 Dual packer (exhaustive 127-candidate search) and the binary64 GEMM
+    of the prefill shape on a subsample of weight rows (time extrapolated
+    linearly to all 9728 rows)."""
+    import oracle as O
+    cores = O.max_threads()
+    legs = {}
+    O.set_threads(1)
+    try:
+        gbs, n, el, _ = oracle_gemv_sample(mats, seconds)
+    finally:
+        O.set_threads(cores)
+    legs["gemv_m1_1thread"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": 1,
+                               "sample": f"{n} whole-matrix GEMVs over the 5 sweep matrices in {el:.1f} s"}
+
+    def timed(fn):
+        t0 = time.perf_counter()
+        fn()
+        return time.perf_counter() - t0
+
+    W = I.sweep_weights(2560, 9728, 3)
+    rows = 4096
+    el = timed(lambda: O.pack_nvfp4(W[:rows].contiguous()))
+    legs["pack_nvfp4"] = {"value": round(rows * 2560 / el / 1e6, 2), "unit": "Mweights/s", "cores": cores,
+                          "sample": f"abs-max pack of {rows} of the 9728 rows of the 2560-wide Student-t matrix "
+                                    f"in {el:.2f} s"}
+    L = I.rocm_weights()
+    rows = 1024
+    el = timed(lambda: O.pack_rocmfp4(L[:rows].contiguous(), O.FMT_DUAL))
+    legs["pack_rocmfp4_dual"] = {"value": round(rows * 2560 / el / 1e6, 3), "unit": "Mweights/s", "cores": cores,
+                                 "sample": f"Dual pack (127 candidates per half) of {rows} of the 9728 rows of the "
+                                           f"2560-wide Laplace matrix in {el:.2f} s"}
+    Wp, x = I.prefill()
+    rows = 256
+    c, s_, g = O.pack_nvfp4(Wp[:rows].contiguous())
+    wh = O.dequant_nvfp4(c, s_, g)
+    el = timed(lambda: O.matmul(x, wh))
+    full_s = el * 9728 / rows
+    legs["gemm_prefill"] = {"value": round(2.0 * 2048 * 2560 * rows / el / 1e9, 3), "unit": "GFLOP/s",
+                            "cores": cores,
+                            "sample": f"binary64 GEMM M=2048 K=2560 over {rows} of the 9728 weight rows in {el:.2f} s; "
+                                      f"all rows extrapolated linearly: {full_s:.0f} s"}
+    return legs
+
+
 # ------------------------------------------------------------------------------ main
 def run_ours(args, world, rank, local):
     import w4a16_inputs as I
@@ -452,7 +560,9 @@ def run_ours(args, world, rank, local):
         B.build()
     pk = peaks()
     mats = sweep_setup(W4, I, M=1)
+    R = len(mats[0]["copies"])
     step_bytes = sum(m["bytes"] for m in mats)
+    assert step_bytes == sweep_step_bytes()
 
     xs, ys = [m["x"] for m in mats], [m["y"] for m in mats]
 
@@ -460,15 +570,15 @@ def run_ours(args, world, rank, local):
         def run():
             W4.w4a16_gemv_grouped([m["copies"][r] for m in mats], xs, outs=ys)
         return run
-    graphs = [capture(step_fn(r)) for r in range(ROTATE)]
-    # the ROTATE steps of one rotation in a single graph (one graph launch per
-    # ROTATE steps); single-step graphs cover a remainder
-    graph_rot = capture(lambda: [step_fn(r)() for r in range(ROTATE)])
+    graphs = [capture(step_fn(r)) for r in range(R)]
+    # the R steps of one rotation in a single graph (one graph launch per R
+    # steps); single-step graphs cover a remainder
+    graph_rot = capture(lambda: [step_fn(r)() for r in range(R)])
 
     def run_steps(n):
-        for _ in range(n // ROTATE):
+        for _ in range(n // R):
             graph_rot.replay()
-        for i in range(n % ROTATE):
+        for i in range(n % R):
             graphs[i].replay()
 
     clocks = Clocks(local)
@@ -476,7 +586,7 @@ def run_ours(args, world, rank, local):
     # untimed pre-heat (~1 s) so the timed steps run at load clocks, then W warm-up steps
     t_end = time.perf_counter() + 1.0
     while time.perf_counter() < t_end:
-        run_steps(60)
+        run_steps(4 * R)
         torch.cuda.synchronize()
     run_steps(args.warmup)
     torch.cuda.synchronize()
@@ -494,21 +604,26 @@ def run_ours(args, world, rank, local):
     ms_step = ms_total / args.steps
     value = replica_value(world, step_bytes, ms_total, args.steps)  # GB/s over all ranks
     launches = args.steps
+    # distribution of the step time: REPEATS rotations timed one by one
+    dist = summary(time_replays(graph_rot, REPEATS, warmup=2), R)
 
     # the step is one launch of the dominant kernel (the grouped M=1 GEMV)
     achieved = step_bytes / ms_step / 1e6
+    traffic, traffic_note = measured_traffic()
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-            "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": TRAFFIC_PER_LAUNCH,
+            "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": traffic,
             "kernel": "w4::gemv_nvfp4_m1_grouped_kernel",
             "note": f"one launch per step: algorithmic bytes of the 5 sweep matrices ({step_bytes} B) / "
-                    f"average step duration in the timed graphs (CUDA events on the launching stream); "
-                    f"peak = {pk['source']} copy bandwidth; traffic = ncu DRAM bytes of one launch"}
+                    f"average step duration over the timed steps (CUDA events on the launching stream); "
+                    f"peak = {pk['source']} copy bandwidth ({'of measured' if pk['source'] == 'measured' else 'of fallback'}); "
+                    f"{traffic_note}"}
 
     # end-to-end through the public API with pinned host buffers
     xh = [m["x"].cpu().pin_memory() for m in mats]
     yh = [torch.empty_like(m["y"], device="cpu").pin_memory() for m in mats]
     xd = [torch.empty_like(m["x"]) for m in mats]
     e2e_steps = max(20, min(args.steps, 200))
+
     def e2e_step(r):
         for i in range(len(mats)):
             xd[i].copy_(xh[i], non_blocking=True)
@@ -521,8 +636,8 @@ def run_ours(args, world, rank, local):
     barrier(world)
     ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ea.record()
-    for s in range(e2e_steps):
-        e2e_step(s % ROTATE)
+    for s_ in range(e2e_steps):
+        e2e_step(s_ % R)
     eb.record()
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(world, ea.elapsed_time(eb)) / e2e_steps
@@ -543,40 +658,44 @@ def run_ours(args, world, rank, local):
         torch.cuda.empty_cache()
 
     if not args.no_extras:
-        extra("sweep_separate_launches", lambda: separate_sweep(W4, mats))
-        extra("per_shape_isolated", lambda: per_shape(W4, mats))
+        extra("sweep_separate_launches", lambda: separate_sweep(W4, mats, pk))
         extra("sweep_skinny", lambda: sweep_m_bench(W4, I, mats, pk))
+        extra("per_shape_isolated", lambda: per_shape(W4, mats, pk))
         del graphs, graph_rot, mats
         torch.cuda.empty_cache()
         extra("gemm", lambda: gemm_bench(W4, I, pk))
+        extra("rocm_gemv", lambda: rocm_gemv_bench(W4, I, pk))
         extra("packers", lambda: pack_bench(W4, I))
         extra("quality", lambda: quality_report(W4, I))
-        extra("rocm_gemv", lambda: rocm_gemv_bench(W4, I, pk))
         extra("stream", lambda: stream_bench(W4, I))
     err = W4.w4_device_error(clear=True)
 
     cpu = None
     if rank == 0 and world == 1:
-        gbs, n, el, cores = oracle_gemv_sample(oracle_sweep_setup(I), args.cpu_seconds)
+        secs = max(2.0, args.cpu_seconds)
+        omats = oracle_sweep_setup(I)
+        gbs, n, el, cores = oracle_gemv_sample(omats, secs)
         cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                "sample": f"{n} whole-matrix oracle GEMVs (dequantise + fp64 dot) over the 5 sweep "
                          f"matrices at M=1 in {el:.1f} s"}
+        if not args.no_extras:
+            try:
+                cpu["legs"] = oracle_legs(I, secs / 3, omats)
+            except Exception as e:  # noqa: BLE001
+                cpu["legs"] = {"error": f"{type(e).__name__}: {e}"[:300]}
     if rank == 0:
         line = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4-w/bf16-x/f32-acc",
                 "data": "synthetic (seeded Student-t(4) weights, N(0,1) activations)",
-                "config": {"workload": WORKLOAD, "M": 1,
-                           "step": f"5 GEMVs in one grouped launch; {ROTATE} steps per CUDA graph",
-                           "l2": f"{ROTATE} rotating packed copies per matrix (248 MB > L2)",
-                           "bytes_per_step": step_bytes, "parallelism": f"replicas x{world}"},
+                "config": headline_config(world), "step_time": dist,
                 "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
                 "clocks": ck, "device_error": err, **extras}
         print(json.dumps(line), flush=True)
 
 
 def run_reference(args, world, rank):
-    """The oracle as the reference arm: same metric and workload on the host cores."""
+    """The oracle as the reference arm: same metric, workload and config on the host cores."""
     if rank != 0:
         return
     import w4a16_inputs as I
@@ -594,20 +713,37 @@ def run_reference(args, world, rank):
     sample = (f"per step: whole-matrix oracle GEMVs (dequantise + fp64 dot) over the 5 sweep matrices "
               f"at M=1 for >= {per_step:.1f} s; value = median over steps")
     line = {"impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * total_el / args.steps, 1), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "M": 1},
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * total_el / args.steps, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": headline_config(world),
             "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": O.max_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-# ncu-measured DRAM bytes (read + write) of one launch of the dominant kernel,
-# w4::gemv_nvfp4_m1_grouped_kernel, on the five sweep matrices
-# (profiles/gemv_nvfp4_m1_grouped_sweep.md).
-# Set to None when that kernel changes until it is measured again.
-TRAFFIC_PER_LAUNCH = 41381888
+# DRAM bytes (read + write, ncu dram__bytes_read.sum + dram__bytes_write.sum) of
+# one launch of the dominant kernel, w4::gemv_nvfp4_m1_grouped_kernel, on the
+# five sweep matrices, with the SHA-256 of the kernel sources it was measured
+# on.  The bench reports it only while those sources are unchanged.
+TRAFFIC = {"bytes": None, "source_sha256": None}
+TRAFFIC_SOURCES = ("common.cuh", "gemv_tc.cuh", "gemv_m1.cuh")
+
+
+def kernel_source_sha256() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, "w4a16_matmul_pack_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic():
+    sha = kernel_source_sha256()
+    if TRAFFIC["bytes"] is not None and TRAFFIC["source_sha256"] == sha:
+        return TRAFFIC["bytes"], "traffic = ncu DRAM bytes (read + write) of one launch, measured on these sources"
+    return None, f"traffic = null: no ncu capture of the current kernel sources (sha256 {sha[:16]})"
 
 
 def main():
