@@ -126,13 +126,13 @@ def test_save_reload_in_fresh_process(tmp_path):
     x = I.sweep_x(1, 2560, 1)
     pw = W4.pack_nvfp4(W.cuda())
     y = W4.w4a16_gemv(pw, x.cuda())
-    path = tmp_path / "packed.pt"
-    torch.save({"codes": pw.codes.cpu(), "scales": pw.scales.cpu(), "g": pw.global_scale.cpu(), "x": x,
-                "y": y.cpu()}, path)
+    path = tmp_path / "packed.w4"
+    W4.save_packed(pw, path)                     # versioned header + the packed bytes
+    torch.save({"x": x, "y": y.cpu()}, tmp_path / "xy.pt")
     code = (
         "import torch, w4a16_matmul_pack_b200 as W4\n"
-        f"d = torch.load({str(path)!r})\n"
-        "pw = W4.PackedWeights(W4.FMT_NVFP4, 2560, 1024, d['codes'].cuda(), d['scales'].cuda(), d['g'].cuda())\n"
+        f"pw = W4.load_packed({str(path)!r})\n"
+        f"d = torch.load({str(tmp_path / 'xy.pt')!r})\n"
         "y = W4.w4a16_gemv(pw, d['x'].cuda()).cpu()\n"
         "assert torch.equal(y, d['y']), (y - d['y']).abs().max()\n"
     )

@@ -17,6 +17,7 @@ from __future__ import annotations
 
 import ctypes
 import os
+import struct
 from dataclasses import dataclass
 from typing import Optional
 
@@ -26,7 +27,7 @@ __all__ = [
     "W4Error", "PackedWeights", "FMT_NVFP4", "FMT_ROCMFP4_DUAL", "FMT_ROCMFP4_FAST", "FMT_Q4_0",
     "pack_q4_0", "reconstruction_error", "plan_grouped",
     "LAUNCH_PDL", "set_wait_limit", "pack_nvfp4", "pack_rocmfp4", "w4a16_gemv", "w4a16_gemv_grouped", "w4a16_gemm",
-    "w4a16_workspace_bytes", "pack_nvfp4_workspace_bytes", "w4_encode_scalars",
+    "w4a16_workspace_bytes", "pack_nvfp4_workspace_bytes", "w4_encode_scalars", "save_packed", "load_packed",
     "w4_device_error", "lib", "library_path",
 ]
 
@@ -142,6 +143,63 @@ class PackedWeights:
         if self.scales is not None:
             n += self.scales.numel()
         return n
+
+
+# Packed weights on disk: a 64-byte little-endian header, then the codes, the
+# scales and the global scale as stored in memory.  Header: magic "W4A16PK",
+# layout version (1), then int32 fmt, K, N, block, and int64 byte counts of
+# codes, scales and global scale.
+_MAGIC = b"W4A16PK"
+_LAYOUT_VERSION = 1
+_HEADER = struct.Struct("<7sB4i3q")
+
+
+def _expected_bytes(fmt: int, K: int, N: int):
+    if fmt == FMT_NVFP4:
+        return N * K // 2, N * K // 16, 4
+    if fmt in BLOCK_BYTES or fmt == FMT_Q4_0:
+        return N * (K // 32) * (18 if fmt in (FMT_ROCMFP4_DUAL, FMT_Q4_0) else 17), 0, 0
+    raise ValueError(f"unknown format {fmt}")
+
+
+def save_packed(w: "PackedWeights", path) -> None:
+    """Write packed weights with a versioned header (format, K, N, block, sizes)."""
+    parts = [w.codes, w.scales, w.global_scale]
+    raw = [b"" if t is None else t.detach().contiguous().cpu().view(torch.uint8).numpy().tobytes() for t in parts]
+    if tuple(len(r) for r in raw) != _expected_bytes(w.fmt, w.K, w.N):
+        raise ValueError("packed tensors do not match their format and shape")
+    block = 16 if w.fmt == FMT_NVFP4 else 32
+    with open(path, "wb") as f:
+        f.write(_HEADER.pack(_MAGIC, _LAYOUT_VERSION, w.fmt, w.K, w.N, block, *(len(r) for r in raw)))
+        f.write(b"\0" * (64 - _HEADER.size))
+        for r in raw:
+            f.write(r)
+
+
+def load_packed(path, device="cuda") -> "PackedWeights":
+    """Read packed weights written by save_packed; refuses unknown versions and
+    headers whose sizes do not match the format and shape."""
+    with open(path, "rb") as f:
+        head = f.read(64)
+        if len(head) != 64:
+            raise ValueError("truncated header")
+        magic, ver, fmt, K, N, block, nc, ns, ng = _HEADER.unpack(head[:_HEADER.size])
+        if magic != _MAGIC or ver != _LAYOUT_VERSION:
+            raise ValueError(f"not a packed-weights file of layout version {_LAYOUT_VERSION}")
+        if K <= 0 or N <= 0 or block != (16 if fmt == FMT_NVFP4 else 32) or K % block:
+            raise ValueError("bad shape in header")
+        if (nc, ns, ng) != _expected_bytes(fmt, K, N):
+            raise ValueError("byte counts do not match the format and shape")
+        data = [f.read(n) for n in (nc, ns, ng)]
+        if [len(d) for d in data] != [nc, ns, ng] or f.read(1):
+            raise ValueError("truncated or oversized payload")
+    def t(b, shape, dtype):
+        return torch.frombuffer(bytearray(b), dtype=torch.uint8).view(dtype).reshape(shape).to(device)
+    if fmt == FMT_NVFP4:
+        return PackedWeights(fmt, K, N, t(data[0], (N, K // 2), torch.uint8), t(data[1], (N, K // 16), torch.uint8),
+                             t(data[2], (1,), torch.float32))
+    bb = nc // (N * (K // 32))
+    return PackedWeights(fmt, K, N, t(data[0], (N, K // 32, bb), torch.uint8))
 
 
 def pack_nvfp4_workspace_bytes() -> int:
