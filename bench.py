@@ -64,7 +64,8 @@ def headline_config(world: int) -> dict:
     """The config both arms report (the same keys and values)."""
     nb = sweep_step_bytes()
     return {"workload": WORKLOAD, "M": 1,
-            "step": "5 GEMVs in one grouped launch; one rotation of steps per CUDA graph",
+            "step": "5 GEMVs in one grouped launch (programmatic dependent launch between steps); one rotation "
+                    "of steps per CUDA graph",
             "l2": f"{n_copies(nb)} rotating packed copies per matrix ({n_copies(nb) * nb / 1e6:.0f} MB > 4x the "
                   f"126 MB L2)",
             "bytes_per_step": nb, "parallelism": f"replicas x{world}"}
@@ -568,7 +569,9 @@ def run_ours(args, world, rank, local):
 
     def step_fn(r):
         def run():
-            W4.w4a16_gemv_grouped([m["copies"][r] for m in mats], xs, outs=ys)
+            # programmatic dependent launch: a step streams its first weight
+            # stages while the previous step drains, and reads x only after it
+            W4.w4a16_gemv_grouped([m["copies"][r] for m in mats], xs, outs=ys, flags=W4.LAUNCH_PDL)
         return run
     graphs = [capture(step_fn(r)) for r in range(R)]
     # the R steps of one rotation in a single graph (one graph launch per R

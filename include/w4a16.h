@@ -210,10 +210,11 @@ size_t w4_reconstruction_workspace_bytes(void);
  * the end in binary64, so the output is finite whenever the exact result is.
  * ROCmFP4: level * scale products in binary32.  The result is deterministic (a
  * fixed summation order for a given shape and M).
- *   w        packed NVFP4 or ROCmFP4 weights (Q4_0: W4_ERR_UNSUPPORTED).
- *            K % 256 == 0 (NVFP4, ROCmFP4 Dual) or K % 512 == 0 (ROCmFP4 FAST),
- *            so that every row piece the kernels copy starts on 16 bytes;
- *            other K return W4_ERR_UNSUPPORTED.
+ *   w        packed NVFP4 or ROCmFP4 weights (Q4_0: W4_ERR_UNSUPPORTED), any K
+ *            the packers accept.  K % 256 == 0 (NVFP4, ROCmFP4 Dual) or
+ *            K % 512 == 0 (ROCmFP4 FAST) takes the tensor-core kernels (every
+ *            row piece they copy starts on 16 bytes); other K take a general
+ *            CUDA-core path (one warp per row, binary64 sums, no workspace).
  *   x        [M][K] BF16, 1 <= M <= 16.
  *   y        out [M][N] float.
  *   workspace>= w4a16_workspace_bytes(w, M) bytes (0 for most shapes: NULL
@@ -345,8 +346,10 @@ w4_status w4_device_error(int *out, int clear);
  * runs to its end: before exiting it still waits (up to 2 s, whatever this
  * limit) for the copies and MMAs it has already issued, so no asynchronous
  * write outlives it.  The outputs of a call whose wait expired are undefined.
- * Meant for exercising that failure path (a short limit makes the first waits
- * expire); it applies to kernels launched after it returns.  Synchronous.
+ * A wait that cannot pass at once suspends the thread in steps of about
+ * 128 ns; a limit below that step expires the first such wait.  Meant for
+ * exercising that failure path (a short limit makes the first waits expire);
+ * it applies to kernels launched after it returns.  Synchronous.
  */
 w4_status w4_set_wait_limit(unsigned long long ns);
 

@@ -76,11 +76,60 @@ def test_unsupported_inputs():
     with pytest.raises(W4.W4Error) as e:
         W4.w4a16_gemm(pw, I.activations(4, 96, 1).cuda())
     assert e.value.status == 3
-    b = O.pack_rocmfp4(I.matrix("laplace", 64, 128, 2, 0.015), O.FMT_DUAL)
-    pr = W4.PackedWeights(W4.FMT_ROCMFP4_DUAL, 128, 64, torch.from_numpy(b).cuda())
-    with pytest.raises(W4.W4Error) as e:
-        W4.w4a16_gemm(pr, I.activations(4, 128, 1).cuda())
-    assert e.value.status == 3
+    # ROCmFP4 rows must be whole 16-byte pieces: K % 256 (Dual), K % 512 (FAST)
+    for fmt, K in ((O.FMT_DUAL, 128), (O.FMT_FAST, 256)):
+        b = O.pack_rocmfp4(I.matrix("laplace", 64, K, 2, 0.015), fmt)
+        pr = W4.PackedWeights(fmt, K, 64, torch.from_numpy(b).cuda())
+        with pytest.raises(W4.W4Error) as e:
+            W4.w4a16_gemm(pr, I.activations(4, K, 1).cuda())
+        assert e.value.status == 3
+
+
+def rocm_check(fmt, W, x, rows=None, workspace=None):
+    b = O.pack_rocmfp4(W, fmt)
+    pr = W4.PackedWeights(fmt, W.shape[1], W.shape[0], torch.from_numpy(b).cuda())
+    y32, y16 = W4.w4a16_gemm(pr, x.cuda(), workspace=workspace)
+    torch.cuda.synchronize()
+    y32, y16 = np_of(y32), np_of(y16.float())
+    rows = np.arange(W.shape[0]) if rows is None else np.asarray(rows)
+    wh = np.concatenate([O.dequant_rocmfp4(b, fmt, int(r), 1) for r in rows])
+    yr, ar = O.matmul(x, wh)
+    assert_within_tolerance(y32[:, rows], yr, ar)
+    err16 = np.abs(y16[:, rows] - yr)
+    assert np.all(err16 <= 1e-3 * ar + half_ulp_bf16(yr)), float((err16 - 1e-3 * ar - half_ulp_bf16(yr)).max())
+
+
+@pytest.mark.parametrize("fmt", [O.FMT_DUAL, O.FMT_FAST])
+@pytest.mark.parametrize("with_workspace", [True, False])
+def test_rocm_prefill_full_size_sampled_rows(fmt, with_workspace):
+    """ROCmFP4 prefill GEMM on the 2560 x 9728 Laplace matrix, 2048 tokens with 16
+    outlier channels: f16 operands (x rescaled per row, with the workspace) and
+    BF16 operands (without); every token, sampled weight rows incl. both edges."""
+    W = I.rocm_weights()
+    _, x = I.prefill()
+    rng = np.random.default_rng(1)
+    rows = np.unique(np.concatenate([np.arange(0, 130), np.arange(9600, 9728), rng.integers(0, 9728, 48)]))
+    ws = None if with_workspace else torch.empty(0, dtype=torch.uint8, device="cuda")
+    rocm_check(fmt, W, x, rows, ws)
+
+
+@pytest.mark.parametrize("fmt", [O.FMT_DUAL, O.FMT_FAST])
+@pytest.mark.parametrize("M,N,K", [(1, 77, 512), (300, 200, 1024), (513, 384, 2048), (2048, 136, 512)])
+def test_rocm_ragged_shapes(fmt, M, N, K):
+    W = I.matrix("laplace", N, K, M + N + K, 0.015, 1e-3)
+    x = I.activations(M, K, 8, outlier_cols=min(16, K // 8))
+    rocm_check(fmt, W, x)
+
+
+def test_rocm_operand_modes_per_token_tile():
+    M, N, K = 600, 256, 1024
+    W = I.matrix("laplace", N, K, 21, 0.015, 1e-3)
+    x = I.activations(M, K, 22, outlier_cols=16).double()
+    x[300, :8] *= 2.0 ** 40            # token tile 1: BF16 operands
+    x[300, 8:16] *= 2.0 ** -40
+    x[520:530] *= 2.0 ** 100           # token tile 2: large, exact after scaling
+    rocm_check(O.FMT_DUAL, W, I.bf16_rne(x))
+    rocm_check(O.FMT_FAST, W, I.bf16_rne(x))
 
 
 def test_operand_modes_per_token_tile():

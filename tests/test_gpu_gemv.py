@@ -112,11 +112,20 @@ def test_deterministic_and_pdl_flag_and_graph():
     assert W4.w4_device_error(clear=True) == 0
 
 
-def test_unsupported_k_is_reported():
-    pw, _ = nvfp4_packed(I.matrix("normal", 4, 288, 1, 0.02))
-    with pytest.raises(W4.W4Error) as e:
-        W4.w4a16_gemv(pw, I.activations(1, 288, 1).cuda())
-    assert e.value.status == 3
+@pytest.mark.parametrize("K", [16, 272, 288, 2576])
+@pytest.mark.parametrize("M", [1, 5, 16])
+def test_nvfp4_any_k(K, M):
+    """K that is not a multiple of 256 takes the general path (binary64 sums)."""
+    pw, wh = nvfp4_packed(I.matrix("student_t4", 37, K, K + M, 0.02, 1e-3))
+    run_and_check(pw, wh, I.activations(M, K, 60 + M))
+
+
+@pytest.mark.parametrize("fmt,K", [(W4.FMT_ROCMFP4_DUAL, 32), (W4.FMT_ROCMFP4_DUAL, 288),
+                                   (W4.FMT_ROCMFP4_FAST, 256), (W4.FMT_ROCMFP4_FAST, 2592)])
+@pytest.mark.parametrize("M", [1, 8])
+def test_rocm_any_k(fmt, K, M):
+    pw, wh = rocm_packed(I.matrix("laplace", 41, K, K + M, 0.015, 1e-3), fmt)
+    run_and_check(pw, wh, I.activations(M, K, 70 + M))
 
 
 def test_save_reload_in_fresh_process(tmp_path):

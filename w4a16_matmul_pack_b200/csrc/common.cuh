@@ -71,6 +71,12 @@ __device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float v0, float v1) {
     return ((uint32_t)r & 0x77u) | s;
 }
 
+__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
@@ -97,13 +103,27 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
+// Non-blocking test of phase `parity`.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+// Test of phase `parity` that may suspend the thread for up to about
+// kSuspendNs while the phase is incomplete.
+constexpr uint32_t kSuspendNs = 128;
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity) : "memory");
+        : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity), "n"(kSuspendNs) : "memory");
     return ok != 0;
 }
 
@@ -113,23 +133,29 @@ __device__ __forceinline__ unsigned long long global_ns() {
     return t;
 }
 
-// Wait for phase `parity` of an mbarrier, for at most kWaitLimitNs.  `abort`
+// Wait for phase `parity` of an mbarrier, for at most g_wait_limit_ns.  `abort`
 // is a CTA-shared flag: once any wait of the CTA has expired every later wait
 // returns false at once, so all threads run to the end of the kernel (and
 // through its barriers) instead of spinning.  Returns false on expiry/abort and
-// records W4_ERR_TIMEOUT.
+// records W4_ERR_TIMEOUT.  The limit is checked after every suspension that
+// ended with the phase still incomplete; a limit shorter than one suspension
+// (kSuspendNs) allows none, so the first wait that cannot pass at once expires.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const unsigned long long t0 = global_ns(), limit = g_wait_limit_ns;
-    while (!mbar_try_wait(bar, parity)) {
-        if (*abort) return false;
-        if (global_ns() - t0 > limit) {
-            *abort = 1;
-            record_error(W4_ERR_TIMEOUT);
-            return false;
+    if (mbar_test_wait(bar, parity)) return true;
+    const unsigned long long limit = g_wait_limit_ns;
+    if (limit >= kSuspendNs) {
+        const unsigned long long t0 = global_ns();
+        for (;;) {
+            if (mbar_try_wait(bar, parity)) return true;
+            if (*abort) return false;
+            if (global_ns() - t0 > limit) break;
         }
+    } else if (*abort) {
+        return false;
     }
-    return true;
+    *abort = 1;
+    record_error(W4_ERR_TIMEOUT);
+    return false;
 }
 
 // Global -> shared bulk copy (no multicast), completion counted in bytes on `bar`.
@@ -186,7 +212,7 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, i
 // (still bounded, by kWaitLimitNs): for the completions a CTA must see before it
 // releases tensor memory or exits -- its own bulk copies and MMAs in flight.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_test_wait(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
     while (!mbar_try_wait(bar, parity)) {
         if (global_ns() - t0 > kWaitLimitNs) {

@@ -1,39 +1,50 @@
 // gemm.cuh -- prefill W4A16 GEMM on the 5th-generation tensor cores (sm_100a).
 //
-// y[m][n] = g * sum_k x[m][k] * (e2m1[n][k] * scale[n][k/16])   (NVFP4 weights,
-// "EdgeRock-4B-NVFP4" card, intro; BF16 activations).  e2m1 * scale has at most
-// 6 significant bits and lies in [2^-10, 2688], so it is exact in BF16 and in
-// f16: the dequant warps write it, per 64-k stage, into tensor memory, where it
-// is the A operand of tcgen05.mma kind::f16 (A from TMEM, B = x from shared
-// memory, FP32 accumulators in TMEM).  The global scale g is applied in the
+// NVFP4: y[m][n] = g * sum_k x[m][k] * (e2m1[n][k] * scale[n][k/16])
+// ("EdgeRock-4B-NVFP4" card, intro).  ROCmFP4 Dual / FAST: y[m][n] = sum_k
+// x[m][k] * level[n][k] * dec(u) ("rocmwhy" page, format table and sections
+// 01-02; no global scale).  x is BF16.  The decoded weight (e2m1 * scale, at
+// most 6 significant bits in [2^-10, 2688]; level * dec(u), at most 7 bits in
+// [2^-9, 4480]) is exact in BF16 and in f16, so the dequantised tile is an
+// exact operand of tcgen05.mma kind::f16: the dequant warps write it, per 64-k
+// stage, into tensor memory (A), B = x is staged by TMA in shared memory, and
+// the accumulators are FP32 in tensor memory.  g (NVFP4) is applied in the
 // epilogue.
 //
-// Tile: 128 weight rows (MMA M, A) x 192 tokens (MMA N, B = x, K-major with the
-// 128-byte swizzle, staged by TMA) x 64 k per stage.  Tensor memory holds four
-// A stages (32 columns each) and two 192-column accumulators (512 columns), so
-// the epilogue of a tile overlaps the MMAs of the next.  Persistent CTAs, one
-// per SM, walk the tiles n-major so that CTAs running together share the same
-// packed weight rows in L2.
+// Tile: 128 weight rows (MMA M) x 192 tokens (MMA N) x 64 k per stage.  Tensor
+// memory holds four A stages (32 columns each) and two 192-column accumulators
+// (512 columns), so the epilogue of a tile overlaps the MMAs of the next.
+// Persistent CTAs, one per SM, walk the tiles n-major so that CTAs running
+// together share the same packed weight rows in L2.
 //
-// Warp roles (15 warps):
-//   warp 0      TMA producer: x tiles and the packed codes (128-byte swizzle,
-//               256 k per codes stage), no multicast.
-//   warp 1      allocates / frees the 512 TMEM columns; MMA issuer (one lane):
-//               4 x (128x192x16) per stage, commits to the stage barriers and
-//               to the accumulator barrier per tile.  It never waits on an
-//               mbarrier: a thread with MMAs queued stalls on any shared-memory
-//               access until they drain (measured: one wait per four
-//               128x256x16 MMAs turns 128 cycles per MMA into 270), so warp 14
-//               waits and releases it through named barrier 2 once per stage.
-//   warps 2-5   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
-//               32*(w%4)..+31), times g (and 2^sigma_m, below), float32 / BF16
-//               stores.
-//   warps 6-13  dequantise: warp w owns TMEM lanes 32*(w%4)..+31 = weight rows;
-//               thread (row r, k-half h) turns 32 codes + 2 scales of row r into
-//               16 words and stores them with one tcgen05.st, two stages per
-//               round (one store wait and one arrival per round).
-//   warp 14     waits on the x / A stage barriers and the accumulator barriers
-//               for the MMA issuer.
+// The dequantisation is what limits a tile of this shape if it runs as one
+// chain per stage (decode, store to tensor memory, wait for the store, signal
+// the MMA): the chain takes several times the 4 x 96 cycles of MMA per stage.
+// So it runs in four groups of four warps, group g owning A stage g (the k-steps
+// i = g mod 4): a group decodes its next k-step into registers while the MMAs
+// of the previous use of its stage run, and only the store and its signal wait
+// for the stage to be free.  Each thread writes one weight row (one TMEM lane)
+// of 64 k with one tcgen05.st.
+//
+// Warp roles (24 warps):
+//   warp 0       TMA producer of x (the 192 x 64 BF16 / f16 tile of each stage,
+//                128-byte swizzle, six stages), no multicast.
+//   warp 1       allocates / frees the 512 TMEM columns; MMA issuer (one lane):
+//                4 x (128x192x16) per stage, commits to the stage barriers and
+//                to the accumulator barrier per tile.  It never waits on an
+//                mbarrier: a thread with MMAs queued stalls on any shared-memory
+//                access until they drain, so warp 22 waits and releases it
+//                through named barrier 2 once per stage.
+//   warps 2-5    epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
+//                32*(w%4)..+31), times g (and 2^sigma_m, below), FP32 / BF16
+//                stores.
+//   warps 6-21   dequantise, four groups of four (warp w owns TMEM lanes
+//                32*(w%4)..+31 = weight rows).
+//   warp 22      waits on the x / A stage barriers and the accumulator barriers
+//                for the MMA issuer.
+//   warp 23      TMA producer of the packed weights (NVFP4: codes with the
+//                128-byte swizzle plus the E4M3 scales, 256 k per stage; ROCmFP4:
+//                the 18- / 17-byte blocks of 128 rows, 256 / 512 k per stage).
 // Every mbarrier wait is bounded (common.cuh: mbar_wait).
 //
 // Operand precision per tile of 192 tokens.  In f16, e2m1 * scale costs one cvt
@@ -44,10 +55,10 @@
 // |x * 2^-sigma_m| below 2^-17, or Inf / NaN).  A tile whose rows all converted
 // exactly runs kind::f16 with f16 operands and the epilogue multiplies token m
 // by 2^sigma_m; any other tile (or every tile, without a workspace) runs on
-// BF16 operands (e2m1 -> f16 -> binary32 * scale -> BF16).
+// BF16 operands (decoded in binary32, times 2^fold for NVFP4, rounded to BF16).
 #pragma once
 
-#include "common.cuh"
+#include "gemv_tc.cuh"
 
 namespace w4 {
 
@@ -56,17 +67,37 @@ namespace gemm {
 constexpr int BM = 128;      // weight rows per tile (MMA M)
 constexpr int BN = 192;      // tokens per tile (MMA N)
 constexpr int BK = 64;       // k per stage (one 128-byte swizzle row of BF16)
-constexpr int STAGES = 4;
-constexpr int kWarps = 15;
+constexpr int STAGES = 4;    // A stages in tensor memory (32 columns each), one per dequant group
+constexpr int XSTAGES = 6;   // x stages in shared memory
+constexpr int kGroups = STAGES;
+constexpr int kDqWarp0 = 6;
+constexpr int kDqWarps = 4 * kGroups;
+constexpr int kWaitWarp = kDqWarp0 + kDqWarps;   // 22
+constexpr int kWProdWarp = kWaitWarp + 1;        // 23
+constexpr int kWarps = kWProdWarp + 1;           // 24
 constexpr int kThreads = kWarps * 32;
-constexpr int kDequantThreads = 256;
 constexpr int kEpiThreads = 128;
 constexpr uint32_t X_STAGE_BYTES = BN * BK * 2;   // 24 KB
 constexpr uint32_t TMEM_COLS = 512;               // 4 A stages (32 columns each) + two 192-column accumulators
 constexpr uint32_t ACC_COL0 = STAGES * (BK / 2);  // accumulators after the A stages
-constexpr int WK = 256;                           // k per packed-weight stage (4 k-steps)
-constexpr int WSTAGES = 4;
-constexpr uint32_t W_STAGE_BYTES = BM * WK / 2;   // 16 KB of codes (128 rows x 128 bytes)
+constexpr int kMaxTilesM = 256;   // token tiles whose operand mode is kept in shared memory (M <= 49152)
+
+// Packed-weight stages per format: k per stage (WK), bytes per row of a stage,
+// block bytes, scale bytes per row, stages in the ring.
+//   NVFP4: 256 k = 128 code bytes per row (128-byte swizzle) + 16 scale bytes.
+//   ROCmFP4 Dual: 256 k = 8 blocks of 18 bytes = 144 bytes per row; FAST: 512 k =
+//          16 blocks of 17 bytes = 272 bytes (a TMA box row must be a multiple of
+//          16 bytes).  Scales travel inside the blocks.  No swizzle.
+template <int FMT> struct WFormat;
+template <> struct WFormat<W4_FMT_NVFP4> {
+    static constexpr int WK = 256, ROW_BYTES = 128, BB = 0, SCALE_BYTES = 16, WSTAGES = 4;
+};
+template <> struct WFormat<W4_FMT_ROCMFP4_DUAL> {
+    static constexpr int WK = 256, ROW_BYTES = 144, BB = 18, SCALE_BYTES = 0, WSTAGES = 4;
+};
+template <> struct WFormat<W4_FMT_ROCMFP4_FAST> {
+    static constexpr int WK = 512, ROW_BYTES = 272, BB = 17, SCALE_BYTES = 0, WSTAGES = 2;
+};
 
 // Instruction descriptor, kind::f16: D = F32 (bit 4), A = BF16 (bits 7-9),
 // B = BF16 (bits 10-12), both K-major, N >> 3 at bit 17, M >> 4 at bit 24.
@@ -74,20 +105,22 @@ constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >
                            ((uint32_t)(BM >> 4) << 24);
 // The same with A = B = F16 (format 0).
 constexpr uint32_t IDESC_F16 = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
-constexpr int kMaxTilesM = 256;
-constexpr int kWaitWarp = 14;     // waits on mbarriers for the MMA issuer (warp 1)   // token tiles whose operand mode is kept in shared memory (M <= 65536)
 
+template <int FMT>
 struct SharedStorage {
-    uint8_t x[STAGES][X_STAGE_BYTES];   // 1024-byte aligned (swizzle atoms)
-    uint8_t w[WSTAGES][W_STAGE_BYTES];  // packed codes, 128-byte swizzle
-    uint64_t w_full[WSTAGES], w_empty[WSTAGES];
-    uint64_t x_full[STAGES], x_empty[STAGES];
+    using F = WFormat<FMT>;
+    static constexpr uint32_t W_CODE_BYTES = BM * F::ROW_BYTES;
+    static constexpr uint32_t W_STAGE_BYTES = W_CODE_BYTES + BM * F::SCALE_BYTES;
+    uint8_t x[XSTAGES][X_STAGE_BYTES];          // 1024-byte aligned (swizzle atoms)
+    uint8_t w[F::WSTAGES][W_STAGE_BYTES];       // packed weights of 128 rows (each stage 1024-byte aligned)
+    uint64_t w_full[F::WSTAGES], w_empty[F::WSTAGES];
+    uint64_t x_full[XSTAGES], x_empty[XSTAGES];
     uint64_t a_full[STAGES], a_empty[STAGES];
     uint64_t acc_full[2], acc_empty[2];
-    uint64_t mma_done;                  // the issuer's last commit: every MMA has finished
+    uint64_t mma_done;                          // the issuer's last commit: every MMA has finished
     uint32_t tmem_base;
     int abort;
-    int f16_tile[kMaxTilesM];   // token tile mt runs with f16 operands (else BF16)
+    int f16_tile[kMaxTilesM];                   // token tile mt runs with f16 operands (else BF16)
 };
 
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row atoms of
@@ -104,22 +137,13 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ void mma_f16kind(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                            uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
-}
-
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t a) {
     uint4 v;
     asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
     return v;
 }
 
-// The same with A from tensor memory (K-major: lane = row, 32-bit column = two k).
+// D (TMEM) += A (TMEM; K-major: lane = row, 32-bit column = two k) * B (shared memory).
 __device__ __forceinline__ void mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
                                        uint32_t accumulate) {
     asm volatile(
@@ -129,12 +153,15 @@ __device__ __forceinline__ void mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_
         ::"r"(tmem_d), "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *v) {
+// 32 consecutive 32-bit columns of this warp's 32 TMEM lanes (one lane per thread).
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
     asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-            taddr),
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
         "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
-        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
+        "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+        "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
         : "memory");
 }
 
@@ -143,21 +170,17 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
                  ::"r"(smem_addr(bar)) : "memory");
 }
 
-#define W4_TMEM_LD32(taddr, v)                                                                              \
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "                                                  \
-                 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"                                   \
-                 "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"                  \
+#define W4_TMEM_LD16(taddr, v)                                                                              \
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 "                                                  \
+                 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"                           \
                  : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),       \
                    "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),   \
-                   "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),             \
-                   "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),             \
-                   "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])              \
+                   "=r"(v[14]), "=r"(v[15])                                                                  \
                  : "r"(taddr))
 
 // 4 code bytes (8 E2M1 values, element 2i in the low nibble of byte i) times a
-// scale -> 4 BF16x2 words.  Exact.
-__device__ __forceinline__ uint4 dequant8(uint32_t cw, float s) {
-    uint32_t o[4];
+// scale -> 4 BF16x2 words at o[0..3].  Exact.
+__device__ __forceinline__ void dequant8_bf16(uint32_t cw, float s, uint32_t *o) {
 #pragma unroll
     for (int i = 0; i < 4; i++) {
         const uint32_t h = e2m1x2_to_f16x2(cw >> (8 * i));
@@ -166,84 +189,159 @@ __device__ __forceinline__ uint4 dequant8(uint32_t cw, float s) {
         const __nv_bfloat162 b = __float22bfloat162_rn(v);
         o[i] = *reinterpret_cast<const uint32_t *>(&b);
     }
-    return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 // The same 8 weights as f16x2 words: cvt E2M1 -> f16x2, HMUL2 by the scale
-// (s2 = the scale in both halves).  Exact (at most 6 significant bits, in
-// [2^-10, 2688]).
-__device__ __forceinline__ uint4 dequant8_f16(uint32_t cw, uint32_t s2) {
-    uint32_t o[4];
+// (s2 = the scale in both halves).  Exact.
+__device__ __forceinline__ void dequant8_f16(uint32_t cw, uint32_t s2, uint32_t *o) {
 #pragma unroll
-    for (int i = 0; i < 4; i++) {
-        const uint32_t h = e2m1x2_to_f16x2(cw >> (8 * i));
-        const __half2 v = __hmul2(*reinterpret_cast<const __half2 *>(&h), *reinterpret_cast<const __half2 *>(&s2));
-        o[i] = *reinterpret_cast<const uint32_t *>(&v);
-    }
-    return make_uint4(o[0], o[1], o[2], o[3]);
+    for (int i = 0; i < 4; i++) o[i] = hmul2_u32(e2m1x2_to_f16x2(cw >> (8 * i)), s2);
 }
 
-// The power of two a BF16-operand tile folds into its weights: the exponent of
-// g, clamped so that e2m1 * scale * 2^fold stays an exact BF16 value (e2m1 *
-// scale lies in [2^-10, 2688] with at most 6 significant bits).  The products
-// x * A then have the size of the true x * w_hat, so the accumulator overflows
-// only if the result itself does; the epilogue multiplies by g * 2^-fold.
+// One ROCmFP4 block (32 weights at shared-memory byte address A: Dual = two
+// UE4M3 half scales + 16 code bytes, FAST = one scale + 16 code bytes; code byte
+// j holds elements j (low nibble) and j + 16) -> 16 words in k order at o[0..15],
+// word c = elements 2c, 2c+1, each level * dec(u) ("rocmwhy" page, format table
+// and sections 01-02), as f16x2 (f16) or BF16x2.  Codebook10 level / 2 is the
+// E2M1 value of the same nibble with index 7 (6) lowered to 5, so a level is the
+// E2M1 conversion clamped to [-5, 5] times 2; level * dec(u) has at most 7
+// significant bits and lies in [2^-9, 4480], exact in f16 and in BF16.  The
+// block may start on any byte: six aligned words are read and realigned with
+// funnel shifts (up to 6 bytes past the block, still inside shared memory).
+template <bool DUAL>
+__device__ __forceinline__ void dequant_rocm_block(uint32_t A, bool f16, uint32_t *o) {
+    const uint32_t base = A & ~3u, sh = (A & 3u) * 8u;
+    uint32_t W[6], S[5];
+#pragma unroll
+    for (int i = 0; i < 6; i++) W[i] = ld_shared_u32(base + 4u * i);
+#pragma unroll
+    for (int i = 0; i < 5; i++) S[i] = __funnelshift_r(W[i], W[i + 1], sh);   // bytes A + 4i .. + 3
+    const uint32_t u0 = S[0] & 0xFFu, u1 = DUAL ? (S[0] >> 8) & 0xFFu : u0;
+    uint32_t C[4];
+#pragma unroll
+    for (int j = 0; j < 4; j++) C[j] = __funnelshift_r(S[j], S[j + 1], DUAL ? 16 : 8);
+    const __half2 lim = __floats2half2_rn(5.0f, 5.0f), nlim = __floats2half2_rn(-5.0f, -5.0f);
+    const uint32_t sc = e4m3x2_to_f16x2(u0 | (u1 << 8));           // (dec u0, dec u1), exact
+    const __half2 sc2 = __hadd2(*reinterpret_cast<const __half2 *>(&sc), *reinterpret_cast<const __half2 *>(&sc));
+    const __half2 s0 = __low2half2(sc2), s1 = __high2half2(sc2);    // 2 dec(u): elements 0..15 / 16..31
+    const float2 f2 = __half22float2(sc2);
+#pragma unroll
+    for (int q = 0; q < 4; q++) {
+        // low nibbles: elements 4q .. 4q+3; high nibbles: 4q+16 .. 4q+19; pair them as (k, k+1)
+        const uint32_t lo = C[q] & 0x0F0F0F0Fu, hi = (C[q] >> 4) & 0x0F0F0F0Fu;
+        const uint32_t plo = (lo | (lo >> 4)) & 0x00FF00FFu, phi = (hi | (hi >> 4)) & 0x00FF00FFu;
+        const uint32_t pb[4] = {plo, plo >> 16, phi, phi >> 16};
+        const int col[4] = {2 * q, 2 * q + 1, 8 + 2 * q, 9 + 2 * q};
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+            const uint32_t h = e2m1x2_to_f16x2(pb[e]);
+            const __half2 v = __hmin2(__hmax2(*reinterpret_cast<const __half2 *>(&h), nlim), lim);
+            uint32_t w;
+            if (f16) {
+                const __half2 r = __hmul2(v, e < 2 ? s0 : s1);
+                w = *reinterpret_cast<const uint32_t *>(&r);
+            } else {
+                const float sv = e < 2 ? f2.x : f2.y;
+                const float2 fv = __fmul2_rn(__half22float2(v), make_float2(sv, sv));
+                const __nv_bfloat162 b = __float22bfloat162_rn(fv);
+                w = *reinterpret_cast<const uint32_t *>(&b);
+            }
+            o[col[e]] = w;
+        }
+    }
+}
+
+// The power of two a BF16-operand NVFP4 tile folds into its weights: the
+// exponent of g, clamped so that e2m1 * scale * 2^fold stays an exact BF16 value
+// (e2m1 * scale lies in [2^-10, 2688] with at most 6 significant bits).  The
+// products x * A then have the size of the true x * w_hat, so the accumulator
+// overflows only if the result itself does; the epilogue multiplies by
+// g * 2^-fold.
 __device__ __forceinline__ int bf16_fold(float g) {
     const int eg = (int)((__float_as_uint(g) >> 23) & 0xFF) - 127;
     return max(-123, min(116, eg));
 }
 
+// g * 2^e as binary32 when it is exactly a normal binary32 value or zero, else
+// NaN (the caller then forms the product in binary64).
+__device__ __forceinline__ float epilogue_factor(float g, int e) {
+    const double gd = (double)g * __longlong_as_double((long long)(1023 + e) << 52);
+    const double a = fabs(gd);
+    return (gd == 0.0 || (a >= 0x1p-126 && a < 0x1p128)) ? (float)gd : __int_as_float(0x7FC00000);
+}
+
 // Row m of x -> f16 as x * 2^-sigma_m, sigma_m chosen so that the row's largest
 // |x * 2^-sigma_m| lies in [2^14, 2^15); bad[m] = 1 when some nonzero value
 // lands below 2^-17 (then it may be inexact in f16) or the row holds Inf / NaN.
-// One block per row; every launch rewrites sigma and bad of every row.
-__global__ void __launch_bounds__(256) x_to_f16_kernel(const uint16_t *x, uint16_t *xh, int *sigma, int *bad, int K) {
-    __shared__ uint32_t red[8];
-    const int m = blockIdx.x;
+// One warp per row, eight rows per block; every launch rewrites sigma and bad of
+// every row.  Rows of up to kXRowVec * 32 * 8 values are read once (kept in
+// registers); longer rows are read twice.
+constexpr int kXRowVec = 16;
+
+__device__ __forceinline__ uint4 x_row_to_f16(uint4 v, int sg, bool &b) {
+    const float tiny = 7.62939453125e-06f;   // 2^-17
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        const float a0 = mul_pow2(__uint_as_float(w[j] << 16), -sg), a1 = mul_pow2(__uint_as_float(w[j] & 0xFFFF0000u), -sg);
+        b |= (a0 != 0.0f && fabsf(a0) < tiny) | (a1 != 0.0f && fabsf(a1) < tiny);
+        const __half2 hv = __floats2half2_rn(a0, a1);
+        o[j] = *reinterpret_cast<const uint32_t *>(&hv);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__device__ __forceinline__ uint32_t absmax_bf16x8(uint32_t mx, uint4 v) {
+    mx = __vmaxu2(mx, v.x & 0x7FFF7FFFu);
+    mx = __vmaxu2(mx, v.y & 0x7FFF7FFFu);
+    mx = __vmaxu2(mx, v.z & 0x7FFF7FFFu);
+    return __vmaxu2(mx, v.w & 0x7FFF7FFFu);
+}
+
+__global__ void __launch_bounds__(256) x_to_f16_kernel(const uint16_t *x, uint16_t *xh, int *sigma, int *bad, int M,
+                                                       int K) {
+    const int m = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (m >= M) return;   // whole warps
     const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)m * K);
     uint4 *dst = reinterpret_cast<uint4 *>(xh + (size_t)m * K);
     const int nv = K / 8;
+    const bool in_regs = nv <= kXRowVec * 32;
+    uint4 keep[kXRowVec];
     uint32_t mx = 0;
-    for (int i = threadIdx.x; i < nv; i += blockDim.x) {
-        const uint4 v = __ldg(src + i);
-        mx = __vmaxu2(mx, v.x & 0x7FFF7FFFu);
-        mx = __vmaxu2(mx, v.y & 0x7FFF7FFFu);
-        mx = __vmaxu2(mx, v.z & 0x7FFF7FFFu);
-        mx = __vmaxu2(mx, v.w & 0x7FFF7FFFu);
+    if (in_regs) {
+#pragma unroll
+        for (int r = 0; r < kXRowVec; r++) {
+            const int i = lane + r * 32;
+            keep[r] = i < nv ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+            mx = absmax_bf16x8(mx, keep[r]);
+        }
+    } else {
+        for (int i = lane; i < nv; i += 32) mx = absmax_bf16x8(mx, __ldg(src + i));
     }
     mx = max(mx & 0xFFFFu, mx >> 16);
 #pragma unroll
     for (int o = 16; o; o >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
-    __syncthreads();
-    for (int i = 0; i < 8; i++) mx = max(mx, red[i]);
     const int sg = (mx == 0) ? 0 : max((int)(mx >> 7), 1) - 127 - 14;
-    const float tiny = 7.62939453125e-06f;   // 2^-17
     bool b = mx >= 0x7F80u;
-    for (int i = threadIdx.x; i < nv; i += blockDim.x) {
-        const uint4 v = __ldg(src + i);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        uint32_t o[4];
+    if (in_regs) {
 #pragma unroll
-        for (int j = 0; j < 4; j++) {
-            const float x0 = __uint_as_float(w[j] << 16), x1 = __uint_as_float(w[j] & 0xFFFF0000u);
-            const float a0 = ldexpf(x0, -sg), a1 = ldexpf(x1, -sg);
-            b |= (a0 != 0.0f && fabsf(a0) < tiny) | (a1 != 0.0f && fabsf(a1) < tiny);
-            const __half2 hv = __floats2half2_rn(a0, a1);
-            o[j] = *reinterpret_cast<const uint32_t *>(&hv);
+        for (int r = 0; r < kXRowVec; r++) {
+            const int i = lane + r * 32;
+            if (i < nv) dst[i] = x_row_to_f16(keep[r], sg, b);
         }
-        dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    } else {
+        for (int i = lane; i < nv; i += 32) dst[i] = x_row_to_f16(__ldg(src + i), sg, b);
     }
-    const int any = __syncthreads_or(b ? 1 : 0);
-    if (threadIdx.x == 0) {
+    const bool any = __any_sync(0xFFFFFFFFu, b);
+    if (lane == 0) {
         sigma[m] = sg;
-        bad[m] = any;
+        bad[m] = any ? 1 : 0;
     }
 }
 
 struct Params {
-    const uint8_t *codes;
-    const uint8_t *scales;
+    const uint8_t *scales;   // NVFP4 scales [N][K/16], read directly when scales_tma == 0
     const float *gscale;
     float *y32;
     __nv_bfloat16 *y16;
@@ -251,14 +349,21 @@ struct Params {
     const int *sigma;    // [M] power of two of each f16 row
     int M, N, K;
     int tiles_m, tiles_n;
+    int scales_tma;      // NVFP4 scales staged by TMA with the codes (K % 256 == 0: 16-byte rows)
 };
 
+template <int FMT>
 __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ CUtensorMap xmap,
                                                             const __grid_constant__ CUtensorMap xmap16,
-                                                            const __grid_constant__ CUtensorMap cmap, const Params p) {
+                                                            const __grid_constant__ CUtensorMap cmap,
+                                                            const __grid_constant__ CUtensorMap smap, const Params p) {
+    using SS = SharedStorage<FMT>;
+    using F = WFormat<FMT>;
+    constexpr int WK = F::WK, ROW_BYTES = F::ROW_BYTES, BB = F::BB, WSTAGES = F::WSTAGES;
+    constexpr int KQ = WK / BK;             // k-steps per packed-weight stage
+    constexpr bool NV = FMT == W4_FMT_NVFP4;
     extern __shared__ uint8_t smem_raw[];
-    SharedStorage &sh = *reinterpret_cast<SharedStorage *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    SS &sh = *reinterpret_cast<SS *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KT = p.K / BK;
     const int ntiles = p.tiles_m * p.tiles_n;
@@ -266,15 +371,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
 
     if (threadIdx.x == 0) {
         sh.abort = 0;
-        for (int i = 0; i < STAGES; i++) {
+        for (int i = 0; i < XSTAGES; i++) {
             mbar_init(&sh.x_full[i], 1);
             mbar_init(&sh.x_empty[i], 1);
-            mbar_init(&sh.a_full[i], kDequantThreads / 32);   // one arrival per dequant warp
+        }
+        for (int i = 0; i < STAGES; i++) {
+            mbar_init(&sh.a_full[i], 4);   // the four warps of group i
             mbar_init(&sh.a_empty[i], 1);
         }
         for (int i = 0; i < WSTAGES; i++) {
             mbar_init(&sh.w_full[i], 1);
-            mbar_init(&sh.w_empty[i], kDequantThreads / 32);
+            mbar_init(&sh.w_empty[i], kDqWarps);
         }
         for (int i = 0; i < 2; i++) {
             mbar_init(&sh.acc_full[i], 1);
@@ -285,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     }
     const bool use_f16 = p.bad != nullptr && p.tiles_m <= kMaxTilesM;
     for (int i = threadIdx.x; i < kMaxTilesM; i += kThreads) sh.f16_tile[i] = use_f16 ? 1 : 0;
-    if (warp == 0) {
+    if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                      ::"r"(smem_addr(&sh.tmem_base)), "r"(TMEM_COLS));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -304,33 +411,49 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     if (warp == 0) {
         // ---------------------------- x producer (TMA) ----------------------------
         if (lane == 0) {
-            int it = 0, wit = 0;
-            for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+            int it = 0;
+            for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x) {
                 const int m0 = (t % p.tiles_m) * BN;
-                const int n0 = (t / p.tiles_m) * BM;
+                const CUtensorMap *xm = sh.f16_tile[t % p.tiles_m] ? &xmap16 : &xmap;
                 for (int kt = 0; kt < KT; kt++, it++) {
-                    if (kt % (WK / BK) == 0) {   // packed codes of the next 256 k
-                        const int ws = wit % WSTAGES;
-                        if (wit >= WSTAGES) mbar_wait(&sh.w_empty[ws], ((wit / WSTAGES) - 1) & 1, abort);
-                        if (*abort) break;
-                        mbar_arrive_expect_tx(&sh.w_full[ws], W_STAGE_BYTES);
-                        tma_load_2d(sh.w[ws], &cmap, kt * (BK / 2), n0, &sh.w_full[ws]);
-                        wit++;
-                    }
-                    const int s = it % STAGES;
-                    if (it >= STAGES) mbar_wait(&sh.x_empty[s], ((it / STAGES) - 1) & 1, abort);
+                    const int s = it % XSTAGES;
+                    if (it >= XSTAGES) mbar_wait(&sh.x_empty[s], ((it / XSTAGES) - 1) & 1, abort);
                     if (*abort) break;
                     mbar_arrive_expect_tx(&sh.x_full[s], X_STAGE_BYTES);
-                    tma_load_2d(sh.x[s], sh.f16_tile[t % p.tiles_m] ? &xmap16 : &xmap, kt * BK, m0, &sh.x_full[s]);
+                    tma_load_2d(sh.x[s], xm, kt * BK, m0, &sh.x_full[s]);
                 }
-                if (*abort) break;
             }
             // every issued copy has landed before the CTA can exit (after an abort
             // the loop above stops early, with copies possibly in flight)
-            drain_ring(sh.w_full, WSTAGES, wit);
-            drain_ring(sh.x_full, STAGES, it);
+            drain_ring(sh.x_full, XSTAGES, it);
         }
         __syncwarp();   // the whole warp reaches the final barrier together (it is .aligned)
+    } else if (warp == kWProdWarp) {
+        // ------------------------ packed-weight producer (TMA) ------------------------
+        if (lane == 0) {
+            int wit = 0;
+            for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x) {
+                const int n0 = (t / p.tiles_m) * BM;
+                for (int kw = 0; kw < KT; kw += KQ, wit++) {
+                    const int ws = wit % WSTAGES;
+                    if (wit >= WSTAGES) mbar_wait(&sh.w_empty[ws], ((wit / WSTAGES) - 1) & 1, abort);
+                    if (*abort) break;
+                    if constexpr (NV) {
+                        mbar_arrive_expect_tx(&sh.w_full[ws], p.scales_tma ? SS::W_STAGE_BYTES : SS::W_CODE_BYTES);
+                        tma_load_2d(sh.w[ws], &cmap, (kw / KQ) * ROW_BYTES, n0, &sh.w_full[ws]);
+                        if (p.scales_tma)
+                            tma_load_2d(sh.w[ws] + SS::W_CODE_BYTES, &smap, (kw / KQ) * F::SCALE_BYTES, n0,
+                                        &sh.w_full[ws]);
+                    } else {
+                        mbar_arrive_expect_tx(&sh.w_full[ws], SS::W_STAGE_BYTES);
+                        // 2-byte elements: a FAST row of 272 bytes is one 136-element box row
+                        tma_load_2d(sh.w[ws], &cmap, (kw / KQ) * (ROW_BYTES / 2), n0, &sh.w_full[ws]);
+                    }
+                }
+            }
+            drain_ring(sh.w_full, WSTAGES, wit);
+        }
+        __syncwarp();
     } else if (warp == 1) {
         // ------------------------------- MMA issuer -------------------------------
         // A thread that has MMAs queued stalls on any shared-memory access (an
@@ -344,16 +467,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             const uint32_t dtm = tmem + ACC_COL0 + (uint32_t)(b * BN);
             const uint32_t idesc = sh.f16_tile[t % p.tiles_m] ? IDESC_F16 : IDESC;
             for (int kt = 0; kt < KT; kt++, it++) {
-                const int s = it % STAGES;
-                named_barrier_sync(2, 64);   // stage s (and, at kt == 0, accumulator b) is ready
+                const int s = it % STAGES, xs = it % XSTAGES;
+                named_barrier_sync(2, 64);   // stage it (and, at kt == 0, accumulator b) is ready
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t xb = smem_addr(sh.x[s]);
+                    const uint32_t xb = smem_addr(sh.x[xs]);
 #pragma unroll
                     for (int j = 0; j < BK / 16; j++)   // A (16 k = 8 columns) from tensor memory
                         mma_ts(dtm, tmem + (uint32_t)(s * (BK / 2) + 8 * j), sw128_desc(xb + 32 * j), idesc,
                                (kt | j) ? 1u : 0u);
-                    mma_commit(&sh.x_empty[s]);
+                    mma_commit(&sh.x_empty[xs]);
                     mma_commit(&sh.a_empty[s]);
                     if (kt == KT - 1) mma_commit(&sh.acc_full[b]);
                 }
@@ -374,19 +497,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             const int b = lt & 1;
             if (lt >= 2) mbar_wait(&sh.acc_empty[b], ((lt >> 1) - 1) & 1, abort);
             for (int kt = 0; kt < KT; kt++, it++) {
-                const int s = it % STAGES;
-                const uint32_t ph = (it / STAGES) & 1;
                 // on expiry (abort) the stage is garbage, but both warps still meet every barrier
-                mbar_wait(&sh.x_full[s], ph, abort);
-                mbar_wait(&sh.a_full[s], ph, abort);
+                mbar_wait(&sh.x_full[it % XSTAGES], (it / XSTAGES) & 1, abort);
+                mbar_wait(&sh.a_full[it % STAGES], (it / STAGES) & 1, abort);
                 named_barrier_sync(2, 64);
             }
         }
-    } else if (warp < 6) {
+    } else if (warp < kDqWarp0) {
         // -------------------------------- epilogue --------------------------------
         const int q = warp & 3;                 // TMEM lane quadrant of this warp
-        const float g = __ldg(p.gscale);
-        const int fold = bf16_fold(g);
+        const float g = NV ? __ldg(p.gscale) : 1.0f;   // ROCmFP4: no global scale
+        const int fold = NV ? bf16_fold(g) : 0;
         int lt = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, lt++) {
             const int b = lt & 1;
@@ -395,23 +516,27 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             tc_fence_after();
             const int n = n0 + q * 32 + lane;
             const bool f16 = sh.f16_tile[t % p.tiles_m] != 0;
-            for (int c = 0; c < BN / 32; c++) {
-                uint32_t v[32];
-                W4_TMEM_LD32(tmem + ((uint32_t)(q * 32) << 16) + ACC_COL0 + (uint32_t)(b * BN + c * 32), v);
+            for (int c = 0; c < BN / 16; c++) {
+                uint32_t v[16];
+                W4_TMEM_LD16(tmem + ((uint32_t)(q * 32) << 16) + ACC_COL0 + (uint32_t)(b * BN + c * 16), v);
                 asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-                // f16 tiles: token m was scaled by 2^-sigma_m (lane j holds sigma of token c*32+j)
-                const int mlane = m0 + c * 32 + lane;
-                const int sgl = (f16 && mlane < p.M) ? __ldg(p.sigma + mlane) : 0;
+                // f16 tiles: token m was scaled by 2^-sigma_m (lane j < 16 holds sigma of token c*16+j)
+                const int mlane = m0 + c * 16 + (lane & 15);
+                const int el = f16 ? (mlane < p.M ? __ldg(p.sigma + mlane) : 0) : -fold;
+                // g * 2^e as a binary32 factor when that is exact (a normal number or
+                // zero): then acc * factor, rounded once, is the binary64 product of
+                // scale_out rounded once, bit for bit; otherwise scale_out
+                const float gl = epilogue_factor(g, el);
 #pragma unroll
-                for (int j = 0; j < 32; j++) {
-                    const int sg = __shfl_sync(0xFFFFFFFFu, sgl, j);   // every lane takes part
-                    const int m = m0 + c * 32 + j;
-                    if (n < p.N) {
-                        if (m < p.M) {
-                            const float val = scale_out(__uint_as_float(v[j]), g, f16 ? sg : -fold);
-                            if (p.y32) p.y32[(size_t)m * p.N + n] = val;
-                            if (p.y16) p.y16[(size_t)m * p.N + n] = __float2bfloat16_rn(val);
-                        }
+                for (int j = 0; j < 16; j++) {
+                    const int e = __shfl_sync(0xFFFFFFFFu, el, j);   // every lane takes part
+                    const float gj = __shfl_sync(0xFFFFFFFFu, gl, j);
+                    const int m = m0 + c * 16 + j;
+                    if (n < p.N && m < p.M) {
+                        const float acc = __uint_as_float(v[j]);
+                        const float val = isnan(gj) ? scale_out(acc, g, e) : acc * gj;
+                        if (p.y32) p.y32[(size_t)m * p.N + n] = val;
+                        if (p.y16) p.y16[(size_t)m * p.N + n] = __float2bfloat16_rn(val);
                     }
                 }
             }
@@ -421,94 +546,76 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         }
     } else {
         // ------------------------------- dequantise -------------------------------
-        // thread (row r, half h): 32 codes of row r per k-step from the swizzled
-        // codes stage (conflict-free: 8 consecutive rows read 8 distinct 16-byte
-        // chunks), 2 scales from a register ring filled one codes stage ahead.
-        // warp w writes TMEM lanes 32*(w%4) .. +31 (the lanes it may access): row r,
-        // k-half h of each 64-k stage
-        const int r = 32 * (warp & 3) + lane, h = (warp - 6) >> 2;
-        const int fold = bf16_fold(__ldg(p.gscale));
-        const uint32_t a_lane = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-        constexpr int KQ = WK / BK;             // k-steps per codes stage
+        // group gi = (warp - 6) / 4 takes the k-steps i == gi (mod 4) into A stage gi;
+        // thread = weight row r (TMEM lane r) and all 64 k of the k-step.  Rows past
+        // N arrive as zero bytes (TMA fill), which decode to zero weights.
+        const int gi = (warp - kDqWarp0) >> 2;
+        const int r = 32 * (warp & 3) + lane;
+        const int fold = NV ? bf16_fold(__ldg(p.gscale)) : 0;
+        const uint32_t a_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(gi * (BK / 2));
         int it = 0, wit = 0;
-        for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
-            const int n = (t / p.tiles_m) * BM + r;
-            const bool valid = n < p.N;
+        for (int t = blockIdx.x; t < ntiles; t += gridDim.x, it += KT) {
             const bool f16 = sh.f16_tile[t % p.tiles_m] != 0;
-            const uint8_t *srow = p.scales + (size_t)(valid ? n : 0) * (p.K / 16);
-            uint32_t sc[KQ], sn[KQ];
-#pragma unroll
-            for (int q = 0; q < KQ; q++) sc[q] = (valid && q < KT) ? __ldg(reinterpret_cast<const uint32_t *>(srow) + q) : 0u;
+            const int n = (t / p.tiles_m) * BM + r;
+            const uint32_t *srow =
+                NV ? reinterpret_cast<const uint32_t *>(p.scales) + (size_t)(n < p.N ? n : 0) * (p.K / 64) : nullptr;
             for (int kw = 0; kw < KT; kw += KQ, wit++) {
                 const int ws = wit % WSTAGES;
-#pragma unroll
-                for (int q = 0; q < KQ; q++)   // prefetch the next stage's scales
-                    sn[q] = (valid && kw + KQ + q < KT) ? __ldg(reinterpret_cast<const uint32_t *>(srow) + kw + KQ + q) : 0u;
+                // every dequant warp takes every packed stage (and arrives on its
+                // empty barrier), whether or not one of its k-steps lies in it
                 mbar_wait(&sh.w_full[ws], (wit / WSTAGES) & 1, abort);
-                const uint8_t *wrow = sh.w[ws] + r * 128;
-                // two k-steps per round: one proxy fence and one pair of arrivals per two A
-                // stages halves the per-stage synchronisation latency of this chain
-#pragma unroll
-                for (int q = 0; q < KQ; q += 2) {
-                    const int nq = min(2, KT - (kw + q));
-                    if (nq <= 0) break;
-                    // both A stages free first, then both loads, both decodes and both
-                    // stores, so that the two k-steps overlap in this warp
-#pragma unroll
-                    for (int j = 0; j < 2; j++)
-                        if (j < nq && it + j >= STAGES)
-                            mbar_wait(&sh.a_empty[(it + j) % STAGES], (((it + j) / STAGES) - 1) & 1, abort);
-                    tc_fence_after();
-                    uint4 cw[2];
-#pragma unroll
-                    for (int j = 0; j < 2; j++)
-                        cw[j] = ld_shared_v4(smem_addr(wrow + ((((q + j) * 2 + h) ^ (r & 7)) * 16)));
-                    uint32_t av[2][16];
-#pragma unroll
-                    for (int j = 0; j < 2; j++) {
-                        const uint32_t sw = sc[q + j] >> (16 * h);
-                        const uint32_t cws[4] = {cw[j].x, cw[j].y, cw[j].z, cw[j].w};
+                const uint32_t wst = smem_addr(sh.w[ws]);
+                const uint32_t wrow = wst + (uint32_t)(r * ROW_BYTES);
+#pragma unroll 1
+                for (int q = (gi - (it + kw)) & 3; q < KQ && kw + q < KT; q += 4) {
+                    const int i = it + kw + q;   // this group's k-step: i % 4 == gi
+                    uint32_t av[32];
+                    if constexpr (NV) {
+                        // 64 k of row r: chunks 2q, 2q+1 of the swizzled 128-byte row;
+                        // 4 block scales at byte 4q of the row's 16 scale bytes (or the
+                        // row's scale word kw + q in global memory)
+                        const uint4 c0 = ld_shared_v4(wrow + (uint32_t)(((2 * q) ^ (r & 7)) * 16));
+                        const uint4 c1 = ld_shared_v4(wrow + (uint32_t)(((2 * q + 1) ^ (r & 7)) * 16));
+                        const uint32_t sw =
+                            p.scales_tma ? ld_shared_u32(wst + SS::W_CODE_BYTES + (uint32_t)(r * F::SCALE_BYTES + 4 * q))
+                                         : (n < p.N ? __ldg(srow + kw + q) : 0u);
+                        const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
                         if (f16) {
-                            const uint32_t s01 = e4m3x2_to_f16x2(sw & 0xFFFFu);
-                            const uint32_t s0 = __byte_perm(s01, 0, 0x1010), s1 = __byte_perm(s01, 0, 0x3232);
+                            const uint32_t s01 = e4m3x2_to_f16x2(sw & 0xFFFFu), s23 = e4m3x2_to_f16x2(sw >> 16);
+                            const uint32_t sd[4] = {__byte_perm(s01, 0, 0x1010), __byte_perm(s01, 0, 0x3232),
+                                                    __byte_perm(s23, 0, 0x1010), __byte_perm(s23, 0, 0x3232)};
 #pragma unroll
-                            for (int cc = 0; cc < 4; cc++) {
-                                const uint4 o = valid ? dequant8_f16(cws[cc], cc < 2 ? s0 : s1) : make_uint4(0, 0, 0, 0);
-                                av[j][4 * cc] = o.x, av[j][4 * cc + 1] = o.y, av[j][4 * cc + 2] = o.z, av[j][4 * cc + 3] = o.w;
-                            }
+                            for (int c = 0; c < 8; c++) dequant8_f16(cw[c], sd[c >> 1], av + 4 * c);
                         } else {
-                            const float s0 = mul_pow2(e4m3_to_f32(sw & 0xFFu), fold),
-                                        s1 = mul_pow2(e4m3_to_f32((sw >> 8) & 0xFFu), fold);
 #pragma unroll
-                            for (int cc = 0; cc < 4; cc++) {
-                                const uint4 o = valid ? dequant8(cws[cc], cc < 2 ? s0 : s1) : make_uint4(0, 0, 0, 0);
-                                av[j][4 * cc] = o.x, av[j][4 * cc + 1] = o.y, av[j][4 * cc + 2] = o.z, av[j][4 * cc + 3] = o.w;
-                            }
+                            for (int c = 0; c < 8; c++)
+                                dequant8_bf16(cw[c], mul_pow2(e4m3_to_f32((sw >> (8 * (c >> 1))) & 0xFFu), fold),
+                                              av + 4 * c);
                         }
+                    } else {
+                        // blocks 2q, 2q+1 of row r
+                        dequant_rocm_block<FMT == W4_FMT_ROCMFP4_DUAL>(wrow + (uint32_t)(2 * q * BB), f16, av);
+                        dequant_rocm_block<FMT == W4_FMT_ROCMFP4_DUAL>(wrow + (uint32_t)((2 * q + 1) * BB), f16,
+                                                                        av + 16);
                     }
-                    // 32 k of row r: columns 16h .. 16h+15 of A stage s
-#pragma unroll
-                    for (int j = 0; j < 2; j++)
-                        if (j < nq) tmem_st16(a_lane + (uint32_t)(((it + j) % STAGES) * (BK / 2) + 16 * h), av[j]);
-                    // the stores complete, then one arrival per warp and stage
+                    // the stage is free once the MMAs of its previous use have completed
+                    if (i >= STAGES) mbar_wait(&sh.a_empty[gi], ((i / STAGES) - 1) & 1, abort);
+                    tc_fence_after();
+                    tmem_st32(a_addr, av);
                     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0)
-                        for (int j = 0; j < nq; j++) mbar_arrive(&sh.a_full[(it + j) % STAGES]);
-                    it += nq;
+                    if (lane == 0) mbar_arrive(&sh.a_full[gi]);
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sh.w_empty[ws]);
-#pragma unroll
-                for (int q = 0; q < KQ; q++) sc[q] = sn[q];
             }
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 1) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
     }
@@ -525,14 +632,21 @@ inline size_t gemm_workspace_bytes(const w4_weights *w, int M) {
     return (((size_t)M * w->K * 2 + 15) & ~(size_t)15) + (((size_t)M * 8 + 15) & ~(size_t)15);
 }
 
-inline size_t gemm_smem_bytes() { return sizeof(gemm::SharedStorage) + 1024; }
+template <int FMT>
+inline size_t gemm_smem_bytes() { return sizeof(gemm::SharedStorage<FMT>) + 1024; }
 
-inline w4_status gemm_launch(const w4_weights *w, const void *x, int M, float *y32, void *y16, void *ws,
-                             size_t ws_bytes, cudaStream_t st) {
+template <int FMT>
+inline w4_status gemm_launch_fmt(const w4_weights *w, const void *x, int M, float *y32, void *y16, void *ws,
+                                 size_t ws_bytes, cudaStream_t st) {
     using namespace gemm;
-    if (w->fmt != W4_FMT_NVFP4) return W4_ERR_UNSUPPORTED;
+    using F = WFormat<FMT>;
+    static_assert(sizeof(SharedStorage<FMT>) + 1024 <= 227 * 1024, "shared memory of the GEMM");
+    static_assert(SharedStorage<FMT>::W_STAGE_BYTES % 1024 == 0 && (XSTAGES * X_STAGE_BYTES) % 1024 == 0,
+                  "stages on 1024-byte boundaries");
     const int K = w->K, N = w->N;
-    if (K % BK) return W4_ERR_UNSUPPORTED;
+    // NVFP4: 64-k steps (a last partial packed stage reads zeros past K);
+    // ROCmFP4: whole packed stages, whose row pieces are 16-byte multiples
+    if (K % (FMT == W4_FMT_NVFP4 ? BK : F::WK)) return W4_ERR_UNSUPPORTED;
     PFN_encodeTiled enc = get_encode_tiled();
     if (!enc) return W4_ERR_CUDA;
     CUtensorMap map;
@@ -556,22 +670,48 @@ inline w4_status gemm_launch(const w4_weights *w, const void *x, int M, float *y
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return W4_ERR_CUDA;
-    CUtensorMap cmap;
-    const cuuint64_t cdims[2] = {(cuuint64_t)K / 2, (cuuint64_t)N};
-    const cuuint64_t cstrides[1] = {(cuuint64_t)K / 2};
-    const cuuint32_t cbox[2] = {WK / 2, BM};
-    if (enc(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(w->codes), cdims, cstrides, cbox, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return W4_ERR_CUDA;
+    // packed weights: NVFP4 codes [N][K/2] bytes with the 128-byte swizzle and
+    // scales [N][K/16] bytes; ROCmFP4 blocks [N][K/32 * 18|17] bytes as 2-byte
+    // elements (the FAST box row of 272 bytes exceeds 256 one-byte elements)
+    CUtensorMap cmap, smap;
+    // the scales map needs 16-byte rows (K % 256 == 0); otherwise the dequant
+    // warps read the scale words directly
+    const bool scales_tma = FMT == W4_FMT_NVFP4 && K % 256 == 0;
+    if (FMT == W4_FMT_NVFP4) {
+        const cuuint64_t cdims[2] = {(cuuint64_t)K / 2, (cuuint64_t)N};
+        const cuuint64_t cstr[1] = {(cuuint64_t)K / 2};
+        const cuuint32_t cbox[2] = {(cuuint32_t)F::ROW_BYTES, BM};
+        const cuuint64_t sdims[2] = {(cuuint64_t)K / 16, (cuuint64_t)N};
+        const cuuint64_t sstr[1] = {(cuuint64_t)K / 16};
+        const cuuint32_t sbox[2] = {(cuuint32_t)F::SCALE_BYTES, BM};
+        if (enc(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(w->codes), cdims, cstr, cbox, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+            (scales_tma &&
+             enc(&smap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(w->scales), sdims, sstr, sbox, estr,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS))
+            return W4_ERR_CUDA;
+        if (!scales_tma) smap = cmap;   // not read
+    } else {
+        const cuuint64_t row_bytes = (cuuint64_t)(K / F::WK) * F::ROW_BYTES;
+        const cuuint64_t cdims[2] = {row_bytes / 2, (cuuint64_t)N};
+        const cuuint64_t cstr[1] = {row_bytes};
+        const cuuint32_t cbox[2] = {(cuuint32_t)F::ROW_BYTES / 2, BM};
+        if (enc(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint8_t *>(w->codes), cdims, cstr, cbox, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return W4_ERR_CUDA;
+        smap = cmap;   // not read
+    }
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev))
         return W4_ERR_CUDA;
-    const size_t smem = gemm_smem_bytes();
-    if (!set_smem_limit(reinterpret_cast<const void *>(gemm_kernel), smem)) return W4_ERR_CUDA;
+    const size_t smem = gemm_smem_bytes<FMT>();
+    if (!set_smem_limit(reinterpret_cast<const void *>(gemm_kernel<FMT>), smem)) return W4_ERR_CUDA;
     Params p;
-    p.codes = w->codes;
     p.scales = w->scales;
+    p.scales_tma = scales_tma ? 1 : 0;
     p.gscale = w->global_scale;
     p.y32 = y32;
     p.y16 = reinterpret_cast<__nv_bfloat16 *>(y16);
@@ -582,10 +722,22 @@ inline w4_status gemm_launch(const w4_weights *w, const void *x, int M, float *y
     p.tiles_n = (N + BM - 1) / BM;
     p.bad = bad;
     p.sigma = sigma;
-    if (f16) x_to_f16_kernel<<<M, 256, 0, st>>>(reinterpret_cast<const uint16_t *>(x), xh, sigma, bad, K);
+    if (f16)
+        x_to_f16_kernel<<<(M + 7) / 8, 256, 0, st>>>(reinterpret_cast<const uint16_t *>(x), xh, sigma, bad, M, K);
     const int ntiles = p.tiles_m * p.tiles_n;
-    gemm_kernel<<<std::min(ntiles, sms), kThreads, smem, st>>>(map, map16, cmap, p);
+    const int grid = std::max(1, std::min(ntiles, sms));   // persistent, one CTA per SM
+    gemm_kernel<FMT><<<grid, kThreads, smem, st>>>(map, map16, cmap, smap, p);
     return cudaGetLastError() == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
+inline w4_status gemm_launch(const w4_weights *w, const void *x, int M, float *y32, void *y16, void *ws,
+                             size_t ws_bytes, cudaStream_t st) {
+    switch (w->fmt) {
+    case W4_FMT_NVFP4: return gemm_launch_fmt<W4_FMT_NVFP4>(w, x, M, y32, y16, ws, ws_bytes, st);
+    case W4_FMT_ROCMFP4_DUAL: return gemm_launch_fmt<W4_FMT_ROCMFP4_DUAL>(w, x, M, y32, y16, ws, ws_bytes, st);
+    case W4_FMT_ROCMFP4_FAST: return gemm_launch_fmt<W4_FMT_ROCMFP4_FAST>(w, x, M, y32, y16, ws, ws_bytes, st);
+    }
+    return W4_ERR_UNSUPPORTED;
 }
 
 }  // namespace w4

@@ -18,20 +18,23 @@
 // adds s * D with one FFMA each.  No HMUL2, no scale duplication, and every
 // MMA column is used.
 //
-// x is converted to f16 once per CTA with a power-of-two exponent per 16-k
-// block (sigma_b from the block's largest |x|, so its largest |x'| lies in
-// [2^14, 2^15)).  x' = x * 2^-sigma_b is exact in f16 whenever every nonzero
-// |x'| >= 2^-17 (8 significant bits above f16's 2^-24 quantum).  Each warp
-// converts exactly the blocks it later multiplies, so no CTA barrier is needed;
-// its partial sums are kept relative to 2^sigma_ref (the warp's largest
-// sigma_b) and the per-block factor 2^(sigma_b - sigma_ref) is folded into the
-// scale.  A warp with a block it cannot convert exactly (range above 2^31
-// inside a block, factors below binary32's normal range, Inf/NaN) computes its
-// share in binary32 on the CUDA cores from the bf16 x in global memory.
+// x is converted to f16 once per CTA, as x * 2^-sigma with one power of two
+// for the whole slice (its largest |x'| in [2^14, 2^15)), exact whenever every
+// nonzero |x'| >= 2^-17; all consumer warps convert together and permute each
+// 128-k super-chunk to the MMA operand order.  A CTA whose x does not convert
+// exactly (range above 2^31, Inf/NaN) computes in binary32 on the CUDA cores
+// from the bf16 x in global memory.  The output is acc * g * 2^sigma, formed
+// in binary64 (scale_out).
 //
-// Shared memory: x' [kc + 32] f16 (permuted per super-chunk as in the general
-// kernel), the per-block factors [kc/16] binary32, the NS weight stages, the
-// per-warp partial sums, mbarriers and flags.
+// Codes stages (16 rows x KP k) arrive as one 3-D TMA box of 128-byte lines
+// with the 128-byte swizzle; each warp quarter reads two rows whose lines differ
+// by 4 mod 8 (a fixed remap of MMA rows to physical rows), so the 16-byte code
+// loads are free of bank conflicts.  A short tail tile (fewer than 4 rows)
+// comes as row copies in the dense layout.  The super-chunks of a stage are
+// shared out among the 8 consumer warps with an offset that rotates by tile.
+//
+// Shared memory: x' [kc + 32] f16, the NS weight stages (1024-byte aligned),
+// the per-warp partial sums, mbarriers and flags.
 #pragma once
 
 #include "gemv_tc.cuh"
@@ -40,39 +43,16 @@ namespace w4 {
 
 // Offsets (bytes) of the M = 1 kernel's shared-memory regions.
 struct M1Layout {
-    size_t pw, stages, red, bars, total;
+    size_t stages, red, bars, total;
 };
 
 __host__ __device__ __forceinline__ M1Layout m1_layout(int xstride, int kc, int NS, int tile_bytes, int red_tiles) {
     M1Layout L;
-    L.pw = ((size_t)xstride * 2 + 127) & ~(size_t)127;
-    L.stages = (L.pw + (size_t)(kc / 16) * 4 + 127) & ~(size_t)127;
-    L.red = L.stages + (size_t)NS * tile_bytes;
+    L.stages = ((size_t)xstride * 2 + 127) & ~(size_t)127;
+    L.red = L.stages + 1024 + (size_t)NS * tile_bytes;   // + room to align the stages to 1024 bytes
     L.bars = L.red + (size_t)red_tiles * kTcParts * kTcRows * 4;
-    L.total = L.bars + (size_t)(2 * NS + 1) * 8 + 16;
+    L.total = L.bars + (size_t)(2 * NS + 1) * 8 + 4 * (2 + kTcWarps);   // barriers, flags
     return L;
-}
-
-constexpr int kNoSigma = -100000;   // block of zeros (or an unused lane)
-
-// Largest |bf16| bit pattern of 16 values.
-__device__ __forceinline__ uint32_t absmax_bits16(uint4 v0, uint4 v1) {
-    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    uint32_t m = 0;
-#pragma unroll
-    for (int i = 0; i < 8; i++) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
-    return max(m & 0xFFFFu, m >> 16);
-}
-
-// Two bf16 (one word) -> f16x2 of x * 2^-sigma; `bad` when a nonzero result is
-// below 2^-17 (may be inexact in f16) -- results above f16's range cannot occur
-// for x of the block that sigma was taken from.
-__device__ __forceinline__ uint32_t bf16x2_to_f16x2_scaled(uint32_t w, int neg_sigma, bool &bad) {
-    const float x0 = mul_pow2(bf16_lo(w), neg_sigma), x1 = mul_pow2(bf16_hi(w), neg_sigma);
-    const float tiny = 7.62939453125e-06f;   // 2^-17
-    bad |= (x0 != 0.0f && fabsf(x0) < tiny) | (x1 != 0.0f && fabsf(x1) < tiny);
-    const __half2 h = __floats2half2_rn(x0, x1);
-    return *reinterpret_cast<const uint32_t *>(&h);
 }
 
 // 16 code bytes of one row (32 k) -> 16 f16x2 (h[i] = elements 2i, 2i+1), exact.
@@ -100,8 +80,8 @@ __device__ __forceinline__ void m1_body(const CUtensorMap &cmap, const CUtensorM
     const M1Layout L = m1_layout(a.xstride, kc, NS, a.tile_bytes, a.red_tiles);
 
     uint16_t *xs = reinterpret_cast<uint16_t *>(smem);
-    float *pw = reinterpret_cast<float *>(smem + L.pw);   // per-block factor 2^(120 + sigma_b - sigma_ref)
-    uint8_t *stages = smem + L.stages;
+    // stages on 1024 bytes (the codes box's swizzle atom), whatever the base alignment
+    uint8_t *stages = smem + ((smem_addr(smem) + L.stages + 1023) & ~1023u) - smem_addr(smem);
     float *red = reinterpret_cast<float *>(smem + L.red);  // [red_tiles][kTcParts][16]
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bars);
     uint64_t *empty = full + NS;
@@ -122,7 +102,8 @@ __device__ __forceinline__ void m1_body(const CUtensorMap &cmap, const CUtensorM
     const int nstages = ntiles * npieces;
 
     if (threadIdx.x == 0) {
-        flags[0] = 0;
+        flags[0] = 0;   // abort
+        flags[1] = 0;   // x not exact in f16
         for (int i = 0; i < NS; i++) {
             mbar_init(full + i, 1);
             mbar_init(empty + i, kTcWarps);
@@ -144,68 +125,19 @@ __device__ __forceinline__ void m1_body(const CUtensorMap &cmap, const CUtensorM
     pdl_wait_prior_grid();   // y may be read by the previous kernel
     mbar_wait(xfull, 0, abort);
 
-    // Warp w multiplies super-chunks [sb, se) of every piece (the same share in
-    // every tile), i.e. at most 32 blocks per piece: lane l takes block l.
-    // Pass 1: sigma_b per block, kept in pw[] as an int until sigma_ref is known.
-    bool bad = false;
-    int sref = kNoSigma;
-    for (int p = 0; p < npieces; p++) {
-        const int kb = p * KP, SC = min(KP, kcs - kb) / 128;
-        const int sb = warp * SC / kTcWarps, se = (warp + 1) * SC / kTcWarps;
-        if (lane < 8 * (se - sb)) {
-            const int blk = kb / 16 + 8 * sb + lane;
-            const uint4 *src = reinterpret_cast<const uint4 *>(xs + (size_t)blk * 16);
-            const uint32_t m = absmax_bits16(src[0], src[1]);
-            int sg = kNoSigma;
-            if (m != 0) {
-                bad |= m >= 0x7F80u;                        // Inf / NaN
-                sg = max((int)(m >> 7), 1) - 127 - 14;      // largest |x| * 2^-sg in [2^14, 2^15)
-            }
-            reinterpret_cast<int *>(pw)[blk] = sg;
-            sref = max(sref, sg);
-        }
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) sref = max(sref, __shfl_xor_sync(0xFFFFFFFFu, sref, o));
-    if (sref == kNoSigma) sref = 0;   // all of this warp's x are zero
-    // Pass 2: convert in place to f16, permuting each super-chunk: the 8 values
-    // k = 32t + 8j .. +7 go to offset 32j + 8t (block b = 2t + j/2).
-    for (int p = 0; p < npieces; p++) {
-        const int kb = p * KP, SC = min(KP, kcs - kb) / 128;
-        const int sb = warp * SC / kTcWarps, se = (warp + 1) * SC / kTcWarps;
-        const bool mine = lane < 8 * (se - sb);
-        const int blk = kb / 16 + 8 * sb + lane;
-        uint4 o0 = make_uint4(0, 0, 0, 0), o1 = o0;
-        if (mine) {
-            const int sg = reinterpret_cast<const int *>(pw)[blk];
-            const uint4 *src = reinterpret_cast<const uint4 *>(xs + (size_t)blk * 16);
-            const uint4 v0 = src[0], v1 = src[1];
-            const int ns = sg == kNoSigma ? 0 : -sg;
-            o0 = make_uint4(bf16x2_to_f16x2_scaled(v0.x, ns, bad), bf16x2_to_f16x2_scaled(v0.y, ns, bad),
-                            bf16x2_to_f16x2_scaled(v0.z, ns, bad), bf16x2_to_f16x2_scaled(v0.w, ns, bad));
-            o1 = make_uint4(bf16x2_to_f16x2_scaled(v1.x, ns, bad), bf16x2_to_f16x2_scaled(v1.y, ns, bad),
-                            bf16x2_to_f16x2_scaled(v1.z, ns, bad), bf16x2_to_f16x2_scaled(v1.w, ns, bad));
-            int fe = 120;   // a zero block: D = 0, any finite factor
-            if (sg != kNoSigma) {
-                fe = 120 + sg - sref;
-                bad |= fe < 3;   // s * 2^(fe - 120) must stay a normal binary32
-            }
-            pw[blk] = __int_as_float((127 + max(fe, 3)) << 23);
-        }
-        __syncwarp();
-        if (mine) {
-            const int bi = blk & 7;
-            uint16_t *dst = xs + (size_t)(blk >> 3) * 128 + 64 * (bi & 1) + 8 * (bi >> 1);
-            *reinterpret_cast<uint4 *>(dst) = o0;
-            *reinterpret_cast<uint4 *>(dst + 32) = o1;
-        }
-        __syncwarp();
-    }
-    const bool fast = !__any_sync(0xFFFFFFFFu, bad);
-    // binary32 path: partial sums in units of x * 2^fold (the largest block of
-    // this warp has |x| in [2^(sref+14), 2^(sref+15)))
-    const int fold = fast ? 0 : fallback_fold(gs, sref + 14 >= 100);
-    if (!fast) sref = -fold;
+    // x -> f16 with one power of two for the whole slice, permuted per 128-k
+    // super-chunk (convert_x_f16, all consumer warps); a CTA whose x does not
+    // convert exactly computes in binary32 on the CUDA cores from the BF16 x in
+    // global memory.
+    int sigma;
+    uint32_t mx;
+    convert_x_f16<false>(xs, a.xstride, 1, kcs, warp, lane, flags, sigma, mx);
+    named_barrier_sync(1, kTcWarps * 32);
+    const bool fast = flags[1] == 0;
+    // binary32 path: partial sums in units of x * 2^fold
+    const int fold = fast ? 0 : fallback_fold(gs, mx >= ((127u + 100u) << 7));   // largest |x| >= 2^100
+    const int sref = fast ? sigma : -fold;
+    const float p120 = __int_as_float((127 + 120) << 23);   // e4m3_*_scaled(s) * 2^120 = s
 
     // MMA operands.  Lane (g, t) holds rows g, g+8 of the codes of k = 32t .. 32t+31
     // (blocks 2t, 2t+1) and B column g.  Column g is block g: it is nonzero only for
@@ -219,9 +151,15 @@ __device__ __forceinline__ void m1_body(const CUtensorMap &cmap, const CUtensorM
     // active lanes of each load on distinct banks
     const int xoffA = 32 * (odd ? 3 : 0) + 8 * t4, xoffB = 32 * (odd ? 2 : 1) + 8 * t4;
 
+    const int lines = KP / 256;                    // 128-byte lines per row of a swizzled stage
+    const int rdist = swz_row_distance(lines);
     int st_idx = 0;
     for (int tile = 0; tile < ntiles; tile++) {
-        float accA = 0.0f, accB = 0.0f;   // rows g, g+8 (fast) / row lane/2 (binary32)
+        float accA = 0.0f, accB = 0.0f;   // rows pr0, pr0+8 (fast) / row lane/2 (binary32)
+        // this tile's stages: swizzled box, or (a short tail) row copies in the dense layout
+        const int trows = (int)min((long long)kTcRows, r1 - (r0 + (long long)tile * kTcRows));
+        const bool dense = !a.swz || trows < a.box_min_rows;
+        const int pr0 = dense ? g : swz_phys_row(g, rdist);   // physical row of MMA row g
         for (int piece = 0; piece < npieces; piece++, st_idx++) {
             const int st = st_idx % NS;
             // on expiry the tile is garbage, but the warp still reaches every barrier
@@ -230,21 +168,28 @@ __device__ __forceinline__ void m1_body(const CUtensorMap &cmap, const CUtensorM
             const int kbase = piece * KP;
             const int kps = min(KP, kcs - kbase);
             const int SC = kps / 128;
-            const int sb = warp * SC / kTcWarps, se = (warp + 1) * SC / kTcWarps;
+            // super-chunks [sb, se) of this stage; the shares rotate by tile so that a
+            // stage whose count does not divide by 8 does not load one warp alone
+            const int wr = (warp + tile) % kTcWarps;
+            const int sb = wr * SC / kTcWarps, se = (wr + 1) * SC / kTcWarps;
             if (fast) {
-                const uint8_t *c0p = tp + g * CS + 16 * t4;
+                const uint8_t *c0p = tp + pr0 * CS + 16 * t4;
                 const uint8_t *c1p = c0p + 8 * CS;
-                const uint8_t *s0p = tp + kTcRows * CS + g * SS + 2 * t4;
+                const uint8_t *s0p = tp + kTcRows * CS + pr0 * SS + 2 * t4;
                 const uint8_t *s1p = s0p + 8 * SS;
                 const uint16_t *xp = xs + kbase;
-                const float *pp = pw + kbase / 16 + 2 * t4;
 #pragma unroll 2
                 for (int s = sb; s < se; s++) {
-                    const uint4 c0 = *reinterpret_cast<const uint4 *>(c0p + s * 64);
-                    const uint4 c1 = *reinterpret_cast<const uint4 *>(c1p + s * 64);
+                    uint4 c0, c1;
+                    if (dense) {
+                        c0 = *reinterpret_cast<const uint4 *>(c0p + s * 64);
+                        c1 = *reinterpret_cast<const uint4 *>(c1p + s * 64);
+                    } else {
+                        c0 = *reinterpret_cast<const uint4 *>(tp + swz_chunk(pr0, s, t4, lines));
+                        c1 = *reinterpret_cast<const uint4 *>(tp + swz_chunk(pr0 + 8, s, t4, lines));
+                    }
                     const uint32_t sc0 = *reinterpret_cast<const uint16_t *>(s0p + s * 8);
                     const uint32_t sc1 = *reinterpret_cast<const uint16_t *>(s1p + s * 8);
-                    const float2 pv = *reinterpret_cast<const float2 *>(pp + s * 8);
                     uint4 xa = make_uint4(0, 0, 0, 0), xb = xa;
                     if (xact) {
                         xa = *reinterpret_cast<const uint4 *>(xp + s * 128 + xoffA);
@@ -256,20 +201,23 @@ __device__ __forceinline__ void m1_body(const CUtensorMap &cmap, const CUtensorM
                     uint32_t h0[16], h1[16];
                     decode_codes32(c0, h0);
                     decode_codes32(c1, h1);
+                    // four independent chains of two MMAs (the MMA latency, not
+                    // its rate, is what a chain of eight would cost)
                     float d0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, d1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                    float e0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, e1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
                     mma_f16_16816(d0, h0[0], h1[0], h0[1], h1[1], b0.x, b0.y);
-                    mma_f16_16816(d0, h0[2], h1[2], h0[3], h1[3], b0.z, b0.w);
-                    mma_f16_16816(d0, h0[4], h1[4], h0[5], h1[5], b1.x, b1.y);
-                    mma_f16_16816(d0, h0[6], h1[6], h0[7], h1[7], b1.z, b1.w);
+                    mma_f16_16816(e0, h0[2], h1[2], h0[3], h1[3], b0.z, b0.w);
                     mma_f16_16816(d1, h0[8], h1[8], h0[9], h1[9], b2.x, b2.y);
-                    mma_f16_16816(d1, h0[10], h1[10], h0[11], h1[11], b2.z, b2.w);
+                    mma_f16_16816(e1, h0[10], h1[10], h0[11], h1[11], b2.z, b2.w);
+                    mma_f16_16816(d0, h0[4], h1[4], h0[5], h1[5], b1.x, b1.y);
+                    mma_f16_16816(e0, h0[6], h1[6], h0[7], h1[7], b1.z, b1.w);
                     mma_f16_16816(d1, h0[12], h1[12], h0[13], h1[13], b3.x, b3.y);
-                    mma_f16_16816(d1, h0[14], h1[14], h0[15], h1[15], b3.z, b3.w);
-                    // d0 holds block 2t in column 2t, d1 block 2t+1 in column 2t+1
-                    accA = __fmaf_rn(e4m3_lo_scaled(sc0) * pv.x, d0[0], accA);
-                    accA = __fmaf_rn(e4m3_hi_scaled(sc0) * pv.y, d1[1], accA);
-                    accB = __fmaf_rn(e4m3_lo_scaled(sc1) * pv.x, d0[2], accB);
-                    accB = __fmaf_rn(e4m3_hi_scaled(sc1) * pv.y, d1[3], accB);
+                    mma_f16_16816(e1, h0[14], h1[14], h0[15], h1[15], b3.z, b3.w);
+                    // d0 + e0 holds block 2t in column 2t, d1 + e1 block 2t+1 in column 2t+1
+                    accA = __fmaf_rn(e4m3_lo_scaled(sc0) * p120, d0[0] + e0[0], accA);
+                    accA = __fmaf_rn(e4m3_hi_scaled(sc0) * p120, d1[1] + e1[1], accA);
+                    accB = __fmaf_rn(e4m3_lo_scaled(sc1) * p120, d0[2] + e0[2], accB);
+                    accB = __fmaf_rn(e4m3_hi_scaled(sc1) * p120, d1[3] + e1[3], accB);
                 }
             } else {
                 // binary32 on the CUDA cores: lane l takes row l/2, 64 k of each super-chunk
@@ -280,7 +228,9 @@ __device__ __forceinline__ void m1_body(const CUtensorMap &cmap, const CUtensorM
                     const uint4 *xg = reinterpret_cast<const uint4 *>(a.x + k0 + kbase + s * 128 + 64 * half);
 #pragma unroll
                     for (int q = 0; q < 4; q++) {
-                        const uint2 c = *reinterpret_cast<const uint2 *>(cp + 8 * q);
+                        const uint8_t *cq = dense ? cp + 8 * q
+                                                  : tp + swz_chunk(row, s, 2 * half + (q >> 1), lines) + 8 * (q & 1);
+                        const uint2 c = *reinterpret_cast<const uint2 *>(cq);
                         float2 w[8], xv[8];
                         decode_nvfp4(c, w);
                         scale_pairs(w, fold);
@@ -305,8 +255,8 @@ __device__ __forceinline__ void m1_body(const CUtensorMap &cmap, const CUtensorM
             accB += __shfl_xor_sync(0xFFFFFFFFu, accB, 1);
             accB += __shfl_xor_sync(0xFFFFFFFFu, accB, 2);
             if (t4 == 0) {
-                rb[warp * kTcRows + g] = scale_out(accA, gs, sref);
-                rb[warp * kTcRows + g + 8] = scale_out(accB, gs, sref);
+                rb[warp * kTcRows + pr0] = scale_out(accA, gs, sref);
+                rb[warp * kTcRows + pr0 + 8] = scale_out(accB, gs, sref);
             }
         } else {
             accA += __shfl_xor_sync(0xFFFFFFFFu, accA, 1);

@@ -53,110 +53,13 @@ inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s
 // ------------------------------------------------------------------ GEMV ----
 
 constexpr size_t kXBudget = 64 * 1024;      // shared bytes for the x slice
-constexpr int kTileTarget = 24 * 1024;      // bytes per pipeline stage
 
-inline int gemv_rows_per_task(int M) { return M <= 2 ? 4 : (M <= 4 ? 2 : 1); }
-
-// Alignment unit of K for the bulk-copy path: row pieces must start on 16 bytes.
+// Alignment unit of K for the GEMV stages: row pieces must start on 16 bytes.
 inline int k_unit(int fmt) { return fmt == W4_FMT_ROCMFP4_FAST ? 512 : 256; }
-
-struct GemvPlan {
-    int S = 1, kc = 0, TR = 0, P = 0, NS = 0, tile_bytes = 0, grid = 0;
-    size_t smem = 0;
-    size_t ws_bytes = 0;
-};
-
-int piece_bytes(int fmt, int kc) {
-    if (fmt == W4_FMT_NVFP4) return kc / 2 + kc / 16;
-    return (kc / 32) * (fmt == W4_FMT_ROCMFP4_DUAL ? 18 : 17);
-}
-
-w4_status plan_gemv(int fmt, int K, int N, int M, bool pdl, GemvPlan &p) {
-    DeviceInfo d;
-    if (device_info(d) != W4_OK) return W4_ERR_CUDA;
-    const int unit = k_unit(fmt);
-    // split-K slices so that x[M][kc] fits the x budget
-    const int units = K / unit;
-    int per = (int)std::max<size_t>(1, kXBudget / ((size_t)2 * M * unit));
-    per = std::min(per, units);
-    p.kc = per * unit;
-    p.S = (units + per - 1) / per;
-    const int R = gemv_rows_per_task(M);
-    const int rowB = piece_bytes(fmt, p.kc);
-    int TR = R;
-    while (TR * 2 <= 8 * R && TR * 2 * rowB <= kTileTarget) TR *= 2;
-    p.TR = TR;
-    p.P = 8 * R / TR;
-    p.tile_bytes = (TR * rowB + 127) & ~127;
-    const size_t xs = ((size_t)M * p.kc * 2 + 127) & ~(size_t)127;
-    const size_t red = (size_t)2 * TR * p.P * M * 4 + 16;  // + abort flag
-    const size_t budget = std::min<size_t>(pdl ? 110 * 1024 : 200 * 1024, (size_t)d.smem_optin);
-    int NS = 8;
-    while (NS > 2 && xs + (size_t)NS * p.tile_bytes + red + 16 * NS > budget) NS--;
-    p.NS = NS;
-    p.smem = xs + (size_t)NS * p.tile_bytes + red + 16 * NS;
-    if (p.smem > (size_t)d.smem_optin) return W4_ERR_UNSUPPORTED;
-    p.grid = std::min(d.sms, N);
-    p.ws_bytes = p.S > 1 ? (size_t)p.S * M * N * sizeof(float) : 0;
-    return W4_OK;
-}
-
-template <int FMT, int M>
-w4_status launch_gemv_m(const w4_weights *w, const void *x, float *y, void *ws, const GemvPlan &p, bool pdl,
-                        cudaStream_t st) {
-    constexpr int R = M <= 2 ? 4 : (M <= 4 ? 2 : 1);
-    auto kern = gemv_kernel<FMT, M, R>;
-    if (!set_smem_limit(reinterpret_cast<const void *>(kern), p.smem)) return W4_ERR_CUDA;
-    GemvArgs a;
-    a.codes = w->codes;
-    a.scales = w->scales;
-    a.gscale = w->global_scale;
-    a.x = reinterpret_cast<const uint16_t *>(x);
-    a.y = y;
-    a.partial = reinterpret_cast<float *>(ws);
-    a.K = w->K;
-    a.N = w->N;
-    a.kc = p.kc;
-    a.TR = p.TR;
-    a.P = p.P;
-    a.NS = p.NS;
-    a.tile_bytes = p.tile_bytes;
-
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.grid, p.S, 1);
-    cfg.blockDim = dim3(kGemvThreads, 1, 1);
-    cfg.dynamicSmemBytes = p.smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
-    if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return W4_ERR_CUDA;
-    if (p.S > 1) {
-        const int MN = M * w->N;
-        gemv_finalize_kernel<<<std::min((MN + 255) / 256, 1024), 256, 0, st>>>(
-            a.partial, p.S, MN, FMT == W4_FMT_NVFP4 ? w->global_scale : nullptr, y);
-    }
-    return launch_status();
-}
-
-template <int FMT>
-w4_status launch_gemv_fmt(const w4_weights *w, const void *x, int M, float *y, void *ws, const GemvPlan &p,
-                          bool pdl, cudaStream_t st) {
-    switch (M) {
-#define W4_CASE(m) \
-    case m: return launch_gemv_m<FMT, m>(w, x, y, ws, p, pdl, st);
-        W4_CASE(1) W4_CASE(2) W4_CASE(3) W4_CASE(4) W4_CASE(5) W4_CASE(6) W4_CASE(7) W4_CASE(8)
-        W4_CASE(9) W4_CASE(10) W4_CASE(11) W4_CASE(12) W4_CASE(13) W4_CASE(14) W4_CASE(15) W4_CASE(16)
-#undef W4_CASE
-    }
-    return W4_ERR_ARG;
-}
 
 // NVFP4 decode GEMV on the tensor cores (gemv_tc.cuh).
 struct GemvTcPlan {
-    int S = 1, kc = 0, KP = 0, NS = 0, xstride = 0, tile_bytes = 0, grid = 0;
+    int M = 1, S = 1, kc = 0, KP = 0, NS = 0, xstride = 0, tile_bytes = 0, grid = 0;
     int rows_mode = 0, tiles_per_cta = 0, box_min_rows = 4, red_tiles = 2;
     size_t smem = 0, ws_bytes = 0;
 };
@@ -168,33 +71,55 @@ constexpr double kCopyUs = 0.2;         // cost of one bulk / tensor copy on an 
 
 // force_grid > 0: exactly that many CTAs, each on a balanced range of rows (the
 // grouped launch gives every problem its own share of the SMs).
-w4_status plan_gemv_tc(int K, int N, int M, bool pdl, GemvTcPlan &p, int force_grid = 0) {
+inline int block_bytes(int fmt) { return fmt == W4_FMT_ROCMFP4_DUAL ? 18 : 17; }
+
+w4_status plan_gemv_tc(int fmt, int K, int N, int M, bool pdl, GemvTcPlan &p, int force_grid = 0) {
     DeviceInfo d;
     if (device_info(d) != W4_OK) return W4_ERR_CUDA;
-    const int unit = 256;
+    p.M = M;
+    const bool nv = fmt == W4_FMT_NVFP4;
+    const int unit = k_unit(fmt);
     const int units = K / unit;
     int per = (int)std::max<size_t>(1, kXBudget / ((size_t)2 * M * unit));
     per = std::min(per, units);
     p.kc = per * unit;
     p.S = (units + per - 1) / per;
-    const int npieces = (p.kc + kTcPieceMax - 1) / kTcPieceMax;
+    // ROCmFP4 stages: a box row of KP/32 blocks is at most 256 8-byte elements
+    const int piece_max = nv ? kTcPieceMax : 3584;
+    int npieces = (p.kc + piece_max - 1) / piece_max;
     p.KP = ((p.kc + npieces - 1) / npieces + unit - 1) / unit * unit;
+    // the swizzled one-token layout needs KP/256 lines per row that are not a
+    // multiple of 8: take the next such KP (the last piece is then shorter), or
+    // one more piece when that would pass the box limit (KP/16 scale bytes <= 256)
+    while (nv && M == 1 && (p.KP / 256) % 8 == 0) {
+        if (p.KP + unit <= piece_max) {
+            p.KP += unit;
+        } else {
+            npieces++;
+            p.KP = ((p.kc + npieces - 1) / npieces + unit - 1) / unit * unit;
+        }
+    }
     p.xstride = p.kc + 32;
-    p.tile_bytes = (kTcRows * (p.KP / 2 + p.KP / 16) + 127) & ~127;
+    // stages start on 1024 bytes (the swizzle atom of the one-token codes box)
+    p.tile_bytes = nv ? (kTcRows * (p.KP / 2 + p.KP / 16) + 1023) & ~1023
+                      : (kTcRows * stage_row_bytes(fmt, block_bytes(fmt), p.KP) + 127) & ~127;
     const size_t xs = ((size_t)M * p.xstride * 2 + 127) & ~(size_t)127;
     const size_t tail = 16 + 4 * kTcWarps;   // flags
-    const size_t budget = std::min<size_t>(pdl ? 110 * 1024 : 200 * 1024, (size_t)d.smem_optin);
+    const size_t budget = std::min<size_t>(200 * 1024, (size_t)d.smem_optin);
 
-    // rows per CTA: balanced ranges (a partial last tile per CTA) or whole tiles
-    const double rowB = (double)K / 2 + K / 16;
+    // rows per CTA: balanced ranges (a partial last tile per CTA) or whole tiles.
+    // With split-K the S slices of a row range run side by side, so the row
+    // grid takes SMs / S: the launch stays one wave of resident CTAs.
+    const int row_sms = std::max(1, d.sms / p.S);
+    const double rowB = nv ? (double)K / 2 + K / 16 : (double)stage_row_bytes(fmt, block_bytes(fmt), K);
     const int T = (N + kTcRows - 1) / kTcRows;
-    const int gA = std::min(d.sms, N);
+    const int gA = std::min(row_sms, N);
     const int rowsA = (N + gA - 1) / gA, tailA = rowsA % kTcRows, fullA = rowsA / kTcRows;
     const int readA = fullA * kTcRows + (tailA >= p.box_min_rows ? kTcRows : tailA);
     const int copiesA = 2 * fullA + (tailA == 0 ? 0 : (tailA >= p.box_min_rows ? 2 : 2 * tailA));
     const double costA = std::max(readA * rowB / kSmBytesPerUs, (double)N * rowB / kHbmBytesPerUs) +
                          copiesA * p.S * kCopyUs;
-    const int q = (T + d.sms - 1) / d.sms, gB = (T + q - 1) / q;
+    const int q = (T + row_sms - 1) / row_sms, gB = (T + q - 1) / q;
     const double costB = std::max(q * kTcRows * rowB / kSmBytesPerUs, (double)T * kTcRows * rowB / kHbmBytesPerUs) +
                          2 * q * p.S * kCopyUs;
     int tiles_max;
@@ -221,7 +146,7 @@ w4_status plan_gemv_tc(int K, int N, int M, bool pdl, GemvTcPlan &p, int force_g
     const size_t red = (size_t)p.red_tiles * part_bytes;
 
     auto total = [&](int ns) -> size_t {
-        if (M == 1) return m1_layout(p.xstride, p.kc, ns, p.tile_bytes, p.red_tiles).total;
+        if (nv && M == 1) return m1_layout(p.xstride, p.kc, ns, p.tile_bytes, p.red_tiles).total;
         return xs + (size_t)ns * p.tile_bytes + red + 16 * ns + tail;
     };
     int NS = 8;
@@ -243,16 +168,39 @@ w4_status gemv_tc_setup(const w4_weights *w, const void *x, float *y, void *ws, 
     const cuuint64_t cdims[2] = {(cuuint64_t)K / 16, (cuuint64_t)N};   // codes as 8-byte elements
     const cuuint64_t cstr[1] = {(cuuint64_t)K / 2};
     const cuuint32_t cbox[2] = {(cuuint32_t)p.KP / 16, (cuuint32_t)kTcRows};
+    // one token: codes as [N][K/256][16 x 8 bytes], 3-D box of 16 rows x KP/256
+    // lines of 128 bytes, 128-byte swizzle (the consumers' chunk XOR)
+    const bool nv = w->fmt == W4_FMT_NVFP4;
+    const bool swz = nv && p.M == 1;
+    // ROCmFP4: blocks as 8-byte elements, a box of 16 rows x KP/32 blocks, no scales map
+    const int bb = nv ? 0 : block_bytes(w->fmt);
+    const cuuint64_t rdims[2] = {(cuuint64_t)stage_row_bytes(w->fmt, bb, K) / 8, (cuuint64_t)N};
+    const cuuint64_t rstr[1] = {(cuuint64_t)stage_row_bytes(w->fmt, bb, K)};
+    const cuuint32_t rbox[2] = {(cuuint32_t)stage_row_bytes(w->fmt, bb, p.KP) / 8, (cuuint32_t)kTcRows};
+    const cuuint64_t zdims[3] = {16, (cuuint64_t)K / 256, (cuuint64_t)N};
+    const cuuint64_t zstr[2] = {128, (cuuint64_t)K / 2};
+    const cuuint32_t zbox[3] = {16, (cuuint32_t)p.KP / 256, (cuuint32_t)kTcRows};
+    const cuuint32_t zestr[3] = {1, 1, 1};
     const cuuint64_t sdims[2] = {(cuuint64_t)K / 16, (cuuint64_t)N};
     const cuuint64_t sstr[1] = {(cuuint64_t)K / 16};
     const cuuint32_t sbox[2] = {(cuuint32_t)p.KP / 16, (cuuint32_t)kTcRows};
     const cuuint32_t estr[2] = {1, 1};
-    if (enc(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<uint8_t *>(w->codes), cdims, cstr, cbox, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+    if (!nv) {
+        if (enc(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<uint8_t *>(w->codes), rdims, rstr, rbox, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return W4_ERR_CUDA;
+        smap = cmap;
+    }
+    if (nv && ((swz ? enc(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT64, 3, const_cast<uint8_t *>(w->codes), zdims, zstr, zbox,
+                   zestr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE)
+             : enc(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<uint8_t *>(w->codes), cdims, cstr, cbox,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE)) != CUDA_SUCCESS ||
         enc(&smap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(w->scales), sdims, sstr, sbox, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS))
         return W4_ERR_CUDA;
     a.codes = w->codes;
     a.scales = w->scales;
@@ -272,14 +220,17 @@ w4_status gemv_tc_setup(const w4_weights *w, const void *x, float *y, void *ws, 
     a.box_min_rows = p.box_min_rows;
     a.red_tiles = p.red_tiles;
     a.pdl = pdl ? 1 : 0;
+    a.swz = swz ? 1 : 0;
+    a.fmt = w->fmt;
+    a.bb = bb;
     return W4_OK;
 }
 
-template <int M>
+template <int FMT, int M>
 w4_status launch_gemv_tc_m(const w4_weights *w, const void *x, float *y, void *ws, const GemvTcPlan &p, bool pdl,
                            cudaStream_t st) {
-    // one token: block scales applied after the MMA (gemv_m1.cuh)
-    auto kern = M == 1 ? gemv_nvfp4_m1_kernel : gemv_nvfp4_tc_kernel<M>;
+    // one NVFP4 token: block scales applied after the MMA (gemv_m1.cuh)
+    auto kern = (M == 1 && FMT == W4_FMT_NVFP4) ? gemv_nvfp4_m1_kernel : gemv_tc_kernel<FMT, M>;
     if (!set_smem_limit(reinterpret_cast<const void *>(kern), p.smem)) return W4_ERR_CUDA;
     const int N = w->N;
     CUtensorMap cmap, smap;
@@ -360,7 +311,7 @@ w4_status launch_gemv_grouped(const w4_weights *w, const void *const *x, float *
     size_t smem = 0;
     for (int p = 0; p < G; p++) {
         GemvTcPlan plan;
-        w4_status s = plan_gemv_tc(w[p].K, w[p].N, 1, pdl, plan, alloc[p]);
+        w4_status s = plan_gemv_tc(W4_FMT_NVFP4, w[p].K, w[p].N, 1, pdl, plan, alloc[p]);
         if (s != W4_OK) return s;
         if (plan.S != 1) return W4_ERR_UNSUPPORTED;
         s = gemv_tc_setup(&w[p], x[p], y[p], nullptr, plan, pdl, g.cmap[p], g.smap[p], g.a[p]);
@@ -383,16 +334,43 @@ w4_status launch_gemv_grouped(const w4_weights *w, const void *const *x, float *
     return launch_status();
 }
 
-w4_status launch_gemv_tc(const w4_weights *w, const void *x, int M, float *y, void *ws, const GemvTcPlan &p, bool pdl,
-                         cudaStream_t st) {
+template <int FMT>
+w4_status launch_gemv_tc_fmt(const w4_weights *w, const void *x, int M, float *y, void *ws, const GemvTcPlan &p,
+                             bool pdl, cudaStream_t st) {
     switch (M) {
 #define W4_CASE(m) \
-    case m: return launch_gemv_tc_m<m>(w, x, y, ws, p, pdl, st);
+    case m: return launch_gemv_tc_m<FMT, m>(w, x, y, ws, p, pdl, st);
         W4_CASE(1) W4_CASE(2) W4_CASE(3) W4_CASE(4) W4_CASE(5) W4_CASE(6) W4_CASE(7) W4_CASE(8)
         W4_CASE(9) W4_CASE(10) W4_CASE(11) W4_CASE(12) W4_CASE(13) W4_CASE(14) W4_CASE(15) W4_CASE(16)
 #undef W4_CASE
     }
     return W4_ERR_ARG;
+}
+
+w4_status launch_gemv_tc(const w4_weights *w, const void *x, int M, float *y, void *ws, const GemvTcPlan &p, bool pdl,
+                         cudaStream_t st) {
+    switch (w->fmt) {
+    case W4_FMT_NVFP4: return launch_gemv_tc_fmt<W4_FMT_NVFP4>(w, x, M, y, ws, p, pdl, st);
+    case W4_FMT_ROCMFP4_DUAL: return launch_gemv_tc_fmt<W4_FMT_ROCMFP4_DUAL>(w, x, M, y, ws, p, pdl, st);
+    case W4_FMT_ROCMFP4_FAST: return launch_gemv_tc_fmt<W4_FMT_ROCMFP4_FAST>(w, x, M, y, ws, p, pdl, st);
+    }
+    return W4_ERR_ARG;
+}
+
+// Any K the packers accept (gemv_any_kernel): one warp per weight row.
+template <int FMT>
+w4_status launch_gemv_any(const w4_weights *w, const void *x, int M, float *y, cudaStream_t st) {
+    const int grid = (w->N + 7) / 8;
+    const uint16_t *xb = reinterpret_cast<const uint16_t *>(x);
+    switch (M) {
+#define W4_CASE(m) \
+    case m: gemv_any_kernel<FMT, m><<<grid, 256, 0, st>>>(w->codes, w->scales, w->global_scale, xb, y, w->K, w->N); break;
+        W4_CASE(1) W4_CASE(2) W4_CASE(3) W4_CASE(4) W4_CASE(5) W4_CASE(6) W4_CASE(7) W4_CASE(8)
+        W4_CASE(9) W4_CASE(10) W4_CASE(11) W4_CASE(12) W4_CASE(13) W4_CASE(14) W4_CASE(15) W4_CASE(16)
+#undef W4_CASE
+    default: return W4_ERR_ARG;
+    }
+    return launch_status();
 }
 
 w4_status check_weights(const w4_weights *w) {
@@ -540,19 +518,11 @@ w4_status w4_reconstruction_error(const w4_weights *w, const void *W, double *ou
 
 size_t w4a16_workspace_bytes(const w4_weights *w, int M) {
     if (check_weights(w) != W4_OK || M < 1) return 0;
-    if (M <= 16 && w->fmt == W4_FMT_NVFP4) {
-        if (w->K % 256) return 0;   // (the tensor-memory path needs none either)
-        GemvTcPlan p, q;
-        if (plan_gemv_tc(w->K, w->N, M, false, p) != W4_OK) return 0;
-        if (plan_gemv_tc(w->K, w->N, M, true, q) != W4_OK) return p.ws_bytes;
-        return std::max(p.ws_bytes, q.ws_bytes);
-    }
     if (M <= 16) {
         if (w->K % k_unit(w->fmt)) return 0;
-        GemvPlan p;
-        if (plan_gemv(w->fmt, w->K, w->N, M, false, p) != W4_OK) return 0;
-        GemvPlan q;
-        if (plan_gemv(w->fmt, w->K, w->N, M, true, q) != W4_OK) return p.ws_bytes;
+        GemvTcPlan p, q;
+        if (plan_gemv_tc(w->fmt, w->K, w->N, M, false, p) != W4_OK) return 0;
+        if (plan_gemv_tc(w->fmt, w->K, w->N, M, true, q) != W4_OK) return p.ws_bytes;
         return std::max(p.ws_bytes, q.ws_bytes);
     }
     return gemm_workspace_bytes(w, M);
@@ -564,23 +534,21 @@ w4_status w4a16_gemv_ex(const w4_weights *w, const void *x, int M, float *y, voi
     if (s != W4_OK) return s;
     if (!x || !y || M < 1 || M > 16 || (flags & ~W4_LAUNCH_PDL)) return W4_ERR_ARG;
     if (!aligned16(x) || !aligned16(y) || (workspace && !aligned16(workspace))) return W4_ERR_ALIGN;
-    if (w->K % k_unit(w->fmt)) return W4_ERR_UNSUPPORTED;
     const bool pdl = (flags & W4_LAUNCH_PDL) != 0;
     cudaStream_t st = as_stream(stream);
-    if (w->fmt == W4_FMT_NVFP4) {
-        GemvTcPlan p;
-        if ((s = plan_gemv_tc(w->K, w->N, M, pdl, p)) != W4_OK) return s;
-        if (p.ws_bytes && (!workspace || workspace_bytes < p.ws_bytes)) return W4_ERR_WORKSPACE;
-        return launch_gemv_tc(w, x, M, y, workspace, p, pdl, st);
+    if (w->K % k_unit(w->fmt)) {
+        // K the fast kernels' 16-byte row pieces do not fit: the general path
+        switch (w->fmt) {
+        case W4_FMT_NVFP4: return launch_gemv_any<W4_FMT_NVFP4>(w, x, M, y, st);
+        case W4_FMT_ROCMFP4_DUAL: return launch_gemv_any<W4_FMT_ROCMFP4_DUAL>(w, x, M, y, st);
+        case W4_FMT_ROCMFP4_FAST: return launch_gemv_any<W4_FMT_ROCMFP4_FAST>(w, x, M, y, st);
+        }
+        return W4_ERR_ARG;
     }
-    GemvPlan p;
-    if ((s = plan_gemv(w->fmt, w->K, w->N, M, pdl, p)) != W4_OK) return s;
+    GemvTcPlan p;
+    if ((s = plan_gemv_tc(w->fmt, w->K, w->N, M, pdl, p)) != W4_OK) return s;
     if (p.ws_bytes && (!workspace || workspace_bytes < p.ws_bytes)) return W4_ERR_WORKSPACE;
-    switch (w->fmt) {
-    case W4_FMT_ROCMFP4_DUAL: return launch_gemv_fmt<W4_FMT_ROCMFP4_DUAL>(w, x, M, y, workspace, p, pdl, st);
-    case W4_FMT_ROCMFP4_FAST: return launch_gemv_fmt<W4_FMT_ROCMFP4_FAST>(w, x, M, y, workspace, p, pdl, st);
-    }
-    return W4_ERR_ARG;
+    return launch_gemv_tc(w, x, M, y, workspace, p, pdl, st);
 }
 
 w4_status w4_plan_grouped(const w4_weights *w, int G, int sms, unsigned flags, int *ctas) {
