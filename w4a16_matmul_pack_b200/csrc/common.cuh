@@ -158,6 +158,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     return false;
 }
 
+// Waits on barriers that another CTA of the cluster arrives on (a remote
+// arrival, a multicast commit) take the same form as local ones: the arrival
+// orders the arriving CTA's prior work, the wait acquires at CTA scope.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    return mbar_wait(bar, parity, abort);
+}
+
 // Global -> shared bulk copy (no multicast), completion counted in bytes on `bar`.
 // dst, src 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
@@ -199,15 +206,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
-// 3-D tiled TMA load (no multicast) of the box at (c0, c1, c2).
-__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int c0, int c1, int c2, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
-        "[%0], [%1, {%2, %3, %4}], [%5];"
-        ::"r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar))
-        : "memory");
-}
-
 // Wait as mbar_wait, but ignoring the CTA's abort flag and the settable limit
 // (still bounded, by kWaitLimitNs): for the completions a CTA must see before it
 // releases tensor memory or exits -- its own bulk copies and MMAs in flight.
@@ -221,6 +219,11 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
         }
     }
     return true;
+}
+
+// mbar_wait_bounded for barriers that another CTA of the cluster arrives on.
+__device__ __forceinline__ bool mbar_wait_bounded_cluster(uint64_t *bar, uint32_t parity) {
+    return mbar_wait_bounded(bar, parity);
 }
 
 // Raise a kernel's dynamic shared-memory limit to at least `bytes` on the

@@ -27,8 +27,8 @@
 // of 64 k with one tcgen05.st.
 //
 // Warp roles (24 warps):
-//   warp 0       TMA producer of x (the 192 x 64 BF16 / f16 tile of each stage,
-//                128-byte swizzle, six stages), no multicast.
+//   warp 0       TMA producer of x: three stages of 128 k, each two 192 x 64
+//                BF16 / f16 boxes with the 128-byte swizzle, no multicast.
 //   warp 1       allocates / frees the 512 TMEM columns; MMA issuer (one lane):
 //                4 x (128x192x16) per stage, commits to the stage barriers and
 //                to the accumulator barrier per tile.  It never waits on an
@@ -68,7 +68,8 @@ constexpr int BM = 128;      // weight rows per tile (MMA M)
 constexpr int BN = 192;      // tokens per tile (MMA N)
 constexpr int BK = 64;       // k per stage (one 128-byte swizzle row of BF16)
 constexpr int STAGES = 4;    // A stages in tensor memory (32 columns each), one per dequant group
-constexpr int XSTAGES = 6;   // x stages in shared memory
+constexpr int XK = 2;        // k-steps per x stage (one 192 x 64 swizzled box each)
+constexpr int XSTAGES = 3;   // x stages in shared memory (48 KB each)
 constexpr int kGroups = STAGES;
 constexpr int kDqWarp0 = 6;
 constexpr int kDqWarps = 4 * kGroups;
@@ -77,7 +78,8 @@ constexpr int kWProdWarp = kWaitWarp + 1;        // 23
 constexpr int kWarps = kWProdWarp + 1;           // 24
 constexpr int kThreads = kWarps * 32;
 constexpr int kEpiThreads = 128;
-constexpr uint32_t X_STAGE_BYTES = BN * BK * 2;   // 24 KB
+constexpr uint32_t X_BOX_BYTES = BN * BK * 2;    // 24 KB: one k-step of x
+constexpr uint32_t X_STAGE_BYTES = XK * X_BOX_BYTES;
 constexpr uint32_t TMEM_COLS = 512;               // 4 A stages (32 columns each) + two 192-column accumulators
 constexpr uint32_t ACC_COL0 = STAGES * (BK / 2);  // accumulators after the A stages
 constexpr int kMaxTilesM = 256;   // token tiles whose operand mode is kept in shared memory (M <= 49152)
@@ -411,16 +413,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     if (warp == 0) {
         // ---------------------------- x producer (TMA) ----------------------------
         if (lane == 0) {
-            int it = 0;
+            // x stages of XK k-steps: fewer, larger copies stream faster than
+            // one stage per k-step
+            int it = 0;   // x stages issued
             for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x) {
                 const int m0 = (t % p.tiles_m) * BN;
                 const CUtensorMap *xm = sh.f16_tile[t % p.tiles_m] ? &xmap16 : &xmap;
-                for (int kt = 0; kt < KT; kt++, it++) {
-                    const int s = it % XSTAGES;
+                for (int kt = 0; kt < KT; kt += XK, it++) {
+                    const int s = it % XSTAGES, nk = min(XK, KT - kt);
                     if (it >= XSTAGES) mbar_wait(&sh.x_empty[s], ((it / XSTAGES) - 1) & 1, abort);
                     if (*abort) break;
-                    mbar_arrive_expect_tx(&sh.x_full[s], X_STAGE_BYTES);
-                    tma_load_2d(sh.x[s], xm, kt * BK, m0, &sh.x_full[s]);
+                    mbar_arrive_expect_tx(&sh.x_full[s], (uint32_t)nk * X_BOX_BYTES);
+                    for (int j = 0; j < nk; j++)
+                        tma_load_2d(sh.x[s] + j * X_BOX_BYTES, xm, (kt + j) * BK, m0, &sh.x_full[s]);
                 }
             }
             // every issued copy has landed before the CTA can exit (after an abort
@@ -461,26 +466,27 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         // pipe idle between stages.  So this warp never waits on an mbarrier:
         // warp kWaitWarp waits for each stage (and each accumulator) and then
         // meets it at named barrier 2; lane 0 issues.
-        int it = 0;
+        int it = 0, xi = 0;   // k-steps, x stages
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
             const int b = ((t - blockIdx.x) / gridDim.x) & 1;
             const uint32_t dtm = tmem + ACC_COL0 + (uint32_t)(b * BN);
             const uint32_t idesc = sh.f16_tile[t % p.tiles_m] ? IDESC_F16 : IDESC;
             for (int kt = 0; kt < KT; kt++, it++) {
-                const int s = it % STAGES, xs = it % XSTAGES;
-                named_barrier_sync(2, 64);   // stage it (and, at kt == 0, accumulator b) is ready
+                const int s = it % STAGES, xs = xi % XSTAGES, sub = kt % XK;
+                named_barrier_sync(2, 64);   // k-step it (and, at kt == 0, accumulator b) is ready
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t xb = smem_addr(sh.x[xs]);
+                    const uint32_t xb = smem_addr(sh.x[xs]) + (uint32_t)(sub * X_BOX_BYTES);
 #pragma unroll
                     for (int j = 0; j < BK / 16; j++)   // A (16 k = 8 columns) from tensor memory
                         mma_ts(dtm, tmem + (uint32_t)(s * (BK / 2) + 8 * j), sw128_desc(xb + 32 * j), idesc,
                                (kt | j) ? 1u : 0u);
-                    mma_commit(&sh.x_empty[xs]);
                     mma_commit(&sh.a_empty[s]);
+                    if (sub == XK - 1 || kt == KT - 1) mma_commit(&sh.x_empty[xs]);
                     if (kt == KT - 1) mma_commit(&sh.acc_full[b]);
                 }
                 __syncwarp();
+                if (sub == XK - 1 || kt == KT - 1) xi++;
             }
         }
         // tensor memory is released after the final barrier: every MMA this
@@ -492,15 +498,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         __syncwarp();
     } else if (warp == kWaitWarp) {
         // ------------------------- waits on behalf of the MMA issuer -------------------------
-        int it = 0, lt = 0;
+        int it = 0, lt = 0, xi = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, lt++) {
             const int b = lt & 1;
             if (lt >= 2) mbar_wait(&sh.acc_empty[b], ((lt >> 1) - 1) & 1, abort);
             for (int kt = 0; kt < KT; kt++, it++) {
                 // on expiry (abort) the stage is garbage, but both warps still meet every barrier
-                mbar_wait(&sh.x_full[it % XSTAGES], (it / XSTAGES) & 1, abort);
+                if (kt % XK == 0) mbar_wait(&sh.x_full[xi % XSTAGES], (xi / XSTAGES) & 1, abort);
                 mbar_wait(&sh.a_full[it % STAGES], (it / STAGES) & 1, abort);
                 named_barrier_sync(2, 64);
+                if (kt % XK == XK - 1 || kt == KT - 1) xi++;
             }
         }
     } else if (warp < kDqWarp0) {

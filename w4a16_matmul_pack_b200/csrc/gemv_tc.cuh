@@ -56,7 +56,6 @@ struct GemvTcArgs {
     int red_tiles;       // tiles whose partial sums fit the reduction buffer at once (>= ntiles:
                          // one barrier per CTA; else 2 and a barrier per tile)
     int pdl;             // launched with programmatic dependent launch: prefetch weights before x
-    int swz;             // codes staged by the 3-D box with the 128-byte swizzle (one-token kernel)
     int fmt;             // w4_format
     int bb;              // ROCmFP4 block bytes (18 Dual, 17 FAST)
 };
@@ -65,27 +64,6 @@ struct GemvTcArgs {
 // codes), or ROCmFP4 blocks.
 __host__ __device__ __forceinline__ int stage_row_bytes(int fmt, int bb, int kp) {
     return fmt == W4_FMT_NVFP4 ? kp / 2 : (kp / 32) * bb;
-}
-
-// One-token kernel, swizzled codes stage: a tile's codes arrive as [row][KP/256]
-// lines of 128 bytes (two 128-k super-chunks each), the 16-byte chunk index
-// XORed with the line index mod 8.  The MMA row g of a warp's quarter (rows g
-// and g^1 are read together) maps to a physical row chosen so that the two rows'
-// lines differ by 4 mod 8: their chunks then fall in opposite halves of the 32
-// banks.  d is that row distance for `lines` lines per row (lines % 8 != 0).
-__host__ __device__ __forceinline__ int swz_row_distance(int lines) {
-    return (lines & 1) ? 4 : ((lines & 3) == 2 ? 2 : 1);
-}
-__device__ __forceinline__ int swz_phys_row(int g, int d) {   // g in 0..7
-    const int i = g >> 1, j = g & 1;
-    const int b = d == 1 ? 2 * i : (d == 2 ? (i & 1) + 4 * (i >> 1) : i);
-    return b + j * d;
-}
-// Byte offset of 16-byte chunk c (0..7 within the 128-k super-chunk pair; chunk
-// 4*(s&1) + t of super-chunk s) of physical row pr in a swizzled codes stage.
-__device__ __forceinline__ uint32_t swz_chunk(int pr, int s, int t, int lines) {
-    const int line = pr * lines + (s >> 1);
-    return (uint32_t)(line * 128 + ((((s & 1) << 2) | t) ^ (line & 7)) * 16);
 }
 
 // v * 2^e for |e| <= 252 as two exact multiplies (each factor a normal power of two).
@@ -260,10 +238,7 @@ __device__ __forceinline__ void tc_produce(const CUtensorMap &cmap, const CUtens
         } else if (rows == kTcRows || rows >= a.box_min_rows) {
             // two boxes of 16 rows x KP (k beyond K and rows beyond N are zero-filled)
             mbar_arrive_expect_tx(full + st, (uint32_t)(kTcRows * (CS + SS)));
-            if (a.swz)
-                tma_load_3d(dst, &cmap, 0, kpos / 256, (int)rt, full + st);
-            else
-                tma_load_2d(dst, &cmap, kpos / 16, (int)rt, full + st);
+            tma_load_2d(dst, &cmap, kpos / 16, (int)rt, full + st);
             tma_load_2d(dsts, &smap, kpos / 16, (int)rt, full + st);
         } else {
             // a short tail: row-piece copies of exactly the bytes needed
@@ -286,15 +261,15 @@ __device__ __forceinline__ void tc_produce(const CUtensorMap &cmap, const CUtens
 // first put x[j], x[j+16] side by side within each 32-k block).  sigma puts the
 // largest |x| in [2^14, 2^15); flags[1] is set when some x does not convert
 // exactly (a nonzero |x'| below 2^-17 scaled back differs, Inf / NaN), and the
-// caller then takes the binary32 path.  All consumer warps take part (named
-// barrier 1); flags[2 .. 2 + kTcWarps) is scratch.  mx: the largest |x| (BF16 bits).
-template <bool VIRT>
+// caller then takes the binary32 path.  All NW consumer warps take part (named
+// barrier 1); flags[2 .. 2 + NW) is scratch.  mx: the largest |x| (BF16 bits).
+template <bool VIRT, int NW = kTcWarps>
 __device__ __forceinline__ void convert_x_f16(uint16_t *xs, int XS, int M, int kcs, int warp, int lane, int *flags,
                                               int &sigma, uint32_t &mx) {
     mx = 0;
     {
         const int nvec = kcs / 8;
-        for (int i = threadIdx.x; i < M * nvec; i += kTcWarps * 32) {
+        for (int i = threadIdx.x; i < M * nvec; i += NW * 32) {
             const int m = i / nvec, v = i % nvec;
             const uint4 val = *reinterpret_cast<const uint4 *>(xs + (size_t)m * XS + v * 8);
             const uint32_t w4v[4] = {val.x, val.y, val.z, val.w};
@@ -305,15 +280,15 @@ __device__ __forceinline__ void convert_x_f16(uint16_t *xs, int XS, int M, int k
 #pragma unroll
     for (int o = 16; o; o >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
     if (lane == 0) flags[2 + warp] = (int)mx;
-    named_barrier_sync(1, kTcWarps * 32);
-    for (int i = 0; i < kTcWarps; i++) mx = max(mx, (uint32_t)flags[2 + i]);
+    named_barrier_sync(1, NW * 32);
+    for (int i = 0; i < NW; i++) mx = max(mx, (uint32_t)flags[2 + i]);
     const int emax = (int)((mx >> 7) & 0xFFu);
     sigma = (mx == 0) ? 0 : max(emax, 1) - 127 - 14;
     // A warp owns whole super-chunks (lane l converts vector l % 16 of super-chunk
     // 2i + l / 16), so __syncwarp orders its loads before its stores.
     const int nsc = kcs / 128, total = M * nsc;
     bool bad = mx >= 0x7F80u;   // NaN / Inf: binary32 path
-    for (int base = 2 * warp; base < total; base += 2 * kTcWarps) {
+    for (int base = 2 * warp; base < total; base += 2 * NW) {
         const int sc = base + (lane >> 4), q = lane & 15;
         uint4 out = make_uint4(0, 0, 0, 0);
         uint16_t *row = nullptr;

@@ -73,9 +73,45 @@ constexpr double kCopyUs = 0.2;         // cost of one bulk / tensor copy on an 
 // grouped launch gives every problem its own share of the SMs).
 inline int block_bytes(int fmt) { return fmt == W4_FMT_ROCMFP4_DUAL ? 18 : 17; }
 
+// One NVFP4 token (gemv_m1.cuh): K slices of at most kM1MaxSlice (x' of a slice
+// in shared memory as f16); a problem with fewer 16-row tiles than half the SMs
+// is also split along K (slices of at least 2048 k) so that the launch still
+// fills the GPU; at most kM1MaxTiles tiles per CTA (its partial-sum buffer).
+constexpr int kM1MaxSlice = 32768;
+constexpr int kM1MaxTiles = 32;
+
+w4_status plan_gemv_m1(int K, int N, GemvTcPlan &p, int force_grid, const DeviceInfo &d) {
+    p.M = 1;
+    const int T = (N + kTcRows - 1) / kTcRows;
+    int S = (K + kM1MaxSlice - 1) / kM1MaxSlice;
+    if (force_grid <= 0 && T < d.sms / 2) S = std::max(S, std::min(d.sms / T, K / 2048));
+    S = std::max(S, 1);
+    p.kc = ((K + S - 1) / S + 255) / 256 * 256;
+    p.S = (K + p.kc - 1) / p.kc;
+    if (force_grid > 0) {
+        if (p.S != 1) return W4_ERR_UNSUPPORTED;
+        p.grid = std::min(force_grid, T);
+    } else {
+        p.grid = std::min(T, std::max(1, d.sms / p.S));
+        p.grid = std::max(p.grid, (T + kM1MaxTiles - 1) / kM1MaxTiles);
+    }
+    p.red_tiles = (T + p.grid - 1) / p.grid;
+    p.xstride = p.kc + 32;
+    p.KP = p.kc;
+    p.NS = 0;
+    p.tile_bytes = 0;
+    p.rows_mode = 1;
+    p.tiles_per_cta = p.red_tiles;
+    p.smem = m1_layout(p.xstride, p.red_tiles).total;
+    if (p.smem > (size_t)d.smem_optin) return W4_ERR_UNSUPPORTED;
+    p.ws_bytes = p.S > 1 ? (size_t)p.S * N * sizeof(float) : 0;
+    return W4_OK;
+}
+
 w4_status plan_gemv_tc(int fmt, int K, int N, int M, bool pdl, GemvTcPlan &p, int force_grid = 0) {
     DeviceInfo d;
     if (device_info(d) != W4_OK) return W4_ERR_CUDA;
+    if (fmt == W4_FMT_NVFP4 && M == 1) return plan_gemv_m1(K, N, p, force_grid, d);
     p.M = M;
     const bool nv = fmt == W4_FMT_NVFP4;
     const int unit = k_unit(fmt);
@@ -88,20 +124,8 @@ w4_status plan_gemv_tc(int fmt, int K, int N, int M, bool pdl, GemvTcPlan &p, in
     const int piece_max = nv ? kTcPieceMax : 3584;
     int npieces = (p.kc + piece_max - 1) / piece_max;
     p.KP = ((p.kc + npieces - 1) / npieces + unit - 1) / unit * unit;
-    // the swizzled one-token layout needs KP/256 lines per row that are not a
-    // multiple of 8: take the next such KP (the last piece is then shorter), or
-    // one more piece when that would pass the box limit (KP/16 scale bytes <= 256)
-    while (nv && M == 1 && (p.KP / 256) % 8 == 0) {
-        if (p.KP + unit <= piece_max) {
-            p.KP += unit;
-        } else {
-            npieces++;
-            p.KP = ((p.kc + npieces - 1) / npieces + unit - 1) / unit * unit;
-        }
-    }
     p.xstride = p.kc + 32;
-    // stages start on 1024 bytes (the swizzle atom of the one-token codes box)
-    p.tile_bytes = nv ? (kTcRows * (p.KP / 2 + p.KP / 16) + 1023) & ~1023
+    p.tile_bytes = nv ? (kTcRows * (p.KP / 2 + p.KP / 16) + 127) & ~127
                       : (kTcRows * stage_row_bytes(fmt, block_bytes(fmt), p.KP) + 127) & ~127;
     const size_t xs = ((size_t)M * p.xstride * 2 + 127) & ~(size_t)127;
     const size_t tail = 16 + 4 * kTcWarps;   // flags
@@ -145,10 +169,7 @@ w4_status plan_gemv_tc(int fmt, int K, int N, int M, bool pdl, GemvTcPlan &p, in
     p.red_tiles = (tiles_max * part_bytes <= 24 * 1024) ? std::max(tiles_max, 2) : 2;
     const size_t red = (size_t)p.red_tiles * part_bytes;
 
-    auto total = [&](int ns) -> size_t {
-        if (nv && M == 1) return m1_layout(p.xstride, p.kc, ns, p.tile_bytes, p.red_tiles).total;
-        return xs + (size_t)ns * p.tile_bytes + red + 16 * ns + tail;
-    };
+    auto total = [&](int ns) -> size_t { return xs + (size_t)ns * p.tile_bytes + red + 16 * ns + tail; };
     int NS = 8;
     while (NS > 2 && total(NS) > budget) NS--;
     p.NS = NS;
@@ -171,16 +192,12 @@ w4_status gemv_tc_setup(const w4_weights *w, const void *x, float *y, void *ws, 
     // one token: codes as [N][K/256][16 x 8 bytes], 3-D box of 16 rows x KP/256
     // lines of 128 bytes, 128-byte swizzle (the consumers' chunk XOR)
     const bool nv = w->fmt == W4_FMT_NVFP4;
-    const bool swz = nv && p.M == 1;
+    const bool direct = nv && p.M == 1;   // the one-token kernel loads its operands directly
     // ROCmFP4: blocks as 8-byte elements, a box of 16 rows x KP/32 blocks, no scales map
     const int bb = nv ? 0 : block_bytes(w->fmt);
     const cuuint64_t rdims[2] = {(cuuint64_t)stage_row_bytes(w->fmt, bb, K) / 8, (cuuint64_t)N};
     const cuuint64_t rstr[1] = {(cuuint64_t)stage_row_bytes(w->fmt, bb, K)};
     const cuuint32_t rbox[2] = {(cuuint32_t)stage_row_bytes(w->fmt, bb, p.KP) / 8, (cuuint32_t)kTcRows};
-    const cuuint64_t zdims[3] = {16, (cuuint64_t)K / 256, (cuuint64_t)N};
-    const cuuint64_t zstr[2] = {128, (cuuint64_t)K / 2};
-    const cuuint32_t zbox[3] = {16, (cuuint32_t)p.KP / 256, (cuuint32_t)kTcRows};
-    const cuuint32_t zestr[3] = {1, 1, 1};
     const cuuint64_t sdims[2] = {(cuuint64_t)K / 16, (cuuint64_t)N};
     const cuuint64_t sstr[1] = {(cuuint64_t)K / 16};
     const cuuint32_t sbox[2] = {(cuuint32_t)p.KP / 16, (cuuint32_t)kTcRows};
@@ -192,15 +209,13 @@ w4_status gemv_tc_setup(const w4_weights *w, const void *x, float *y, void *ws, 
             return W4_ERR_CUDA;
         smap = cmap;
     }
-    if (nv && ((swz ? enc(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT64, 3, const_cast<uint8_t *>(w->codes), zdims, zstr, zbox,
-                   zestr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE)
-             : enc(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<uint8_t *>(w->codes), cdims, cstr, cbox,
-                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE)) != CUDA_SUCCESS ||
-        enc(&smap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(w->scales), sdims, sstr, sbox, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS))
+    if (nv && !direct &&
+        (enc(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<uint8_t *>(w->codes), cdims, cstr, cbox, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+         enc(&smap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(w->scales), sdims, sstr, sbox, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS))
         return W4_ERR_CUDA;
     a.codes = w->codes;
     a.scales = w->scales;
@@ -220,7 +235,6 @@ w4_status gemv_tc_setup(const w4_weights *w, const void *x, float *y, void *ws, 
     a.box_min_rows = p.box_min_rows;
     a.red_tiles = p.red_tiles;
     a.pdl = pdl ? 1 : 0;
-    a.swz = swz ? 1 : 0;
     a.fmt = w->fmt;
     a.bb = bb;
     return W4_OK;
@@ -229,9 +243,12 @@ w4_status gemv_tc_setup(const w4_weights *w, const void *x, float *y, void *ws, 
 template <int FMT, int M>
 w4_status launch_gemv_tc_m(const w4_weights *w, const void *x, float *y, void *ws, const GemvTcPlan &p, bool pdl,
                            cudaStream_t st) {
-    // one NVFP4 token: block scales applied after the MMA (gemv_m1.cuh)
-    auto kern = (M == 1 && FMT == W4_FMT_NVFP4) ? gemv_nvfp4_m1_kernel : gemv_tc_kernel<FMT, M>;
-    if (!set_smem_limit(reinterpret_cast<const void *>(kern), p.smem)) return W4_ERR_CUDA;
+    // one NVFP4 token: block scales applied after the MMA, operands loaded
+    // directly (gemv_m1.cuh); otherwise TMA-staged tiles (gemv_tc.cuh)
+    constexpr bool direct = M == 1 && FMT == W4_FMT_NVFP4;
+    const void *kern = direct ? reinterpret_cast<const void *>(gemv_nvfp4_m1_kernel)
+                              : reinterpret_cast<const void *>(gemv_tc_kernel<FMT, M>);
+    if (!set_smem_limit(kern, p.smem)) return W4_ERR_CUDA;
     const int N = w->N;
     CUtensorMap cmap, smap;
     GemvTcArgs a;
@@ -239,7 +256,7 @@ w4_status launch_gemv_tc_m(const w4_weights *w, const void *x, float *y, void *w
     if (s0 != W4_OK) return s0;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.grid, p.S, 1);
-    cfg.blockDim = dim3(kTcThreads, 1, 1);
+    cfg.blockDim = dim3(direct ? kM1Threads : kTcThreads, 1, 1);
     cfg.dynamicSmemBytes = p.smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -247,7 +264,12 @@ w4_status launch_gemv_tc_m(const w4_weights *w, const void *x, float *y, void *w
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    if (cudaLaunchKernelEx(&cfg, kern, cmap, smap, a) != cudaSuccess) return W4_ERR_CUDA;
+    cudaError_t e;
+    if constexpr (direct)
+        e = cudaLaunchKernelEx(&cfg, gemv_nvfp4_m1_kernel, a);
+    else
+        e = cudaLaunchKernelEx(&cfg, gemv_tc_kernel<FMT, M>, cmap, smap, a);
+    if (e != cudaSuccess) return W4_ERR_CUDA;
     if (p.S > 1) {
         const int MN = M * N;
         // the slice partials already carry the global scale (scale_out)
@@ -314,7 +336,8 @@ w4_status launch_gemv_grouped(const w4_weights *w, const void *const *x, float *
         w4_status s = plan_gemv_tc(W4_FMT_NVFP4, w[p].K, w[p].N, 1, pdl, plan, alloc[p]);
         if (s != W4_OK) return s;
         if (plan.S != 1) return W4_ERR_UNSUPPORTED;
-        s = gemv_tc_setup(&w[p], x[p], y[p], nullptr, plan, pdl, g.cmap[p], g.smap[p], g.a[p]);
+        CUtensorMap unused_c, unused_s;
+        s = gemv_tc_setup(&w[p], x[p], y[p], nullptr, plan, pdl, unused_c, unused_s, g.a[p]);
         if (s != W4_OK) return s;
         g.cta0[p + 1] = g.cta0[p] + plan.grid;
         smem = std::max(smem, plan.smem);
@@ -322,7 +345,7 @@ w4_status launch_gemv_grouped(const w4_weights *w, const void *const *x, float *
     if (!set_smem_limit(reinterpret_cast<const void *>(gemv_nvfp4_m1_grouped_kernel), smem)) return W4_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(g.cta0[G], 1, 1);
-    cfg.blockDim = dim3(kTcThreads, 1, 1);
+    cfg.blockDim = dim3(kM1Threads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
