@@ -123,6 +123,8 @@ struct SharedStorage {
     uint32_t tmem_base;
     int abort;
     int f16_tile[kMaxTilesM];                   // token tile mt runs with f16 operands (else BF16)
+    float fac[BN];                              // epilogue: g * 2^e of each token of the tile (NaN: not exact)
+    int fac_exact;                              // every factor of the tile is exact
 };
 
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row atoms of
@@ -303,6 +305,7 @@ __device__ __forceinline__ uint32_t absmax_bf16x8(uint32_t mx, uint4 v) {
 
 __global__ void __launch_bounds__(256) x_to_f16_kernel(const uint16_t *x, uint16_t *xh, int *sigma, int *bad, int M,
                                                        int K) {
+    pdl_allow_dependents();   // the GEMM may start its prologue; it waits for this grid before reading x
     const int m = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
     if (m >= M) return;   // whole warps
     const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)m * K);
@@ -403,6 +406,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sh.tmem_base;
+    // with the f16 pass launched just before (programmatic dependent launch),
+    // everything above overlapped its tail; x, sigma and bad are its output
+    pdl_wait_prior_grid();
     if (use_f16) {
         // a token tile runs on f16 operands only if all of its rows converted exactly
         for (int i = threadIdx.x; i < p.M; i += kThreads)
@@ -516,35 +522,51 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         const float g = NV ? __ldg(p.gscale) : 1.0f;   // ROCmFP4: no global scale
         const int fold = NV ? bf16_fold(g) : 0;
         int lt = 0;
+        const int et = threadIdx.x - 2 * 32;   // 0..127 over the four epilogue warps
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, lt++) {
             const int b = lt & 1;
             const int m0 = (t % p.tiles_m) * BN, n0 = (t / p.tiles_m) * BM;
+            const bool f16 = sh.f16_tile[t % p.tiles_m] != 0;
+            // the tile's per-token factors g * 2^e (f16 tiles: token m was scaled by
+            // 2^-sigma_m), exact in binary32 when a normal number or zero: then acc *
+            // factor rounded once is the binary64 product of scale_out rounded once,
+            // bit for bit; otherwise NaN, and that token goes through scale_out
+            named_barrier_sync(3, kEpiThreads);   // the previous tile's factors are no longer read
+            if (et == 0) sh.fac_exact = 1;
+            named_barrier_sync(3, kEpiThreads);
+            for (int i = et; i < BN; i += kEpiThreads) {
+                const int m = m0 + i;
+                const int e = f16 ? (m < p.M ? __ldg(p.sigma + m) : 0) : -fold;
+                const float f = epilogue_factor(g, e);
+                sh.fac[i] = f;
+                if (isnan(f)) sh.fac_exact = 0;
+            }
+            named_barrier_sync(3, kEpiThreads);
+            const bool exact = sh.fac_exact != 0;
             mbar_wait(&sh.acc_full[b], (lt >> 1) & 1, abort);
             tc_fence_after();
             const int n = n0 + q * 32 + lane;
-            const bool f16 = sh.f16_tile[t % p.tiles_m] != 0;
+            const bool nok = n < p.N;
             for (int c = 0; c < BN / 16; c++) {
                 uint32_t v[16];
                 W4_TMEM_LD16(tmem + ((uint32_t)(q * 32) << 16) + ACC_COL0 + (uint32_t)(b * BN + c * 16), v);
                 asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-                // f16 tiles: token m was scaled by 2^-sigma_m (lane j < 16 holds sigma of token c*16+j)
-                const int mlane = m0 + c * 16 + (lane & 15);
-                const int el = f16 ? (mlane < p.M ? __ldg(p.sigma + mlane) : 0) : -fold;
-                // g * 2^e as a binary32 factor when that is exact (a normal number or
-                // zero): then acc * factor, rounded once, is the binary64 product of
-                // scale_out rounded once, bit for bit; otherwise scale_out
-                const float gl = epilogue_factor(g, el);
+                const int mc = m0 + c * 16;
 #pragma unroll
                 for (int j = 0; j < 16; j++) {
-                    const int e = __shfl_sync(0xFFFFFFFFu, el, j);   // every lane takes part
-                    const float gj = __shfl_sync(0xFFFFFFFFu, gl, j);
-                    const int m = m0 + c * 16 + j;
-                    if (n < p.N && m < p.M) {
-                        const float acc = __uint_as_float(v[j]);
-                        const float val = isnan(gj) ? scale_out(acc, g, e) : acc * gj;
-                        if (p.y32) p.y32[(size_t)m * p.N + n] = val;
-                        if (p.y16) p.y16[(size_t)m * p.N + n] = __float2bfloat16_rn(val);
+                    const int m = mc + j;
+                    if (!nok || m >= p.M) continue;
+                    const float acc = __uint_as_float(v[j]);
+                    const float gj = sh.fac[c * 16 + j];   // the same address in every lane
+                    float val;
+                    if (exact) {
+                        val = acc * gj;
+                    } else {
+                        const int e = f16 ? __ldg(p.sigma + m) : -fold;
+                        val = isnan(gj) ? scale_out(acc, g, e) : acc * gj;
                     }
+                    if (p.y32) p.y32[(size_t)m * p.N + n] = val;
+                    if (p.y16) p.y16[(size_t)m * p.N + n] = __float2bfloat16_rn(val);
                 }
             }
             tc_fence_before();
@@ -733,7 +755,17 @@ inline w4_status gemm_launch_fmt(const w4_weights *w, const void *x, int M, floa
         x_to_f16_kernel<<<(M + 7) / 8, 256, 0, st>>>(reinterpret_cast<const uint16_t *>(x), xh, sigma, bad, M, K);
     const int ntiles = p.tiles_m * p.tiles_n;
     const int grid = std::max(1, std::min(ntiles, sms));   // persistent, one CTA per SM
-    gemm_kernel<FMT><<<grid, kThreads, smem, st>>>(map, map16, cmap, smap, p);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = f16 ? 1 : 0;   // overlap the prologue with the f16 pass just launched
+    if (cudaLaunchKernelEx(&cfg, gemm_kernel<FMT>, map, map16, cmap, smap, p) != cudaSuccess) return W4_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
 
