@@ -45,6 +45,17 @@ __device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
     return r;
 }
 
+// 4 code bytes (8 E2M1 values, element 2i in the low nibble of byte i) -> 4
+// f16x2 (h[i] = elements 2i, 2i+1), exact.  The word is split into its bytes
+// as a vector move, so the conversions read their bytes in place instead of
+// after a shift and a truncation each.
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t *h) {
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3]) : "r"(w));
+}
+
 // E4M3FN byte (low 8 bits) -> float.  Exact.
 __device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
     uint32_t r;

@@ -185,9 +185,11 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
 // 4 code bytes (8 E2M1 values, element 2i in the low nibble of byte i) times a
 // scale -> 4 BF16x2 words at o[0..3].  Exact.
 __device__ __forceinline__ void dequant8_bf16(uint32_t cw, float s, uint32_t *o) {
+    uint32_t hh[4];
+    e2m1x8_to_f16x2(cw, hh);
 #pragma unroll
     for (int i = 0; i < 4; i++) {
-        const uint32_t h = e2m1x2_to_f16x2(cw >> (8 * i));
+        const uint32_t h = hh[i];
         const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h));
         const float2 v = __fmul2_rn(f, make_float2(s, s));
         const __nv_bfloat162 b = __float22bfloat162_rn(v);
@@ -198,8 +200,9 @@ __device__ __forceinline__ void dequant8_bf16(uint32_t cw, float s, uint32_t *o)
 // The same 8 weights as f16x2 words: cvt E2M1 -> f16x2, HMUL2 by the scale
 // (s2 = the scale in both halves).  Exact.
 __device__ __forceinline__ void dequant8_f16(uint32_t cw, uint32_t s2, uint32_t *o) {
+    e2m1x8_to_f16x2(cw, o);
 #pragma unroll
-    for (int i = 0; i < 4; i++) o[i] = hmul2_u32(e2m1x2_to_f16x2(cw >> (8 * i)), s2);
+    for (int i = 0; i < 4; i++) o[i] = hmul2_u32(o[i], s2);
 }
 
 // One ROCmFP4 block (32 weights at shared-memory byte address A: Dual = two

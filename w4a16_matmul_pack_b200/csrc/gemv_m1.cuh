@@ -68,9 +68,10 @@ __host__ __device__ __forceinline__ M1Layout m1_layout(int xstride, int red_tile
 
 // 16 code bytes of one row (32 k) -> 16 f16x2 (h[i] = elements 2i, 2i+1), exact.
 __device__ __forceinline__ void decode_codes32(uint4 c, uint32_t (&h)[16]) {
-    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
-#pragma unroll
-    for (int i = 0; i < 16; i++) h[i] = e2m1x2_to_f16x2(w[i >> 2] >> (8 * (i & 3)));
+    e2m1x8_to_f16x2(c.x, h);
+    e2m1x8_to_f16x2(c.y, h + 4);
+    e2m1x8_to_f16x2(c.z, h + 8);
+    e2m1x8_to_f16x2(c.w, h + 12);
 }
 
 // E4M3 byte (bits 0..7 of v after the shift) -> its value * 2^-120 as binary32
@@ -78,6 +79,55 @@ __device__ __forceinline__ void decode_codes32(uint4 c, uint32_t (&h)[16]) {
 // a binary32 subnormal of the same scaled value.
 __device__ __forceinline__ float e4m3_lo_scaled(uint32_t v) { return __uint_as_float((v << 20) & 0x07F00000u); }
 __device__ __forceinline__ float e4m3_hi_scaled(uint32_t v) { return __uint_as_float((v << 12) & 0x07F00000u); }
+
+// x' in shared memory: per 128-k super-chunk the 128 values in MMA operand
+// order (the 8 values k = 32t + 8j .. +7 at offset 32j + 8t) followed by 8
+// zeros, so that every lane loads its four B pieces (or zeros) by address.
+constexpr int kM1ScStride = 136;   // halves per super-chunk
+
+// x slice (BF16, global) -> x' = x * 2^-sigma as f16 in that layout, with one
+// power of two for the slice (its largest |x'| in [2^14, 2^15)); flags[1] is
+// set when some x does not convert exactly (a nonzero |x'| below 2^-17 scaled
+// back differs, Inf / NaN).  All kM1Warps warps take part; flags[2 ..] is
+// scratch.  mx: the largest |x| (BF16 bits).
+__device__ __forceinline__ void m1_convert_x(const uint16_t *xg, uint16_t *xs, int kcs, int warp, int lane,
+                                             int *flags, int &sigma, uint32_t &mx) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(xg);
+    const int nvec = kcs / 8;
+    mx = 0;
+    for (int i = threadIdx.x; i < nvec; i += kM1Threads) {
+        const uint4 v = __ldg(src + i);
+        const uint32_t w4v[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; j++) mx = max(mx, max(w4v[j] & 0x7FFFu, (w4v[j] >> 16) & 0x7FFFu));
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+    if (lane == 0) flags[2 + warp] = (int)mx;
+    __syncthreads();
+    for (int i = 0; i < kM1Warps; i++) mx = max(mx, (uint32_t)flags[2 + i]);
+    const int emax = (int)((mx >> 7) & 0xFFu);
+    sigma = (mx == 0) ? 0 : max(emax, 1) - 127 - 14;
+    bool bad = mx >= 0x7F80u;   // NaN / Inf: binary32 path
+    for (int i = threadIdx.x; i < nvec; i += kM1Threads) {
+        const int sc = i >> 4, q = i & 15;
+        const uint4 val = __ldg(src + i);
+        const uint32_t in[4] = {val.x, val.y, val.z, val.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const float x0 = bf16_lo(in[j]), x1 = bf16_hi(in[j]);
+            const __half2 h = __floats2half2_rn(mul_pow2(x0, -sigma), mul_pow2(x1, -sigma));
+            const float2 back = __half22float2(h);
+            bad |= (mul_pow2(back.x, sigma) != x0) | (mul_pow2(back.y, sigma) != x1);
+            o[j] = *reinterpret_cast<const uint32_t *>(&h);
+        }
+        uint16_t *row = xs + (size_t)sc * kM1ScStride;
+        *reinterpret_cast<uint4 *>(row + ((q & 3) * 4 + (q >> 2)) * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+        if (q == 0) *reinterpret_cast<uint4 *>(row + 128) = make_uint4(0, 0, 0, 0);
+    }
+    if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) atomicOr(&flags[1], 1);
+}
 
 // Super-chunks [b, e) of tile j for warp w: the share of warp (w + j) mod 16.
 __device__ __forceinline__ void m1_share(int w, int j, int SC, int &b, int &e) {
@@ -171,16 +221,11 @@ __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, 
     const float gs = __ldg(a.gscale);
     pdl_wait_prior_grid();   // x (and y, which the previous kernel may read) belong to it
 
-    // x slice -> shared memory, then f16 with one power of two, permuted per super-chunk
-    {
-        const uint4 *src = reinterpret_cast<const uint4 *>(a.x + k0);
-        uint4 *dst = reinterpret_cast<uint4 *>(xs);
-        for (int i = threadIdx.x; i < kcs / 8; i += kM1Threads) dst[i] = __ldg(src + i);
-    }
-    __syncthreads();
+    // x slice -> f16 with one power of two, in the B-operand layout
+    __syncthreads();   // flags[1] is cleared
     int sigma;
     uint32_t mx;
-    convert_x_f16<false, kM1Warps>(xs, a.xstride, 1, kcs, warp, lane, flags, sigma, mx);
+    m1_convert_x(a.x + k0, xs, kcs, warp, lane, flags, sigma, mx);
     __syncthreads();
     const bool fast = flags[1] == 0;
     // binary32 path: partial sums in units of x * 2^fold
@@ -191,13 +236,14 @@ __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, 
     // MMA operands.  Lane (g, t) holds rows g, g+8 of the codes of k = 32t .. 32t+31
     // (blocks 2t, 2t+1) and B column g.  Column g is block g: it is nonzero only for
     // the k of lanes t = g/2, and only in the MMAs of block g (the first four MMAs
-    // for even g, the last four for odd g).  So the 8 lanes with g/2 == t load x,
-    // two 16-byte pieces each, and the rest feed zeros.
+    // for even g, the last four for odd g).  So lane (g, t) takes its B pieces
+    // j = 0..3 (x of k = 32t + 8j .. +7) from x' when g/2 == t and j/2 == g%2,
+    // and from the super-chunk's eight zeros otherwise: four loads by address.
     const bool xact = (g >> 1) == t4;
     const bool odd = (g & 1) != 0;
-    // pieces j = 2*odd + {0, 1}; the order (odd lanes j = 3 first) keeps the 8
-    // active lanes of each load on distinct banks
-    const int xoffA = 32 * (odd ? 3 : 0) + 8 * t4, xoffB = 32 * (odd ? 2 : 1) + 8 * t4;
+    int xoff[4];
+#pragma unroll
+    for (int j = 0; j < 4; j++) xoff[j] = (xact && (j >> 1) == (odd ? 1 : 0)) ? 32 * j + 8 * t4 : 128;
 
     int cur = -1;                      // tile being accumulated
     float accA = 0.0f, accB = 0.0f;    // rows g, g+8 (fast) / row lane/2 (binary32)
@@ -229,15 +275,12 @@ __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, 
                 if (cur >= 0) flush();
                 cur = b.jt[d];
             }
-            uint4 xa = make_uint4(0, 0, 0, 0), xb = xa;
-            if (xact) {
-                const uint16_t *xp = xs + b.st[d] * 128;
-                xa = *reinterpret_cast<const uint4 *>(xp + xoffA);
-                xb = *reinterpret_cast<const uint4 *>(xp + xoffB);
-            }
             // B pieces of MMA pairs j = 0..3 (x of k = 32t + 8j .. +7, or zero)
-            const uint4 z = make_uint4(0, 0, 0, 0);
-            const uint4 b0 = odd ? z : xa, b1 = odd ? z : xb, b2 = odd ? xb : z, b3 = odd ? xa : z;
+            const uint16_t *xp = xs + b.st[d] * kM1ScStride;
+            const uint4 b0 = *reinterpret_cast<const uint4 *>(xp + xoff[0]);
+            const uint4 b1 = *reinterpret_cast<const uint4 *>(xp + xoff[1]);
+            const uint4 b2 = *reinterpret_cast<const uint4 *>(xp + xoff[2]);
+            const uint4 b3 = *reinterpret_cast<const uint4 *>(xp + xoff[3]);
             uint32_t h0[16], h1[16];
             decode_codes32(b.c0[d], h0);
             decode_codes32(b.c1[d], h1);

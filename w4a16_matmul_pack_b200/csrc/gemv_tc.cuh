@@ -138,7 +138,9 @@ __device__ __forceinline__ void decode_row32(uint4 c, uint32_t s2, uint32_t (&h)
     const uint32_t shi = __byte_perm(sc, 0, 0x3232); // (s_hi, s_hi)
     const uint32_t w[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-    for (int i = 0; i < 16; i++) h[i] = hmul2_u32(e2m1x2_to_f16x2(w[i >> 2] >> (8 * (i & 3))), i < 8 ? slo : shi);
+    for (int q = 0; q < 4; q++) e2m1x8_to_f16x2(w[q], h + 4 * q);
+#pragma unroll
+    for (int i = 0; i < 16; i++) h[i] = hmul2_u32(h[i], i < 8 ? slo : shi);
 }
 
 // One ROCmFP4 block (32 weights at shared-memory byte address A, any byte

@@ -96,7 +96,7 @@ w4_status plan_gemv_m1(int K, int N, GemvTcPlan &p, int force_grid, const Device
         p.grid = std::max(p.grid, (T + kM1MaxTiles - 1) / kM1MaxTiles);
     }
     p.red_tiles = (T + p.grid - 1) / p.grid;
-    p.xstride = p.kc + 32;
+    p.xstride = (p.kc / 128) * kM1ScStride;
     p.KP = p.kc;
     p.NS = 0;
     p.tile_bytes = 0;
