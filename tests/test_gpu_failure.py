@@ -1,8 +1,11 @@
 """Failure detection on the GPU, without a fault: with a wait limit short enough
-that the kernels' first waits expire, every call records W4_ERR_TIMEOUT in the
-sticky device word and returns (each CTA still waits for the copies and MMAs it
-had issued before it exits).  With the default limit restored, the next calls
-on the same context are correct against the oracle and record nothing.
+that the kernels' first waits expire, every call of a kernel that waits on
+mbarriers (the TMA-staged ROCmFP4 GEMV, the prefill GEMM) records
+W4_ERR_TIMEOUT in the sticky device word and returns (each CTA still waits for
+the copies and MMAs it had issued before it exits).  With the default limit
+restored, the next calls on the same context are correct against the oracle and
+record nothing.  The NVFP4 GEMVs wait on no mbarrier and must finish, correct,
+under the same limit.
 
 Also here: the library called from two host threads at once on one device (the
 per-device launch state is shared under a lock) gives the single-thread bits."""
@@ -50,14 +53,21 @@ def expire_then_recover(run, check):
     check(out)
 
 
-@pytest.mark.parametrize("M", [4, 16])
-def test_gemv_wait_expiry(default_limit_after, M):
+@pytest.mark.parametrize("M", [4, 9, 16])
+def test_nvfp4_gemv_kernels_do_not_wait(default_limit_after, M):
+    """The NVFP4 GEMVs for several tokens load their operands directly as the
+    one-token kernels do and wait on no mbarrier: with a 1 ns limit they still
+    finish, correct, and record nothing (K = 9728 also exercises the split-K
+    partials and their finalize)."""
     K, N = 9728, 1024
     pw, wh = nvfp4(K, N, 500 + M)
     x = I.activations(M, K, 501)
-    xd = x.cuda()
     yr, ar = O.matmul(x, wh)
-    expire_then_recover(lambda: W4.w4a16_gemv(pw, xd), lambda y: assert_within_tolerance(np_of(y), yr, ar))
+    W4.set_wait_limit(1)
+    y = W4.w4a16_gemv(pw, x.cuda())
+    torch.cuda.synchronize()
+    assert W4.w4_device_error(clear=True) == 0
+    assert_within_tolerance(np_of(y), yr, ar)
 
 
 def test_one_token_kernels_do_not_wait(default_limit_after):

@@ -156,20 +156,22 @@ struct M1Items {
     }
 };
 
-// kM1Depth items of one warp in registers: tile (-1: none), super-chunk, the
-// lane's code bytes of rows g and g+8, their scale bytes.
+// D items of one warp in registers: tile (-1: none), super-chunk, the lane's
+// code bytes of rows g and g+8, their scale bytes.
+template <int D = kM1Depth>
 struct M1Batch {
-    int jt[kM1Depth], st[kM1Depth];
-    uint4 c0[kM1Depth], c1[kM1Depth];
-    uint32_t s0[kM1Depth], s1[kM1Depth];
+    int jt[D], st[D];
+    uint4 c0[D], c1[D];
+    uint32_t s0[D], s1[D];
 };
 
-// Issue the loads of the warp's next kM1Depth items (streaming: read once).
-__device__ __forceinline__ void m1_load(M1Batch &b, M1Items &it, const GemvTcArgs &a, int warp, int nt, int SC,
+// Issue the loads of the warp's next D items (streaming: read once).
+template <int D>
+__device__ __forceinline__ void m1_load(M1Batch<D> &b, M1Items &it, const GemvTcArgs &a, int warp, int nt, int SC,
                                         int t0, int k0, int g, int t4) {
     const size_t RB = (size_t)a.K / 2, SB = (size_t)a.K / 16;
 #pragma unroll
-    for (int d = 0; d < kM1Depth; d++) {
+    for (int d = 0; d < D; d++) {
         b.jt[d] = it.j < nt ? it.j : -1;
         b.st[d] = it.s;
         b.c0[d] = b.c1[d] = make_uint4(0, 0, 0, 0);
@@ -216,7 +218,7 @@ __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, 
     // warp's items is loaded before waiting for it (and before x is ready).
     M1Items it;
     it.first(warp, nt, SC);
-    M1Batch bA, bB;
+    M1Batch<> bA, bB;
     m1_load(bA, it, a, warp, nt, SC, t0, k0, g, t4);
     const float gs = __ldg(a.gscale);
     pdl_wait_prior_grid();   // x (and y, which the previous kernel may read) belong to it
@@ -267,7 +269,7 @@ __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, 
         accB = 0.0f;
     };
     // the math of one batch (fast path)
-    auto compute = [&](const M1Batch &b) {
+    auto compute = [&](const M1Batch<> &b) {
 #pragma unroll
         for (int d = 0; d < kM1Depth; d++) {
             if (b.jt[d] < 0) break;

@@ -1,0 +1,251 @@
+// gemv_skinny.cuh -- NVFP4 GEMV for M = 2..16 tokens (skinny GEMM: decode of a
+// small batch, the speculative-verify step): y[m][n] = g * sum_k x[m][k] *
+// e2m1[n][k] * scale[n][k/16] ("EdgeRock-4B-NVFP4" card, intro; the batched
+// decode and n-gram verification of the "Nanbeige4.2-3B-NVFP4A16" card,
+// Serving).
+//
+// The structure of the one-token kernel (gemv_m1.cuh): sixteen warps, whole
+// 16-row tiles per CTA, every warp a rotating share of each tile's 128-k
+// super-chunks, its MMA operands loaded straight from HBM into registers.
+// With several tokens the B columns are the tokens, so the block scale is
+// applied to the decoded codes first (E2M1 * E4M3 has at most 6 significant
+// bits: exact in f16, one HMUL2 per pair), and the MMAs accumulate a tile's
+// super-chunks directly in their C operand.  x of the K slice is staged once
+// per CTA as f16 rows (one power of two for all of x, exact whenever every
+// nonzero |x'| >= 2^-17; otherwise the CTA computes in binary32 from global
+// memory), padded by 16 bytes per row so that the eight tokens of an n-tile
+// read distinct banks; token rows past M are zeros.  Per-warp partial sums of
+// the CTA's tiles are added in warp order (no atomics).  A K too long for the
+// x slice runs in slices whose partials gemv_finalize_kernel adds.
+#pragma once
+
+#include "gemv_m1.cuh"
+
+namespace w4 {
+
+// x' of the slice: NT*8 token rows of xstride halves (slice length + 8).
+// Partial sums: [red_tiles][kM1Warps][16][M] float.  Flags: [2 + kM1Warps] int.
+__host__ __device__ __forceinline__ M1Layout skinny_layout(int M, int xstride, int red_tiles) {
+    const int R = (M + 7) / 8 * 8;
+    M1Layout L;
+    L.red = ((size_t)R * xstride * 2 + 127) & ~(size_t)127;
+    L.flags = L.red + (size_t)red_tiles * kM1Warps * kTcRows * M * 4;
+    L.total = L.flags + 4 * (2 + kM1Warps);
+    return L;
+}
+
+// x[M][K] slice (BF16, global) -> x' rows (f16, x * 2^-sigma), rows M .. R-1 zero.
+template <int M>
+__device__ __forceinline__ void skinny_convert_x(const uint16_t *x, int K, int k0, int kcs, uint16_t *xs, int XS,
+                                                 int warp, int lane, int *flags, int &sigma, uint32_t &mx) {
+    constexpr int R = (M + 7) / 8 * 8;
+    const int nvec = kcs / 8;
+    mx = 0;
+    for (int i = threadIdx.x; i < M * nvec; i += kM1Threads) {
+        const int m = i / nvec, v = i % nvec;
+        const uint4 val = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)m * K + k0) + v);
+        const uint32_t w4v[4] = {val.x, val.y, val.z, val.w};
+#pragma unroll
+        for (int j = 0; j < 4; j++) mx = max(mx, max(w4v[j] & 0x7FFFu, (w4v[j] >> 16) & 0x7FFFu));
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+    if (lane == 0) flags[2 + warp] = (int)mx;
+    __syncthreads();
+    for (int i = 0; i < kM1Warps; i++) mx = max(mx, (uint32_t)flags[2 + i]);
+    const int emax = (int)((mx >> 7) & 0xFFu);
+    sigma = (mx == 0) ? 0 : max(emax, 1) - 127 - 14;
+    bool bad = mx >= 0x7F80u;   // NaN / Inf: binary32 path
+    for (int i = threadIdx.x; i < R * nvec; i += kM1Threads) {
+        const int m = i / nvec, v = i % nvec;
+        uint4 out = make_uint4(0, 0, 0, 0);
+        if (m < M) {
+            const uint4 val = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)m * K + k0) + v);
+            const uint32_t in[4] = {val.x, val.y, val.z, val.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const float x0 = bf16_lo(in[j]), x1 = bf16_hi(in[j]);
+                const __half2 h = __floats2half2_rn(mul_pow2(x0, -sigma), mul_pow2(x1, -sigma));
+                const float2 back = __half22float2(h);
+                bad |= (mul_pow2(back.x, sigma) != x0) | (mul_pow2(back.y, sigma) != x1);
+                o[j] = *reinterpret_cast<const uint32_t *>(&h);
+            }
+            out = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        *reinterpret_cast<uint4 *>(xs + (size_t)m * XS + v * 8) = out;
+    }
+    if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) atomicOr(&flags[1], 1);
+}
+
+// The binary32 path of one CTA (x that could not be rescaled exactly into
+// f16): lane l takes row l/2 of each tile and 64 k of each of the warp's
+// super-chunks, every token; writes the warp's partial sums of each tile to
+// red.  Kept out of line so that its registers do not constrain the fast path.
+template <int M>
+__device__ __noinline__ void skinny_fallback(const GemvTcArgs &a, float *red, int warp, int lane, int nt, int SC,
+                                             int t0, int k0, float gs, int fold, int sref) {
+    const int K = a.K, N = a.N;
+    const size_t RB = (size_t)K / 2, SB = (size_t)K / 16;
+    const int row = lane >> 1, half = lane & 1;
+    float facc[M];
+#pragma unroll
+    for (int m = 0; m < M; m++) facc[m] = 0.0f;
+    int cur = -1;
+    auto flush = [&]() {
+        float *rb = red + ((size_t)cur * kM1Warps + warp) * kTcRows * M;
+#pragma unroll
+        for (int m = 0; m < M; m++) {
+            facc[m] += __shfl_xor_sync(0xFFFFFFFFu, facc[m], 1);
+            if ((lane & 1) == 0) rb[(lane >> 1) * M + m] = scale_out(facc[m], gs, sref);
+            facc[m] = 0.0f;
+        }
+    };
+    M1Items it;
+    for (it.first(warp, nt, SC); it.j < nt; it.next(warp, nt, SC)) {
+        if (it.j != cur) {
+            if (cur >= 0) flush();
+            cur = it.j;
+        }
+        const long long r = (long long)(t0 + it.j) * kTcRows + row;
+        if (r >= N) continue;
+        const int kb = k0 + it.s * 128 + 64 * half;
+        const uint8_t *cp = a.codes + r * RB + kb / 2;
+        const uint8_t *sp = a.scales + r * SB + kb / 16;
+        for (int q = 0; q < 4; q++) {
+            const uint2 c = __ldg(reinterpret_cast<const uint2 *>(cp + 8 * q));
+            float2 w[8];
+            decode_nvfp4(c, w);
+            scale_pairs(w, fold);
+            const float sv = e4m3_to_f32(__ldg(sp + q));
+#pragma unroll
+            for (int m = 0; m < M; m++) {
+                float2 xv[8];
+                load_x16(a.x + (size_t)m * K + kb + 16 * q, xv);
+                facc[m] = dot_group<8>(w, xv, sv, facc[m]);
+            }
+        }
+    }
+    if (cur >= 0) flush();
+}
+
+template <int M>
+__global__ void __launch_bounds__(kM1Threads, 1) gemv_nvfp4_skinny_kernel(const GemvTcArgs a) {
+    constexpr int NT = (M + 7) / 8;   // n-tiles of 8 tokens
+    constexpr int D = M <= 8 ? 2 : 1; // super-chunks per batch (two batches in flight)
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int K = a.K, N = a.N, kc = a.kc, XS = a.xstride;
+    const int slice = blockIdx.y, nslices = gridDim.y;
+    const int k0 = slice * kc, kcs = min(kc, K - k0);
+    const int SC = kcs / 128;
+    const M1Layout L = skinny_layout(M, XS, a.red_tiles);
+    uint16_t *xs = reinterpret_cast<uint16_t *>(smem);
+    float *red = reinterpret_cast<float *>(smem + L.red);   // [tile][warp][16][M]
+    int *flags = reinterpret_cast<int *>(smem + L.flags);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int T = (N + kTcRows - 1) / kTcRows;
+    const int cta = blockIdx.x, ncta = gridDim.x;
+    const int t0 = (int)((long long)cta * T / ncta), t1 = (int)((long long)(cta + 1) * T / ncta);
+    const int nt = t1 - t0;
+    const int g = lane >> 2, t4 = lane & 3;
+
+    if (threadIdx.x == 0) flags[1] = 0;
+    pdl_allow_dependents();
+    // the first batch of this warp's weights is loaded before waiting for the
+    // previous kernel (and before x is ready)
+    M1Items it;
+    it.first(warp, nt, SC);
+    M1Batch<D> bA, bB;
+    m1_load(bA, it, a, warp, nt, SC, t0, k0, g, t4);
+    const float gs = __ldg(a.gscale);
+    pdl_wait_prior_grid();
+    __syncthreads();   // flags[1] is cleared
+    int sigma;
+    uint32_t mx;
+    skinny_convert_x<M>(a.x, K, k0, kcs, xs, XS, warp, lane, flags, sigma, mx);
+    __syncthreads();
+    const bool fast = flags[1] == 0;
+    const int fold = fast ? 0 : fallback_fold(gs, mx >= ((127u + 100u) << 7));   // largest |x| >= 2^100
+    const int sref = fast ? sigma : -fold;
+
+    int cur = -1;                       // tile being accumulated
+    float acc[NT][4];                   // MMA C fragments (rows g, g+8 x tokens 8nt + 2t, +1)
+#pragma unroll
+    for (int q = 0; q < NT; q++) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.0f;
+    // this warp's partial sums of tile cur -> shared memory
+    auto flush = [&]() {
+        float *rb = red + ((size_t)cur * kM1Warps + warp) * kTcRows * M;
+#pragma unroll
+        for (int q = 0; q < NT; q++) {
+#pragma unroll
+            for (int e = 0; e < 4; e++) {
+                const int row = g + 8 * (e >> 1), m = 8 * q + 2 * t4 + (e & 1);
+                if (m < M) rb[row * M + m] = scale_out(acc[q][e], gs, sref);
+                acc[q][e] = 0.0f;
+            }
+        }
+    };
+    // the math of one batch (fast path)
+    auto compute = [&](const M1Batch<D> &b) {
+#pragma unroll
+        for (int d = 0; d < D; d++) {
+            if (b.jt[d] < 0) break;
+            if (b.jt[d] != cur) {
+                if (cur >= 0) flush();
+                cur = b.jt[d];
+            }
+            uint32_t h0[16], h1[16];
+            decode_row32(b.c0[d], b.s0[d], h0);   // e2m1 * scale, f16, exact
+            decode_row32(b.c1[d], b.s1[d], h1);
+#pragma unroll
+            for (int q = 0; q < NT; q++) {
+                // x of token 8q + g, k = 32t .. 32t+31 of the super-chunk
+                const uint4 *xp = reinterpret_cast<const uint4 *>(xs + (size_t)(8 * q + g) * XS + b.st[d] * 128 + 32 * t4);
+                uint32_t xv[16];
+#pragma unroll
+                for (int v = 0; v < 4; v++) {
+                    const uint4 u = xp[v];
+                    xv[4 * v] = u.x, xv[4 * v + 1] = u.y, xv[4 * v + 2] = u.z, xv[4 * v + 3] = u.w;
+                }
+#pragma unroll
+                for (int j = 0; j < 8; j++)
+                    mma_f16_16816(acc[q], h0[2 * j], h1[2 * j], h0[2 * j + 1], h1[2 * j + 1], xv[2 * j], xv[2 * j + 1]);
+            }
+        }
+    };
+    if (fast) {
+        // software pipeline: the next batch's loads are in flight while this one is multiplied
+        for (;;) {
+            if (bA.jt[0] < 0) break;
+            m1_load(bB, it, a, warp, nt, SC, t0, k0, g, t4);
+            compute(bA);
+            if (bB.jt[0] < 0) break;
+            m1_load(bA, it, a, warp, nt, SC, t0, k0, g, t4);
+            compute(bB);
+        }
+        if (cur >= 0) flush();
+    } else {
+        skinny_fallback<M>(a, red, warp, lane, nt, SC, t0, k0, gs, fold, sref);
+    }
+    __syncthreads();
+
+    // rows of the CTA's tiles: the partials of the warps with a share of the tile, in warp order
+    for (int i = threadIdx.x; i < nt * kTcRows * M; i += kM1Threads) {
+        const int m = i % M, r = (i / M) % kTcRows, j = i / (M * kTcRows);
+        const long long n = (long long)(t0 + j) * kTcRows + r;
+        if (n >= N) continue;
+        float s = 0.0f;
+        for (int w = 0; w < kM1Warps; w++) {
+            int b, e;
+            m1_share(w, j, SC, b, e);
+            if (b < e) s += red[(((size_t)j * kM1Warps + w) * kTcRows + r) * M + m];
+        }
+        if (nslices == 1)
+            a.y[(size_t)m * N + n] = s;
+        else
+            a.partial[((size_t)slice * M + m) * N + n] = s;
+    }
+}
+
+}  // namespace w4

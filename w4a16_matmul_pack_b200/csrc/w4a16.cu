@@ -10,6 +10,7 @@
 #include "gemv.cuh"
 #include "gemv_tc.cuh"
 #include "gemv_m1.cuh"
+#include "gemv_skinny.cuh"
 #include "gemm.cuh"
 
 using namespace w4;
@@ -108,10 +109,47 @@ w4_status plan_gemv_m1(int K, int N, GemvTcPlan &p, int force_grid, const Device
     return W4_OK;
 }
 
+// NVFP4, M = 2..16 (gemv_skinny.cuh): K slices whose x' (rows padded to 8
+// tokens) fits kSkinnyXBytes; short problems are also split along K as for one
+// token; tiles per CTA as many as the partial-sum buffer holds.
+constexpr size_t kSkinnyXBytes = 96 * 1024;
+
+w4_status plan_gemv_skinny(int K, int N, int M, GemvTcPlan &p, const DeviceInfo &d) {
+    p.M = M;
+    const int R = (M + 7) / 8 * 8;
+    const int T = (N + kTcRows - 1) / kTcRows;
+    const int kmax = std::max(256, (int)((kSkinnyXBytes / (2 * (size_t)R) - 8) / 256 * 256));
+    int S = (K + kmax - 1) / kmax;
+    if (T < d.sms / 2) S = std::max(S, std::min(d.sms / T, K / 2048));
+    S = std::max(S, 1);
+    p.kc = ((K + S - 1) / S + 255) / 256 * 256;
+    p.S = (K + p.kc - 1) / p.kc;
+    p.xstride = p.kc + 8;
+    const size_t xbytes = ((size_t)R * p.xstride * 2 + 127) & ~(size_t)127;
+    const size_t per_tile = (size_t)kM1Warps * kTcRows * M * 4;
+    const size_t room = (size_t)d.smem_optin > xbytes + 4 * (2 + kM1Warps)
+                            ? (size_t)d.smem_optin - xbytes - 4 * (2 + kM1Warps) : 0;
+    const int red_max = (int)(room / per_tile);
+    if (red_max < 1) return W4_ERR_UNSUPPORTED;
+    p.grid = std::min(T, std::max(1, d.sms / p.S));
+    p.grid = std::max(p.grid, (T + red_max - 1) / red_max);
+    p.red_tiles = (T + p.grid - 1) / p.grid;
+    p.KP = p.kc;
+    p.NS = 0;
+    p.tile_bytes = 0;
+    p.rows_mode = 1;
+    p.tiles_per_cta = p.red_tiles;
+    p.smem = skinny_layout(M, p.xstride, p.red_tiles).total;
+    if (p.smem > (size_t)d.smem_optin) return W4_ERR_UNSUPPORTED;
+    p.ws_bytes = p.S > 1 ? (size_t)p.S * M * N * sizeof(float) : 0;
+    return W4_OK;
+}
+
 w4_status plan_gemv_tc(int fmt, int K, int N, int M, bool pdl, GemvTcPlan &p, int force_grid = 0) {
     DeviceInfo d;
     if (device_info(d) != W4_OK) return W4_ERR_CUDA;
     if (fmt == W4_FMT_NVFP4 && M == 1) return plan_gemv_m1(K, N, p, force_grid, d);
+    if (fmt == W4_FMT_NVFP4 && force_grid <= 0) return plan_gemv_skinny(K, N, M, p, d);
     p.M = M;
     const bool nv = fmt == W4_FMT_NVFP4;
     const int unit = k_unit(fmt);
@@ -192,7 +230,7 @@ w4_status gemv_tc_setup(const w4_weights *w, const void *x, float *y, void *ws, 
     // one token: codes as [N][K/256][16 x 8 bytes], 3-D box of 16 rows x KP/256
     // lines of 128 bytes, 128-byte swizzle (the consumers' chunk XOR)
     const bool nv = w->fmt == W4_FMT_NVFP4;
-    const bool direct = nv && p.M == 1;   // the one-token kernel loads its operands directly
+    const bool direct = nv;   // the NVFP4 kernels load their operands directly
     // ROCmFP4: blocks as 8-byte elements, a box of 16 rows x KP/32 blocks, no scales map
     const int bb = nv ? 0 : block_bytes(w->fmt);
     const cuuint64_t rdims[2] = {(cuuint64_t)stage_row_bytes(w->fmt, bb, K) / 8, (cuuint64_t)N};
@@ -245,9 +283,10 @@ w4_status launch_gemv_tc_m(const w4_weights *w, const void *x, float *y, void *w
                            cudaStream_t st) {
     // one NVFP4 token: block scales applied after the MMA, operands loaded
     // directly (gemv_m1.cuh); otherwise TMA-staged tiles (gemv_tc.cuh)
-    constexpr bool direct = M == 1 && FMT == W4_FMT_NVFP4;
-    const void *kern = direct ? reinterpret_cast<const void *>(gemv_nvfp4_m1_kernel)
-                              : reinterpret_cast<const void *>(gemv_tc_kernel<FMT, M>);
+    constexpr bool direct = FMT == W4_FMT_NVFP4;
+    const void *kern = !direct ? reinterpret_cast<const void *>(gemv_tc_kernel<FMT, M>)
+                               : (M == 1 ? reinterpret_cast<const void *>(gemv_nvfp4_m1_kernel)
+                                         : reinterpret_cast<const void *>(gemv_nvfp4_skinny_kernel<M>));
     if (!set_smem_limit(kern, p.smem)) return W4_ERR_CUDA;
     const int N = w->N;
     CUtensorMap cmap, smap;
@@ -265,8 +304,10 @@ w4_status launch_gemv_tc_m(const w4_weights *w, const void *x, float *y, void *w
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
     cudaError_t e;
-    if constexpr (direct)
+    if constexpr (direct && M == 1)
         e = cudaLaunchKernelEx(&cfg, gemv_nvfp4_m1_kernel, a);
+    else if constexpr (direct)
+        e = cudaLaunchKernelEx(&cfg, gemv_nvfp4_skinny_kernel<M>, a);
     else
         e = cudaLaunchKernelEx(&cfg, gemv_tc_kernel<FMT, M>, cmap, smap, a);
     if (e != cudaSuccess) return W4_ERR_CUDA;
