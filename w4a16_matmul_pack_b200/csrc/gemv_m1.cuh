@@ -87,8 +87,8 @@ constexpr int kM1ScStride = 136;   // halves per super-chunk
 
 // x slice (BF16, global) -> x' = x * 2^-sigma as f16 in that layout, with one
 // power of two for the slice (its largest |x'| in [2^14, 2^15)); flags[1] is
-// set when some x does not convert exactly (a nonzero |x'| below 2^-17 scaled
-// back differs, Inf / NaN).  All kM1Warps warps take part; flags[2 ..] is
+// set when some x may not convert exactly (a nonzero |x'| below 2^-17: see
+// x_pair_f16) or is Inf / NaN.  All kM1Warps warps take part; flags[2 ..] is
 // scratch.  mx: the largest |x| (BF16 bits).
 __device__ __forceinline__ void m1_convert_x(const uint16_t *xg, uint16_t *xs, int kcs, int warp, int lane,
                                              int *flags, int &sigma, uint32_t &mx) {
@@ -109,19 +109,12 @@ __device__ __forceinline__ void m1_convert_x(const uint16_t *xg, uint16_t *xs, i
     const int emax = (int)((mx >> 7) & 0xFFu);
     sigma = (mx == 0) ? 0 : max(emax, 1) - 127 - 14;
     bool bad = mx >= 0x7F80u;   // NaN / Inf: binary32 path
+    const XScale xsc = make_xscale(sigma);
     for (int i = threadIdx.x; i < nvec; i += kM1Threads) {
         const int sc = i >> 4, q = i & 15;
         const uint4 val = __ldg(src + i);
-        const uint32_t in[4] = {val.x, val.y, val.z, val.w};
-        uint32_t o[4];
-#pragma unroll
-        for (int j = 0; j < 4; j++) {
-            const float x0 = bf16_lo(in[j]), x1 = bf16_hi(in[j]);
-            const __half2 h = __floats2half2_rn(mul_pow2(x0, -sigma), mul_pow2(x1, -sigma));
-            const float2 back = __half22float2(h);
-            bad |= (mul_pow2(back.x, sigma) != x0) | (mul_pow2(back.y, sigma) != x1);
-            o[j] = *reinterpret_cast<const uint32_t *>(&h);
-        }
+        const uint32_t o[4] = {x_pair_f16(val.x, xsc, bad), x_pair_f16(val.y, xsc, bad), x_pair_f16(val.z, xsc, bad),
+                               x_pair_f16(val.w, xsc, bad)};
         uint16_t *row = xs + (size_t)sc * kM1ScStride;
         *reinterpret_cast<uint4 *>(row + ((q & 3) * 4 + (q >> 2)) * 8) = make_uint4(o[0], o[1], o[2], o[3]);
         if (q == 0) *reinterpret_cast<uint4 *>(row + 128) = make_uint4(0, 0, 0, 0);

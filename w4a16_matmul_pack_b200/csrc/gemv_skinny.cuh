@@ -56,22 +56,14 @@ __device__ __forceinline__ void skinny_convert_x(const uint16_t *x, int K, int k
     const int emax = (int)((mx >> 7) & 0xFFu);
     sigma = (mx == 0) ? 0 : max(emax, 1) - 127 - 14;
     bool bad = mx >= 0x7F80u;   // NaN / Inf: binary32 path
+    const XScale xsc = make_xscale(sigma);
     for (int i = threadIdx.x; i < R * nvec; i += kM1Threads) {
         const int m = i / nvec, v = i % nvec;
         uint4 out = make_uint4(0, 0, 0, 0);
         if (m < M) {
             const uint4 val = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)m * K + k0) + v);
-            const uint32_t in[4] = {val.x, val.y, val.z, val.w};
-            uint32_t o[4];
-#pragma unroll
-            for (int j = 0; j < 4; j++) {
-                const float x0 = bf16_lo(in[j]), x1 = bf16_hi(in[j]);
-                const __half2 h = __floats2half2_rn(mul_pow2(x0, -sigma), mul_pow2(x1, -sigma));
-                const float2 back = __half22float2(h);
-                bad |= (mul_pow2(back.x, sigma) != x0) | (mul_pow2(back.y, sigma) != x1);
-                o[j] = *reinterpret_cast<const uint32_t *>(&h);
-            }
-            out = make_uint4(o[0], o[1], o[2], o[3]);
+            out = make_uint4(x_pair_f16(val.x, xsc, bad), x_pair_f16(val.y, xsc, bad), x_pair_f16(val.z, xsc, bad),
+                             x_pair_f16(val.w, xsc, bad));
         }
         *reinterpret_cast<uint4 *>(xs + (size_t)m * XS + v * 8) = out;
     }

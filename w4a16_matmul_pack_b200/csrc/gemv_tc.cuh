@@ -102,6 +102,40 @@ __device__ __forceinline__ void scale_pairs(float2 (&w)[NP], int e) {
     for (int p = 0; p < NP; p++) w[p] = __fmul2_rn(w[p], make_float2(f, f));
 }
 
+// x * 2^-sigma for the one-power-of-two f16 staging of x: sigma puts the
+// largest |x'| in [2^14, 2^15), so x' never overflows f16, and a BF16 value
+// (8 significant bits) converts exactly unless it is nonzero and below 2^-17
+// after scaling (then its last bit may fall under the f16 subnormal spacing).
+// thr = the BF16 magnitude bits of 2^(sigma - 17): a nonzero |x| whose bits are
+// below thr is flagged (conservative: some such values would convert exactly).
+struct XScale {
+    float p;       // 2^-sigma when that is a normal binary32 value
+    bool one;      // one multiply suffices
+    int sigma;
+    uint32_t thr;
+};
+
+__device__ __forceinline__ XScale make_xscale(int sigma) {
+    XScale x;
+    x.sigma = sigma;
+    x.one = sigma >= -126 && sigma <= 126;
+    x.p = x.one ? __int_as_float((127 - sigma) << 23) : 0.0f;
+    const int e = sigma - 17 + 127;   // BF16 biased exponent of 2^(sigma - 17)
+    x.thr = e >= 1 ? (uint32_t)e << 7 : (e + 6 >= 0 ? 1u << (e + 6) : 0u);
+    return x;
+}
+
+// Two BF16 values (one 32-bit word) -> f16x2 of x * 2^-sigma; bad |= not exact.
+__device__ __forceinline__ uint32_t x_pair_f16(uint32_t w, const XScale &xs, bool &bad) {
+    const float x0 = bf16_lo(w), x1 = bf16_hi(w);
+    const float a0 = xs.one ? x0 * xs.p : mul_pow2(x0, -xs.sigma);
+    const float a1 = xs.one ? x1 * xs.p : mul_pow2(x1, -xs.sigma);
+    const __half2 h = __floats2half2_rn(a0, a1);
+    const uint32_t m0 = w & 0x7FFFu, m1 = (w >> 16) & 0x7FFFu;
+    bad |= (m0 != 0u && m0 < xs.thr) | (m1 != 0u && m1 < xs.thr);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
 constexpr int kTcRows = 16;                    // rows per tile (one MMA M)
 constexpr int kTcWarps = 8;                    // consumer warps, each a contiguous share of a tile's k
 constexpr int kTcParts = kTcWarps;
