@@ -341,15 +341,20 @@ __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, 
     __syncthreads();
 
     // rows of the CTA's tiles: the partials of the warps with a share of the tile, in warp order
+    const bool every = SC >= kM1Warps;   // every warp has a share of every tile
     for (int i = threadIdx.x; i < nt * kTcRows; i += kM1Threads) {
         const int j = i / kTcRows, r = i % kTcRows;
         const long long n = (long long)(t0 + j) * kTcRows + r;
         if (n >= N) continue;
         float s = 0.0f;
         for (int w = 0; w < kM1Warps; w++) {
-            int b, e;
-            m1_share(w, j, SC, b, e);
-            if (b < e) s += red[((size_t)j * kM1Warps + w) * kTcRows + r];
+            bool has = every;
+            if (!every) {
+                int b, e;
+                m1_share(w, j, SC, b, e);
+                has = b < e;
+            }
+            if (has) s += red[((size_t)j * kM1Warps + w) * kTcRows + r];
         }
         if (nslices == 1)
             a.y[n] = s;

@@ -13,9 +13,10 @@
 // super-chunks directly in their C operand.  x of the K slice is staged once
 // per CTA as f16 rows (one power of two for all of x, exact whenever every
 // nonzero |x'| >= 2^-17; otherwise the CTA computes in binary32 from global
-// memory), padded by 16 bytes per row so that the eight tokens of an n-tile
-// read distinct banks; token rows past M are zeros.  Per-warp partial sums of
-// the CTA's tiles are added in warp order (no atomics).  A K too long for the
+// memory); within a super-chunk the 16-byte pieces of the four lanes of a row
+// are interleaved and the rows lie 64 bytes apart modulo 128, so that the
+// loads of a warp fall on distinct banks.  Per-warp partial sums of the CTA's
+// tiles are added in warp order (no atomics).  A K too long for the
 // x slice runs in slices whose partials gemv_finalize_kernel adds.
 #pragma once
 
@@ -23,51 +24,104 @@
 
 namespace w4 {
 
-// x' of the slice: NT*8 token rows of xstride halves (slice length + 8).
-// Partial sums: [red_tiles][kM1Warps][16][M] float.  Flags: [2 + kM1Warps] int.
+// x' of the slice: NT*8 token rows of xstride halves (slice length + 32).
+// Partial sums: [red_tiles][kM1Warps][16][MP] float (MP = M rounded up to 4).
+// Flags: [2 + 2 * kM1Warps] int (the per-warp largest and smallest magnitudes of x).
+constexpr size_t kSkinnyXBytes = 96 * 1024;
+
+__host__ __device__ constexpr int skinny_pad(int M) { return (M + 3) / 4 * 4; }
+
+// Longest K slice whose x' fits kSkinnyXBytes (rows padded to 8 tokens).
+__host__ __device__ constexpr int skinny_kmax(int M) {
+    return (int)((kSkinnyXBytes / (2 * (size_t)((M + 7) / 8 * 8)) - 32) / 256 * 256);
+}
+
+// 16-byte pieces of an x slice that one thread converts, at most.
+__host__ __device__ constexpr int skinny_pieces(int M) {
+    return (M * (skinny_kmax(M) / 8) + kM1Threads - 1) / kM1Threads;
+}
+
 __host__ __device__ __forceinline__ M1Layout skinny_layout(int M, int xstride, int red_tiles) {
     const int R = (M + 7) / 8 * 8;
     M1Layout L;
     L.red = ((size_t)R * xstride * 2 + 127) & ~(size_t)127;
-    L.flags = L.red + (size_t)red_tiles * kM1Warps * kTcRows * M * 4;
-    L.total = L.flags + 4 * (2 + kM1Warps);
+    L.flags = L.red + (size_t)red_tiles * kM1Warps * kTcRows * skinny_pad(M) * 4;
+    L.total = L.flags + 4 * (2 + 2 * kM1Warps);
     return L;
 }
 
-// x[M][K] slice (BF16, global) -> x' rows (f16, x * 2^-sigma), rows M .. R-1 zero.
+// x[M][K] slice (BF16, global; SC super-chunks of 128 k from k0) -> x' rows
+// (f16, x * 2^-sigma).  Each thread holds its pieces in registers between the
+// two passes: the largest magnitude and the smallest nonzero one (two 16-bit
+// lanes at a time) decide sigma and whether the f16 copy is exact; only then
+// is it written.  Token rows M .. 8*NT-1 are left as they are: they only feed
+// MMA columns whose sums are never read.
 template <int M>
-__device__ __forceinline__ void skinny_convert_x(const uint16_t *x, int K, int k0, int kcs, uint16_t *xs, int XS,
-                                                 int warp, int lane, int *flags, int &sigma, uint32_t &mx) {
-    constexpr int R = (M + 7) / 8 * 8;
-    const int nvec = kcs / 8;
-    mx = 0;
-    for (int i = threadIdx.x; i < M * nvec; i += kM1Threads) {
-        const int m = i / nvec, v = i % nvec;
-        const uint4 val = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)m * K + k0) + v);
-        const uint32_t w4v[4] = {val.x, val.y, val.z, val.w};
+__device__ __forceinline__ void skinny_convert_x(const uint16_t *x, int K, int k0, int SC, uint16_t *xs, int XS,
+                                                 int warp, int lane, int *flags, int &sigma, bool &exact,
+                                                 uint32_t &mx) {
+    constexpr int V = skinny_pieces(M);
+    const int total = M * 16 * SC;
+    uint4 val[V];
+    uint32_t mx2 = 0u, mn2 = 0xFFFFFFFFu;   // per 16-bit lane: max |x|, min (|x| - 1) over |x| != 0
 #pragma unroll
-        for (int j = 0; j < 4; j++) mx = max(mx, max(w4v[j] & 0x7FFFu, (w4v[j] >> 16) & 0x7FFFu));
+    for (int u = 0; u < V; u++) {
+        const int i = threadIdx.x + u * kM1Threads;
+        if (i < total) {
+            const int q = i & 15, r = i >> 4, m = r % M, sc = r / M;
+            val[u] = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)m * K + k0 + sc * 128) + q);
+        }
     }
 #pragma unroll
-    for (int o = 16; o; o >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-    if (lane == 0) flags[2 + warp] = (int)mx;
+    for (int u = 0; u < V; u++) {
+        if (threadIdx.x + u * kM1Threads < total) {
+            const uint32_t w4v[4] = {val[u].x, val[u].y, val[u].z, val[u].w};
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const uint32_t mag = w4v[j] & 0x7FFF7FFFu;
+                mx2 = __vmaxu2(mx2, mag);
+                // |x| = 0 -> 0xFFFF, else |x| - 1 (no carry between the lanes: mag <= 0x7FFF)
+                mn2 = __vminu2(mn2, (mag + 0x7FFF7FFFu) ^ 0x80008000u);
+            }
+        }
+    }
+    mx = max(mx2 & 0xFFFFu, mx2 >> 16);
+    uint32_t mn = min(mn2 & 0xFFFFu, mn2 >> 16);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+        mn = min(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
+    }
+    if (lane == 0) flags[2 + warp] = (int)mx, flags[2 + kM1Warps + warp] = (int)mn;
     __syncthreads();
-    for (int i = 0; i < kM1Warps; i++) mx = max(mx, (uint32_t)flags[2 + i]);
+    for (int i = 0; i < kM1Warps; i++) {
+        mx = max(mx, (uint32_t)flags[2 + i]);
+        mn = min(mn, (uint32_t)flags[2 + kM1Warps + i]);
+    }
     const int emax = (int)((mx >> 7) & 0xFFu);
     sigma = (mx == 0) ? 0 : max(emax, 1) - 127 - 14;
-    bool bad = mx >= 0x7F80u;   // NaN / Inf: binary32 path
     const XScale xsc = make_xscale(sigma);
-    for (int i = threadIdx.x; i < R * nvec; i += kM1Threads) {
-        const int m = i / nvec, v = i % nvec;
-        uint4 out = make_uint4(0, 0, 0, 0);
-        if (m < M) {
-            const uint4 val = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)m * K + k0) + v);
-            out = make_uint4(x_pair_f16(val.x, xsc, bad), x_pair_f16(val.y, xsc, bad), x_pair_f16(val.z, xsc, bad),
-                             x_pair_f16(val.w, xsc, bad));
+    // exact: no NaN / Inf, and every nonzero |x| >= 2^(sigma - 17)
+    exact = mx < 0x7F80u && mn + 1u >= xsc.thr;
+    if (!exact) return;
+    bool unused = false;
+#pragma unroll
+    for (int u = 0; u < V; u++) {
+        const int i = threadIdx.x + u * kM1Threads;
+        if (i < total) {
+            const int q = i & 15, r = i >> 4, m = r % M, sc = r / M;
+            uint4 out;
+            if (xsc.one) {
+                out = make_uint4(x_pair_f16_scaled(val[u].x, xsc.p), x_pair_f16_scaled(val[u].y, xsc.p),
+                                 x_pair_f16_scaled(val[u].z, xsc.p), x_pair_f16_scaled(val[u].w, xsc.p));
+            } else {
+                out = make_uint4(x_pair_f16(val[u].x, xsc, unused), x_pair_f16(val[u].y, xsc, unused),
+                                 x_pair_f16(val[u].z, xsc, unused), x_pair_f16(val[u].w, xsc, unused));
+            }
+            // 16-byte piece j of lane t's 32 k of a super-chunk at piece 4j + t
+            *reinterpret_cast<uint4 *>(xs + (size_t)m * XS + sc * 128 + ((q & 3) * 4 + (q >> 2)) * 8) = out;
         }
-        *reinterpret_cast<uint4 *>(xs + (size_t)m * XS + v * 8) = out;
     }
-    if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) atomicOr(&flags[1], 1);
 }
 
 // The binary32 path of one CTA (x that could not be rescaled exactly into
@@ -85,11 +139,11 @@ __device__ __noinline__ void skinny_fallback(const GemvTcArgs &a, float *red, in
     for (int m = 0; m < M; m++) facc[m] = 0.0f;
     int cur = -1;
     auto flush = [&]() {
-        float *rb = red + ((size_t)cur * kM1Warps + warp) * kTcRows * M;
+        float *rb = red + ((size_t)cur * kM1Warps + warp) * kTcRows * skinny_pad(M);
 #pragma unroll
         for (int m = 0; m < M; m++) {
             facc[m] += __shfl_xor_sync(0xFFFFFFFFu, facc[m], 1);
-            if ((lane & 1) == 0) rb[(lane >> 1) * M + m] = scale_out(facc[m], gs, sref);
+            if ((lane & 1) == 0) rb[(lane >> 1) * skinny_pad(M) + m] = scale_out(facc[m], gs, sref);
             facc[m] = 0.0f;
         }
     };
@@ -125,6 +179,7 @@ template <int M>
 __global__ void __launch_bounds__(kM1Threads, 1) gemv_nvfp4_skinny_kernel(const GemvTcArgs a) {
     constexpr int NT = (M + 7) / 8;   // n-tiles of 8 tokens
     constexpr int D = M <= 8 ? 2 : 1; // super-chunks per batch (two batches in flight)
+    constexpr int MP = skinny_pad(M), M4 = MP / 4;
     extern __shared__ __align__(128) uint8_t smem[];
     const int K = a.K, N = a.N, kc = a.kc, XS = a.xstride;
     const int slice = blockIdx.y, nslices = gridDim.y;
@@ -142,7 +197,6 @@ __global__ void __launch_bounds__(kM1Threads, 1) gemv_nvfp4_skinny_kernel(const 
     const int nt = t1 - t0;
     const int g = lane >> 2, t4 = lane & 3;
 
-    if (threadIdx.x == 0) flags[1] = 0;
     pdl_allow_dependents();
     // the first batch of this warp's weights is loaded before waiting for the
     // previous kernel (and before x is ready)
@@ -152,12 +206,11 @@ __global__ void __launch_bounds__(kM1Threads, 1) gemv_nvfp4_skinny_kernel(const 
     m1_load(bA, it, a, warp, nt, SC, t0, k0, g, t4);
     const float gs = __ldg(a.gscale);
     pdl_wait_prior_grid();
-    __syncthreads();   // flags[1] is cleared
     int sigma;
     uint32_t mx;
-    skinny_convert_x<M>(a.x, K, k0, kcs, xs, XS, warp, lane, flags, sigma, mx);
+    bool fast;
+    skinny_convert_x<M>(a.x, K, k0, SC, xs, XS, warp, lane, flags, sigma, fast, mx);
     __syncthreads();
-    const bool fast = flags[1] == 0;
     const int fold = fast ? 0 : fallback_fold(gs, mx >= ((127u + 100u) << 7));   // largest |x| >= 2^100
     const int sref = fast ? sigma : -fold;
 
@@ -167,13 +220,13 @@ __global__ void __launch_bounds__(kM1Threads, 1) gemv_nvfp4_skinny_kernel(const 
     for (int q = 0; q < NT; q++) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.0f;
     // this warp's partial sums of tile cur -> shared memory
     auto flush = [&]() {
-        float *rb = red + ((size_t)cur * kM1Warps + warp) * kTcRows * M;
+        float *rb = red + ((size_t)cur * kM1Warps + warp) * kTcRows * MP;
 #pragma unroll
         for (int q = 0; q < NT; q++) {
 #pragma unroll
             for (int e = 0; e < 4; e++) {
                 const int row = g + 8 * (e >> 1), m = 8 * q + 2 * t4 + (e & 1);
-                if (m < M) rb[row * M + m] = scale_out(acc[q][e], gs, sref);
+                if (m < M) rb[row * MP + m] = scale_out(acc[q][e], gs, sref);
                 acc[q][e] = 0.0f;
             }
         }
@@ -192,12 +245,12 @@ __global__ void __launch_bounds__(kM1Threads, 1) gemv_nvfp4_skinny_kernel(const 
             decode_row32(b.c1[d], b.s1[d], h1);
 #pragma unroll
             for (int q = 0; q < NT; q++) {
-                // x of token 8q + g, k = 32t .. 32t+31 of the super-chunk
-                const uint4 *xp = reinterpret_cast<const uint4 *>(xs + (size_t)(8 * q + g) * XS + b.st[d] * 128 + 32 * t4);
+                // x of token 8q + g, k = 32t .. 32t+31 of the super-chunk (pieces 4v + t)
+                const uint4 *xp = reinterpret_cast<const uint4 *>(xs + (size_t)(8 * q + g) * XS + b.st[d] * 128) + t4;
                 uint32_t xv[16];
 #pragma unroll
                 for (int v = 0; v < 4; v++) {
-                    const uint4 u = xp[v];
+                    const uint4 u = xp[4 * v];
                     xv[4 * v] = u.x, xv[4 * v + 1] = u.y, xv[4 * v + 2] = u.z, xv[4 * v + 3] = u.w;
                 }
 #pragma unroll
@@ -222,21 +275,37 @@ __global__ void __launch_bounds__(kM1Threads, 1) gemv_nvfp4_skinny_kernel(const 
     }
     __syncthreads();
 
-    // rows of the CTA's tiles: the partials of the warps with a share of the tile, in warp order
-    for (int i = threadIdx.x; i < nt * kTcRows * M; i += kM1Threads) {
-        const int m = i % M, r = (i / M) % kTcRows, j = i / (M * kTcRows);
+    // rows of the CTA's tiles, four tokens at a time: the partials of the warps
+    // with a share of the tile, in warp order
+    const bool every = SC >= kM1Warps;   // every warp has a share of every tile
+    for (int i = threadIdx.x; i < nt * kTcRows * M4; i += kM1Threads) {
+        const int c = i % M4, r = (i / M4) % kTcRows, j = i / (M4 * kTcRows);
         const long long n = (long long)(t0 + j) * kTcRows + r;
         if (n >= N) continue;
-        float s = 0.0f;
+        const float4 *src = reinterpret_cast<const float4 *>(red + ((size_t)j * kM1Warps * kTcRows + r) * MP) + c;
+        float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
         for (int w = 0; w < kM1Warps; w++) {
-            int b, e;
-            m1_share(w, j, SC, b, e);
-            if (b < e) s += red[(((size_t)j * kM1Warps + w) * kTcRows + r) * M + m];
+            bool has = every;
+            if (!every) {
+                int b, e;
+                m1_share(w, j, SC, b, e);
+                has = b < e;
+            }
+            if (has) {
+                const float4 v = src[(size_t)w * kTcRows * M4];
+                s0 += v.x, s1 += v.y, s2 += v.z, s3 += v.w;
+            }
         }
-        if (nslices == 1)
-            a.y[(size_t)m * N + n] = s;
-        else
-            a.partial[((size_t)slice * M + m) * N + n] = s;
+        const float o[4] = {s0, s1, s2, s3};
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+            const int m = 4 * c + e;
+            if (m >= M) break;
+            if (nslices == 1)
+                a.y[(size_t)m * N + n] = o[e];
+            else
+                a.partial[((size_t)slice * M + m) * N + n] = o[e];
+        }
     }
 }
 

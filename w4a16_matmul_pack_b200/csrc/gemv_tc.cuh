@@ -136,6 +136,12 @@ __device__ __forceinline__ uint32_t x_pair_f16(uint32_t w, const XScale &xs, boo
     return *reinterpret_cast<const uint32_t *>(&h);
 }
 
+// Two BF16 values -> f16x2 of x * p (p = 2^-sigma, x known to convert exactly).
+__device__ __forceinline__ uint32_t x_pair_f16_scaled(uint32_t w, float p) {
+    const __half2 h = __floats2half2_rn(bf16_lo(w) * p, bf16_hi(w) * p);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
 constexpr int kTcRows = 16;                    // rows per tile (one MMA M)
 constexpr int kTcWarps = 8;                    // consumer warps, each a contiguous share of a tile's k
 constexpr int kTcParts = kTcWarps;

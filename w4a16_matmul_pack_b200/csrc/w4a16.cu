@@ -112,23 +112,22 @@ w4_status plan_gemv_m1(int K, int N, GemvTcPlan &p, int force_grid, const Device
 // NVFP4, M = 2..16 (gemv_skinny.cuh): K slices whose x' (rows padded to 8
 // tokens) fits kSkinnyXBytes; short problems are also split along K as for one
 // token; tiles per CTA as many as the partial-sum buffer holds.
-constexpr size_t kSkinnyXBytes = 96 * 1024;
 
 w4_status plan_gemv_skinny(int K, int N, int M, GemvTcPlan &p, const DeviceInfo &d) {
     p.M = M;
     const int R = (M + 7) / 8 * 8;
     const int T = (N + kTcRows - 1) / kTcRows;
-    const int kmax = std::max(256, (int)((kSkinnyXBytes / (2 * (size_t)R) - 8) / 256 * 256));
+    const int kmax = skinny_kmax(M);
     int S = (K + kmax - 1) / kmax;
     if (T < d.sms / 2) S = std::max(S, std::min(d.sms / T, K / 2048));
     S = std::max(S, 1);
     p.kc = ((K + S - 1) / S + 255) / 256 * 256;
     p.S = (K + p.kc - 1) / p.kc;
-    p.xstride = p.kc + 8;
+    p.xstride = p.kc + 32;   // rows 64 bytes apart modulo 128
     const size_t xbytes = ((size_t)R * p.xstride * 2 + 127) & ~(size_t)127;
-    const size_t per_tile = (size_t)kM1Warps * kTcRows * M * 4;
-    const size_t room = (size_t)d.smem_optin > xbytes + 4 * (2 + kM1Warps)
-                            ? (size_t)d.smem_optin - xbytes - 4 * (2 + kM1Warps) : 0;
+    const size_t per_tile = (size_t)kM1Warps * kTcRows * skinny_pad(M) * 4;
+    const size_t fbytes = 4 * (2 + 2 * kM1Warps);
+    const size_t room = (size_t)d.smem_optin > xbytes + fbytes ? (size_t)d.smem_optin - xbytes - fbytes : 0;
     const int red_max = (int)(room / per_tile);
     if (red_max < 1) return W4_ERR_UNSUPPORTED;
     p.grid = std::min(T, std::max(1, d.sms / p.S));
