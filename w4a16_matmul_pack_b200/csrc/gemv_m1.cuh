@@ -340,21 +340,22 @@ __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, 
     if (cur >= 0) flush();
     __syncthreads();
 
-    // rows of the CTA's tiles: the partials of the warps with a share of the tile, in warp order
-    const bool every = SC >= kM1Warps;   // every warp has a share of every tile
+    // rows of the CTA's tiles: the partials of the warps with a share of the tile,
+    // in warp order (all sixteen loads issued first; the entries of a warp
+    // without a share are never written and not added)
     for (int i = threadIdx.x; i < nt * kTcRows; i += kM1Threads) {
         const int j = i / kTcRows, r = i % kTcRows;
         const long long n = (long long)(t0 + j) * kTcRows + r;
         if (n >= N) continue;
+        float v[kM1Warps];
+#pragma unroll
+        for (int w = 0; w < kM1Warps; w++) v[w] = red[((size_t)j * kM1Warps + w) * kTcRows + r];
         float s = 0.0f;
+#pragma unroll
         for (int w = 0; w < kM1Warps; w++) {
-            bool has = every;
-            if (!every) {
-                int b, e;
-                m1_share(w, j, SC, b, e);
-                has = b < e;
-            }
-            if (has) s += red[((size_t)j * kM1Warps + w) * kTcRows + r];
+            int b, e;
+            m1_share(w, j, SC, b, e);
+            if (b < e) s += v[w];
         }
         if (nslices == 1)
             a.y[n] = s;

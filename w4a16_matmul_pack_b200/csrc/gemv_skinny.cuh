@@ -276,25 +276,22 @@ __global__ void __launch_bounds__(kM1Threads, 1) gemv_nvfp4_skinny_kernel(const 
     __syncthreads();
 
     // rows of the CTA's tiles, four tokens at a time: the partials of the warps
-    // with a share of the tile, in warp order
-    const bool every = SC >= kM1Warps;   // every warp has a share of every tile
+    // with a share of the tile, in warp order (all sixteen loads issued first;
+    // the entries of a warp without a share are never written and not added)
     for (int i = threadIdx.x; i < nt * kTcRows * M4; i += kM1Threads) {
         const int c = i % M4, r = (i / M4) % kTcRows, j = i / (M4 * kTcRows);
         const long long n = (long long)(t0 + j) * kTcRows + r;
         if (n >= N) continue;
         const float4 *src = reinterpret_cast<const float4 *>(red + ((size_t)j * kM1Warps * kTcRows + r) * MP) + c;
+        float4 v[kM1Warps];
+#pragma unroll
+        for (int w = 0; w < kM1Warps; w++) v[w] = src[(size_t)w * kTcRows * M4];
         float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
+#pragma unroll
         for (int w = 0; w < kM1Warps; w++) {
-            bool has = every;
-            if (!every) {
-                int b, e;
-                m1_share(w, j, SC, b, e);
-                has = b < e;
-            }
-            if (has) {
-                const float4 v = src[(size_t)w * kTcRows * M4];
-                s0 += v.x, s1 += v.y, s2 += v.z, s3 += v.w;
-            }
+            int b, e;
+            m1_share(w, j, SC, b, e);
+            if (b < e) s0 += v[w].x, s1 += v[w].y, s2 += v[w].z, s3 += v[w].w;
         }
         const float o[4] = {s0, s1, s2, s3};
 #pragma unroll
