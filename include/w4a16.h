@@ -240,8 +240,9 @@ w4_status w4a16_gemv_ex(const w4_weights *w, const void *x, int M, float *y,
  * y[p][N_p] = x[p][K_p] . w_hat[p] for p < G (the decode GEMV of the
  * "Nanbeige4.2-3B-NVFP4A16" card, Serving, applied to several weight matrices
  * that are ready together: the q, k and v projections of a layer read the same
- * x, as do gate and up).  The SMs are shared out in proportion to each
- * problem's packed bytes, so small matrices do not each pay a launch and a
+ * x, as do gate and up).  The SMs are shared out among the problems so
+ * that the most heavily loaded CTA (a CTA works on whole 16-row tiles) carries
+ * as few bytes as possible, and small matrices do not each pay a launch and a
  * pipeline fill.
  *   w      array of G NVFP4 weights (K_p % 256 == 0, K_p <= 32768).
  *   x      array of G device pointers to [K_p] BF16 (may repeat).
@@ -257,10 +258,11 @@ w4_status w4a16_gemv_grouped(const w4_weights *w, const void *const *x, float *c
 
 /*
  * w4_plan_grouped -- host only (no CUDA call): the CTAs w4a16_gemv_grouped
- * gives each problem on a GPU with `sms` SMs.  ctas[p] is proportional to
- * problem p's packed bytes (rounded down; the spare SMs go one at a time to the
- * problem with the most bytes per CTA), at least 1 and at most one per 16-row
- * tile; the total is min(sms, sum of the maxima) unless G forces more.
+ * gives each problem on a GPU with `sms` SMs.  With T_p 16-row tiles of b_p
+ * packed bytes, ctas[p] = ceil(T_p / floor(L / b_p)) for the smallest load L
+ * (bytes of the heaviest CTA) whose total fits in `sms`; the SMs left over go
+ * one at a time to the problem with the most bytes per CTA.  At least 1 and at
+ * most T_p each; the total is min(sms, sum of T_p) unless G forces more.
  *   w, G, flags  as for w4a16_gemv_grouped.  ctas  out int[G].
  */
 w4_status w4_plan_grouped(const w4_weights *w, int G, int sms, unsigned flags, int *ctas);

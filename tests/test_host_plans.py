@@ -23,21 +23,43 @@ def packed_bytes(w):
     return w.N * (w.K // 2 + w.K // 16)
 
 
-def test_sweep_shares_by_bytes():
+def tile_bytes(w):
+    return 16 * (w.K // 2 + w.K // 16)
+
+
+def heaviest_cta(ws, ctas):
+    """Bytes of the most loaded CTA: CTAs take balanced ranges of whole tiles."""
+    return max(math.ceil(math.ceil(w.N / 16) / c) * tile_bytes(w) for w, c in zip(ws, ctas))
+
+
+def best_load(ws, sms):
+    """Brute force over every possible load (a whole number of one problem's tiles)."""
+    best = None
+    for w in ws:
+        for k in range(1, math.ceil(w.N / 16) + 1):
+            L = k * tile_bytes(w)
+            need = sum(math.ceil(math.ceil(v.N / 16) / max(1, L // tile_bytes(v))) for v in ws)
+            if need <= sms and (best is None or L < best):
+                best = L
+    return best
+
+
+@pytest.mark.parametrize("sms", [148, 132, 100, 37])
+def test_sweep_minimises_the_heaviest_cta(sms):
     ws = [FakeNvfp4(K, N) for K, N in I.SWEEP_SHAPES]
-    ctas = W4.plan_grouped(ws, 148)
-    assert sum(ctas) == 148
+    ctas = W4.plan_grouped(ws, sms)
+    assert sum(ctas) == sms
     for w, c in zip(ws, ctas):
         assert 1 <= c <= math.ceil(w.N / 16)
-    ideal = sum(packed_bytes(w) for w in ws) / 148
-    per_cta = [packed_bytes(w) / c for w, c in zip(ws, ctas)]
-    assert max(per_cta) <= 1.1 * ideal          # the heaviest CTA stays close to an even share
-    # one more CTA for the heaviest problem would have to come from a problem
-    # whose CTAs would then carry more than the heaviest does now
-    p = max(range(len(ws)), key=lambda i: per_cta[i])
-    for q in range(len(ws)):
-        if q != p and ctas[q] > 1:
-            assert packed_bytes(ws[q]) / (ctas[q] - 1) >= per_cta[p] * 0.999
+    assert heaviest_cta(ws, ctas) == best_load(ws, sms)
+    # close to an even share of the bytes
+    assert heaviest_cta(ws, ctas) <= 1.25 * sum(packed_bytes(w) for w in ws) / sms
+
+
+def test_mixed_shapes_minimise_the_heaviest_cta():
+    ws = [FakeNvfp4(4096, 4096), FakeNvfp4(4096, 1024), FakeNvfp4(16384, 4096), FakeNvfp4(1024, 14336)]
+    ctas = W4.plan_grouped(ws, 148)
+    assert heaviest_cta(ws, ctas) == best_load(ws, 148)
 
 
 def test_caps_and_small_problems():

@@ -53,7 +53,8 @@ constexpr int kM1Threads = kM1Warps * 32;
 constexpr int kM1Depth = 2;   // super-chunks per batch (two batches in flight)
 
 // Shared memory of the one-token kernel: x' [xstride] f16, the partial sums
-// [red_tiles][kM1Warps][16] float, flags [2 + kM1Warps] int.
+// [red_tiles][kM1Warps][16] float, flags [2 + 2 * kM1Warps] int (the per-warp
+// largest and smallest magnitudes of x).
 struct M1Layout {
     size_t red, flags, total;
 };
@@ -62,7 +63,7 @@ __host__ __device__ __forceinline__ M1Layout m1_layout(int xstride, int red_tile
     M1Layout L;
     L.red = ((size_t)xstride * 2 + 127) & ~(size_t)127;
     L.flags = L.red + (size_t)red_tiles * kM1Warps * kTcRows * 4;
-    L.total = L.flags + 4 * (2 + kM1Warps);
+    L.total = L.flags + 4 * (2 + 2 * kM1Warps);
     return L;
 }
 
@@ -85,41 +86,76 @@ __device__ __forceinline__ float e4m3_hi_scaled(uint32_t v) { return __uint_as_f
 // zeros, so that every lane loads its four B pieces (or zeros) by address.
 constexpr int kM1ScStride = 136;   // halves per super-chunk
 
-// x slice (BF16, global) -> x' = x * 2^-sigma as f16 in that layout, with one
-// power of two for the slice (its largest |x'| in [2^14, 2^15)); flags[1] is
-// set when some x may not convert exactly (a nonzero |x'| below 2^-17: see
-// x_pair_f16) or is Inf / NaN.  All kM1Warps warps take part; flags[2 ..] is
-// scratch.  mx: the largest |x| (BF16 bits).
+// x slice (BF16, global) -> x' (f16, x * 2^-sigma) in the zero-padded B
+// layout.  Each thread keeps its pieces in registers between the two passes:
+// the largest magnitude and the smallest nonzero one (two 16-bit lanes at a
+// time) decide sigma and whether the f16 copy is exact, and only an exact copy
+// is written (otherwise the CTA computes in binary32 from global memory).
+constexpr int kM1MaxSlice = 32768;   // longest K slice of one CTA
+constexpr int kM1XPieces = kM1MaxSlice / 8 / kM1Threads;
+
 __device__ __forceinline__ void m1_convert_x(const uint16_t *xg, uint16_t *xs, int kcs, int warp, int lane,
-                                             int *flags, int &sigma, uint32_t &mx) {
+                                             int *flags, int &sigma, bool &exact, uint32_t &mx) {
     const uint4 *src = reinterpret_cast<const uint4 *>(xg);
     const int nvec = kcs / 8;
-    mx = 0;
-    for (int i = threadIdx.x; i < nvec; i += kM1Threads) {
-        const uint4 v = __ldg(src + i);
-        const uint32_t w4v[4] = {v.x, v.y, v.z, v.w};
+    uint4 val[kM1XPieces];
+    uint32_t mx2 = 0u, mn2 = 0xFFFFFFFFu;   // per 16-bit lane: max |x|, min (|x| - 1) over |x| != 0
 #pragma unroll
-        for (int j = 0; j < 4; j++) mx = max(mx, max(w4v[j] & 0x7FFFu, (w4v[j] >> 16) & 0x7FFFu));
+    for (int u = 0; u < kM1XPieces; u++) {
+        const int i = threadIdx.x + u * kM1Threads;
+        if (i < nvec) val[u] = __ldg(src + i);
     }
 #pragma unroll
-    for (int o = 16; o; o >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-    if (lane == 0) flags[2 + warp] = (int)mx;
+    for (int u = 0; u < kM1XPieces; u++) {
+        if (threadIdx.x + u * kM1Threads < nvec) {
+            const uint32_t w4v[4] = {val[u].x, val[u].y, val[u].z, val[u].w};
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const uint32_t mag = w4v[j] & 0x7FFF7FFFu;
+                mx2 = __vmaxu2(mx2, mag);
+                mn2 = __vminu2(mn2, (mag + 0x7FFF7FFFu) ^ 0x80008000u);   // 0 -> 0xFFFF, else |x| - 1
+            }
+        }
+    }
+    mx = max(mx2 & 0xFFFFu, mx2 >> 16);
+    uint32_t mn = min(mn2 & 0xFFFFu, mn2 >> 16);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+        mn = min(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
+    }
+    if (lane == 0) flags[2 + warp] = (int)mx, flags[2 + kM1Warps + warp] = (int)mn;
     __syncthreads();
-    for (int i = 0; i < kM1Warps; i++) mx = max(mx, (uint32_t)flags[2 + i]);
+#pragma unroll
+    for (int i = 0; i < kM1Warps; i++) {
+        mx = max(mx, (uint32_t)flags[2 + i]);
+        mn = min(mn, (uint32_t)flags[2 + kM1Warps + i]);
+    }
     const int emax = (int)((mx >> 7) & 0xFFu);
     sigma = (mx == 0) ? 0 : max(emax, 1) - 127 - 14;
-    bool bad = mx >= 0x7F80u;   // NaN / Inf: binary32 path
     const XScale xsc = make_xscale(sigma);
-    for (int i = threadIdx.x; i < nvec; i += kM1Threads) {
-        const int sc = i >> 4, q = i & 15;
-        const uint4 val = __ldg(src + i);
-        const uint32_t o[4] = {x_pair_f16(val.x, xsc, bad), x_pair_f16(val.y, xsc, bad), x_pair_f16(val.z, xsc, bad),
-                               x_pair_f16(val.w, xsc, bad)};
-        uint16_t *row = xs + (size_t)sc * kM1ScStride;
-        *reinterpret_cast<uint4 *>(row + ((q & 3) * 4 + (q >> 2)) * 8) = make_uint4(o[0], o[1], o[2], o[3]);
-        if (q == 0) *reinterpret_cast<uint4 *>(row + 128) = make_uint4(0, 0, 0, 0);
+    // exact: no NaN / Inf, and every nonzero |x| >= 2^(sigma - 17)
+    exact = mx < 0x7F80u && mn + 1u >= xsc.thr;
+    if (!exact) return;
+    bool unused = false;
+#pragma unroll
+    for (int u = 0; u < kM1XPieces; u++) {
+        const int i = threadIdx.x + u * kM1Threads;
+        if (i < nvec) {
+            const int sc = i >> 4, q = i & 15;
+            uint4 out;
+            if (xsc.one) {
+                out = make_uint4(x_pair_f16_scaled(val[u].x, xsc.p), x_pair_f16_scaled(val[u].y, xsc.p),
+                                 x_pair_f16_scaled(val[u].z, xsc.p), x_pair_f16_scaled(val[u].w, xsc.p));
+            } else {
+                out = make_uint4(x_pair_f16(val[u].x, xsc, unused), x_pair_f16(val[u].y, xsc, unused),
+                                 x_pair_f16(val[u].z, xsc, unused), x_pair_f16(val[u].w, xsc, unused));
+            }
+            uint16_t *row = xs + (size_t)sc * kM1ScStride;
+            *reinterpret_cast<uint4 *>(row + ((q & 3) * 4 + (q >> 2)) * 8) = out;
+            if (q == 0) *reinterpret_cast<uint4 *>(row + 128) = make_uint4(0, 0, 0, 0);
+        }
     }
-    if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) atomicOr(&flags[1], 1);
 }
 
 // Super-chunks [b, e) of tile j for warp w: the share of warp (w + j) mod 16.
@@ -196,7 +232,7 @@ __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, 
     const M1Layout L = m1_layout(a.xstride, a.red_tiles);
     uint16_t *xs = reinterpret_cast<uint16_t *>(smem);
     float *red = reinterpret_cast<float *>(smem + L.red);   // [tile][warp][16]
-    int *flags = reinterpret_cast<int *>(smem + L.flags);   // [1] x not exact in f16, [2..] per-warp max
+    int *flags = reinterpret_cast<int *>(smem + L.flags);   // [2..] per-warp statistics of x
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int T = (N + kTcRows - 1) / kTcRows;
@@ -205,7 +241,6 @@ __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, 
     const size_t RB = (size_t)K / 2, SB = (size_t)K / 16;   // row strides of codes and scales
     const int g = lane >> 2, t4 = lane & 3;
 
-    if (threadIdx.x == 0) flags[1] = 0;
     pdl_allow_dependents();
     // The weights do not depend on the previous kernel: the first batch of this
     // warp's items is loaded before waiting for it (and before x is ready).
@@ -217,12 +252,11 @@ __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, 
     pdl_wait_prior_grid();   // x (and y, which the previous kernel may read) belong to it
 
     // x slice -> f16 with one power of two, in the B-operand layout
-    __syncthreads();   // flags[1] is cleared
     int sigma;
     uint32_t mx;
-    m1_convert_x(a.x + k0, xs, kcs, warp, lane, flags, sigma, mx);
+    bool fast;
+    m1_convert_x(a.x + k0, xs, kcs, warp, lane, flags, sigma, fast, mx);
     __syncthreads();
-    const bool fast = flags[1] == 0;
     // binary32 path: partial sums in units of x * 2^fold
     const int fold = fast ? 0 : fallback_fold(gs, mx >= ((127u + 100u) << 7));   // largest |x| >= 2^100
     const int sref = fast ? sigma : -fold;

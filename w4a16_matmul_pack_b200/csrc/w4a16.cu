@@ -78,7 +78,6 @@ inline int block_bytes(int fmt) { return fmt == W4_FMT_ROCMFP4_DUAL ? 18 : 17; }
 // in shared memory as f16); a problem with fewer 16-row tiles than half the SMs
 // is also split along K (slices of at least 2048 k) so that the launch still
 // fills the GPU; at most kM1MaxTiles tiles per CTA (its partial-sum buffer).
-constexpr int kM1MaxSlice = 32768;
 constexpr int kM1MaxTiles = 32;
 
 w4_status plan_gemv_m1(int K, int N, GemvTcPlan &p, int force_grid, const DeviceInfo &d) {
@@ -318,34 +317,47 @@ w4_status launch_gemv_tc_m(const w4_weights *w, const void *x, float *y, void *w
     return launch_status();
 }
 
-// SMs shared out among G problems in proportion to their packed bytes (at
-// least one CTA each, at most max_cta[p]).
+// SMs shared out among G problems so that the heaviest CTA carries as few
+// bytes as whole 16-row tiles allow: with a load L, problem p needs
+// ceil(T_p / floor(L / b_p)) CTAs (T_p = max_cta[p] tiles of b_p bytes each),
+// and the smallest L whose CTAs fit in the SMs is found by bisection.  SMs
+// left over go one at a time to the problem whose CTAs carry the most bytes
+// on average (never more CTAs than tiles).  Every problem gets at least one
+// CTA, even when there are more problems than SMs.
 void share_sms(const w4_weights *w, int G, int sms, const int *max_cta, int *alloc) {
-    double bytes[kMaxGroup], total = 0.0;
-    int sum = 0;
+    long long tb[kMaxGroup], lo = 1, hi = 1;
     for (int p = 0; p < G; p++) {
-        bytes[p] = (double)w[p].N * (w[p].K / 2 + w[p].K / 16);
-        total += bytes[p];
+        tb[p] = (long long)kTcRows * (w[p].K / 2 + w[p].K / 16);
+        lo = std::max(lo, tb[p]);
+        hi = std::max(hi, tb[p] * max_cta[p]);
     }
-    for (int p = 0; p < G; p++) {
-        alloc[p] = std::max(1, std::min(max_cta[p], (int)(sms * bytes[p] / total)));
-        sum += alloc[p];
+    auto ctas_for = [&](long long L, int *a) {
+        long long sum = 0;
+        for (int p = 0; p < G; p++) {
+            const long long k = std::max<long long>(1, L / tb[p]);   // tiles per CTA
+            a[p] = (int)((max_cta[p] + k - 1) / k);
+            sum += a[p];
+        }
+        return sum;
+    };
+    if (ctas_for(hi, alloc) > sms) return;   // one CTA per problem
+    while (lo < hi) {
+        const long long mid = lo + (hi - lo) / 2;
+        if (ctas_for(mid, alloc) <= sms)
+            hi = mid;
+        else
+            lo = mid + 1;
     }
-    while (sum < sms) {   // spare SMs to the problem with the most bytes per CTA
+    long long sum = ctas_for(lo, alloc);
+    while (sum < sms) {
         int best = -1;
         for (int p = 0; p < G; p++)
-            if (alloc[p] < max_cta[p] && (best < 0 || bytes[p] / alloc[p] > bytes[best] / alloc[best])) best = p;
+            if (alloc[p] < max_cta[p] &&
+                (best < 0 || (double)tb[p] * max_cta[p] / alloc[p] > (double)tb[best] * max_cta[best] / alloc[best]))
+                best = p;
         if (best < 0) break;
         alloc[best]++;
         sum++;
-    }
-    while (sum > sms) {   // more problems than the rounding allows: take from the lightest CTAs
-        int best = -1;
-        for (int p = 0; p < G; p++)
-            if (alloc[p] > 1 && (best < 0 || bytes[p] / alloc[p] < bytes[best] / alloc[best])) best = p;
-        if (best < 0) break;
-        alloc[best]--;
-        sum--;
     }
 }
 
@@ -355,9 +367,9 @@ void grouped_max_cta(const w4_weights *w, int G, int *max_cta) {
 }
 
 // Several one-token NVFP4 problems in one launch (gemv_m1.cuh): the SMs are
-// shared out in proportion to each problem's packed bytes (at least one CTA
-// each, at most one per 16-row tile), and every CTA runs the single-problem
-// kernel body on a balanced range of its problem's rows.
+// shared out so that the heaviest CTA carries as few whole tiles' bytes as
+// possible (share_sms), and every CTA runs the single-problem kernel body on a
+// balanced range of its problem's tiles.
 w4_status launch_gemv_grouped(const w4_weights *w, const void *const *x, float *const *y, int G, bool pdl,
                               cudaStream_t st) {
     DeviceInfo d;
