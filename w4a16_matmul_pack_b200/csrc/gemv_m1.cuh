@@ -117,13 +117,8 @@ __device__ __forceinline__ void m1_convert_x(const uint16_t *xg, uint16_t *xs, i
             }
         }
     }
-    mx = max(mx2 & 0xFFFFu, mx2 >> 16);
-    uint32_t mn = min(mn2 & 0xFFFFu, mn2 >> 16);
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-        mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-        mn = min(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
-    }
+    mx = __reduce_max_sync(0xFFFFFFFFu, max(mx2 & 0xFFFFu, mx2 >> 16));
+    uint32_t mn = __reduce_min_sync(0xFFFFFFFFu, min(mn2 & 0xFFFFu, mn2 >> 16));
     if (lane == 0) flags[2 + warp] = (int)mx, flags[2 + kM1Warps + warp] = (int)mn;
     __syncthreads();
 #pragma unroll
@@ -194,29 +189,43 @@ struct M1Batch {
     uint32_t s0[D], s1[D];
 };
 
+// A lane's view of the CTA's weight rows: the codes and scales of row g of the
+// CTA's first tile at the lane's k offset in the K slice, and the last row of
+// the matrix relative to that tile.  Rows past it are read as that row (their
+// sums land in rows that are never written out), so the loads need no test.
+struct M1Rows {
+    const uint8_t *c, *s;
+    uint32_t RB, SB;   // row strides of codes and scales (bytes)
+    int rmax;          // N - 1 - first row of the CTA
+};
+
+__device__ __forceinline__ M1Rows m1_rows(const GemvTcArgs &a, int t0, int k0, int t4) {
+    M1Rows w;
+    const size_t RB = (size_t)a.K / 2, SB = (size_t)a.K / 16, row0 = (size_t)t0 * kTcRows;
+    w.c = a.codes + row0 * RB + (size_t)k0 / 2 + 16 * t4;
+    w.s = a.scales + row0 * SB + (size_t)k0 / 16 + 2 * t4;
+    w.RB = (uint32_t)RB;
+    w.SB = (uint32_t)SB;
+    w.rmax = (int)((long long)a.N - 1 - (long long)row0);
+    return w;
+}
+
 // Issue the loads of the warp's next D items (streaming: read once).
 template <int D>
-__device__ __forceinline__ void m1_load(M1Batch<D> &b, M1Items &it, const GemvTcArgs &a, int warp, int nt, int SC,
-                                        int t0, int k0, int g, int t4) {
-    const size_t RB = (size_t)a.K / 2, SB = (size_t)a.K / 16;
+__device__ __forceinline__ void m1_load(M1Batch<D> &b, M1Items &it, const M1Rows &w, int warp, int nt, int SC,
+                                        int g) {
 #pragma unroll
     for (int d = 0; d < D; d++) {
         b.jt[d] = it.j < nt ? it.j : -1;
         b.st[d] = it.s;
-        b.c0[d] = b.c1[d] = make_uint4(0, 0, 0, 0);
-        b.s0[d] = b.s1[d] = 0;
         if (b.jt[d] >= 0) {
-            const long long r0 = (long long)(t0 + b.jt[d]) * kTcRows + g, r1 = r0 + 8;
-            const size_t kb = (size_t)(k0 + b.st[d] * 128) / 2 + 16 * t4;
-            const size_t sb = (size_t)(k0 + b.st[d] * 128) / 16 + 2 * t4;
-            if (r0 < a.N) {
-                b.c0[d] = __ldcs(reinterpret_cast<const uint4 *>(a.codes + r0 * RB + kb));
-                b.s0[d] = __ldcs(reinterpret_cast<const unsigned short *>(a.scales + r0 * SB + sb));
-            }
-            if (r1 < a.N) {
-                b.c1[d] = __ldcs(reinterpret_cast<const uint4 *>(a.codes + r1 * RB + kb));
-                b.s1[d] = __ldcs(reinterpret_cast<const unsigned short *>(a.scales + r1 * SB + sb));
-            }
+            const uint32_t r0 = (uint32_t)min(b.jt[d] * kTcRows + g, w.rmax);
+            const uint32_t r1 = (uint32_t)min(b.jt[d] * kTcRows + g + 8, w.rmax);
+            const uint32_t kc = (uint32_t)b.st[d] * 64u, ks = (uint32_t)b.st[d] * 8u;
+            b.c0[d] = __ldcs(reinterpret_cast<const uint4 *>(w.c + ((uint64_t)r0 * w.RB + kc)));
+            b.c1[d] = __ldcs(reinterpret_cast<const uint4 *>(w.c + ((uint64_t)r1 * w.RB + kc)));
+            b.s0[d] = __ldcs(reinterpret_cast<const unsigned short *>(w.s + ((uint64_t)r0 * w.SB + ks)));
+            b.s1[d] = __ldcs(reinterpret_cast<const unsigned short *>(w.s + ((uint64_t)r1 * w.SB + ks)));
             it.next(warp, nt, SC);
         }
     }
@@ -247,7 +256,8 @@ __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, 
     M1Items it;
     it.first(warp, nt, SC);
     M1Batch<> bA, bB;
-    m1_load(bA, it, a, warp, nt, SC, t0, k0, g, t4);
+    const M1Rows wrows = m1_rows(a, t0, k0, t4);
+    m1_load(bA, it, wrows, warp, nt, SC, g);
     const float gs = __ldg(a.gscale);
     pdl_wait_prior_grid();   // x (and y, which the previous kernel may read) belong to it
 
@@ -336,10 +346,10 @@ __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, 
         // software pipeline: the next batch's loads are in flight while this one is multiplied
         for (;;) {
             if (bA.jt[0] < 0) break;
-            m1_load(bB, it, a, warp, nt, SC, t0, k0, g, t4);
+            m1_load(bB, it, wrows, warp, nt, SC, g);
             compute(bA);
             if (bB.jt[0] < 0) break;
-            m1_load(bA, it, a, warp, nt, SC, t0, k0, g, t4);
+            m1_load(bA, it, wrows, warp, nt, SC, g);
             compute(bB);
         }
     } else {

@@ -85,13 +85,8 @@ __device__ __forceinline__ void skinny_convert_x(const uint16_t *x, int K, int k
             }
         }
     }
-    mx = max(mx2 & 0xFFFFu, mx2 >> 16);
-    uint32_t mn = min(mn2 & 0xFFFFu, mn2 >> 16);
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-        mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-        mn = min(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
-    }
+    mx = __reduce_max_sync(0xFFFFFFFFu, max(mx2 & 0xFFFFu, mx2 >> 16));
+    uint32_t mn = __reduce_min_sync(0xFFFFFFFFu, min(mn2 & 0xFFFFu, mn2 >> 16));
     if (lane == 0) flags[2 + warp] = (int)mx, flags[2 + kM1Warps + warp] = (int)mn;
     __syncthreads();
     for (int i = 0; i < kM1Warps; i++) {
@@ -203,7 +198,8 @@ __global__ void __launch_bounds__(kM1Threads, 1) gemv_nvfp4_skinny_kernel(const 
     M1Items it;
     it.first(warp, nt, SC);
     M1Batch<D> bA, bB;
-    m1_load(bA, it, a, warp, nt, SC, t0, k0, g, t4);
+    const M1Rows wrows = m1_rows(a, t0, k0, t4);
+    m1_load(bA, it, wrows, warp, nt, SC, g);
     const float gs = __ldg(a.gscale);
     pdl_wait_prior_grid();
     int sigma;
@@ -263,10 +259,10 @@ __global__ void __launch_bounds__(kM1Threads, 1) gemv_nvfp4_skinny_kernel(const 
         // software pipeline: the next batch's loads are in flight while this one is multiplied
         for (;;) {
             if (bA.jt[0] < 0) break;
-            m1_load(bB, it, a, warp, nt, SC, t0, k0, g, t4);
+            m1_load(bB, it, wrows, warp, nt, SC, g);
             compute(bA);
             if (bB.jt[0] < 0) break;
-            m1_load(bA, it, a, warp, nt, SC, t0, k0, g, t4);
+            m1_load(bA, it, wrows, warp, nt, SC, g);
             compute(bB);
         }
         if (cur >= 0) flush();
