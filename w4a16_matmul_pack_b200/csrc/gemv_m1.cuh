@@ -75,12 +75,6 @@ __device__ __forceinline__ void decode_codes32(uint4 c, uint32_t (&h)[16]) {
     e2m1x8_to_f16x2(c.w, h + 12);
 }
 
-// E4M3 byte (bits 0..7 of v after the shift) -> its value * 2^-120 as binary32
-// bits: exponent and mantissa fields moved into place; an E4M3 subnormal becomes
-// a binary32 subnormal of the same scaled value.
-__device__ __forceinline__ float e4m3_lo_scaled(uint32_t v) { return __uint_as_float((v << 20) & 0x07F00000u); }
-__device__ __forceinline__ float e4m3_hi_scaled(uint32_t v) { return __uint_as_float((v << 12) & 0x07F00000u); }
-
 // x' in shared memory: per 128-k super-chunk the 128 values in MMA operand
 // order (the 8 values k = 32t + 8j .. +7 at offset 32j + 8t) followed by 8
 // zeros, so that every lane loads its four B pieces (or zeros) by address.
@@ -270,12 +264,11 @@ __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, 
     // binary32 path: partial sums in units of x * 2^fold
     const int fold = fast ? 0 : fallback_fold(gs, mx >= ((127u + 100u) << 7));   // largest |x| >= 2^100
     const int sref = fast ? sigma : -fold;
-    const float p120 = __int_as_float((127 + 120) << 23);   // e4m3_*_scaled(s) * 2^120 = s
 
     // MMA operands.  Lane (g, t) holds rows g, g+8 of the codes of k = 32t .. 32t+31
     // (blocks 2t, 2t+1) and B column g.  Column g is block g: it is nonzero only for
-    // the k of lanes t = g/2, and only in the MMAs of block g (the first four MMAs
-    // for even g, the last four for odd g).  So lane (g, t) takes its B pieces
+    // the k of lanes t = g/2, and only in the MMAs of block g (the four over the
+    // first 16 of those k for even g, over the last 16 for odd g).  So lane (g, t) takes its B pieces
     // j = 0..3 (x of k = 32t + 8j .. +7) from x' when g/2 == t and j/2 == g%2,
     // and from the super-chunk's eight zeros otherwise: four loads by address.
     const bool xact = (g >> 1) == t4;
@@ -323,23 +316,24 @@ __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, 
             uint32_t h0[16], h1[16];
             decode_codes32(b.c0[d], h0);
             decode_codes32(b.c1[d], h1);
-            // four independent chains of two MMAs (the MMA latency, not its
-            // rate, is what a chain of eight would cost)
+            // two chains of four MMAs: block 2t in column 2t of d0, block 2t+1 in column 2t+1 of d1
             float d0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, d1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-            float e0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, e1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
             mma_f16_16816(d0, h0[0], h1[0], h0[1], h1[1], b0.x, b0.y);
-            mma_f16_16816(e0, h0[2], h1[2], h0[3], h1[3], b0.z, b0.w);
             mma_f16_16816(d1, h0[8], h1[8], h0[9], h1[9], b2.x, b2.y);
-            mma_f16_16816(e1, h0[10], h1[10], h0[11], h1[11], b2.z, b2.w);
+            mma_f16_16816(d0, h0[2], h1[2], h0[3], h1[3], b0.z, b0.w);
+            mma_f16_16816(d1, h0[10], h1[10], h0[11], h1[11], b2.z, b2.w);
             mma_f16_16816(d0, h0[4], h1[4], h0[5], h1[5], b1.x, b1.y);
-            mma_f16_16816(e0, h0[6], h1[6], h0[7], h1[7], b1.z, b1.w);
             mma_f16_16816(d1, h0[12], h1[12], h0[13], h1[13], b3.x, b3.y);
-            mma_f16_16816(e1, h0[14], h1[14], h0[15], h1[15], b3.z, b3.w);
-            // d0 + e0 holds block 2t in column 2t, d1 + e1 block 2t+1 in column 2t+1
-            accA = __fmaf_rn(e4m3_lo_scaled(b.s0[d]) * p120, d0[0] + e0[0], accA);
-            accA = __fmaf_rn(e4m3_hi_scaled(b.s0[d]) * p120, d1[1] + e1[1], accA);
-            accB = __fmaf_rn(e4m3_lo_scaled(b.s1[d]) * p120, d0[2] + e0[2], accB);
-            accB = __fmaf_rn(e4m3_hi_scaled(b.s1[d]) * p120, d1[3] + e1[3], accB);
+            mma_f16_16816(d0, h0[6], h1[6], h0[7], h1[7], b1.z, b1.w);
+            mma_f16_16816(d1, h0[14], h1[14], h0[15], h1[15], b3.z, b3.w);
+            // the two scales of each row, exact in f16 and then in binary32
+            const uint32_t sa = e4m3x2_to_f16x2(b.s0[d]), sb = e4m3x2_to_f16x2(b.s1[d]);
+            const float2 fa = __half22float2(*reinterpret_cast<const __half2 *>(&sa));
+            const float2 fb = __half22float2(*reinterpret_cast<const __half2 *>(&sb));
+            accA = __fmaf_rn(fa.x, d0[0], accA);
+            accA = __fmaf_rn(fa.y, d1[1], accA);
+            accB = __fmaf_rn(fb.x, d0[2], accB);
+            accB = __fmaf_rn(fb.y, d1[3], accB);
         }
     };
     if (fast) {
