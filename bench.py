@@ -758,7 +758,7 @@ def run_reference(args, world, rank):
 # five sweep matrices, with the SHA-256 of the kernel sources it was measured
 # on.  The bench reports it only while those sources are unchanged.
 TRAFFIC = {"bytes": 41384960, "source_sha256": "efa8f076790253dadabb26aae671a4089879ffafbdf8d1cb9b93deeaf0ffce28"}
-TRAFFIC_SOURCES = ("common.cuh", "gemv_tc.cuh", "gemv_m1.cuh")
+TRAFFIC_SOURCES = ("common.cuh", "gemv_tc.cuh", "gemv_m1.cuh", "w4a16.cu")
 
 
 def kernel_source_sha256() -> str:
