@@ -26,20 +26,20 @@
 // at HBM speed -- on B200 a ring of shared-memory stages fed by bulk copies
 // delivered less per SM than direct loads for this access pattern.
 //
-// Work split.  A CTA owns whole 16-row tiles [t0, t1) of one K slice; every
-// warp takes a contiguous share of the super-chunks of every tile (the share
-// rotates with the tile, so that a slice whose super-chunk count is not a
-// multiple of 16 does not load the same warps every time), writes its partial
-// sums of each tile to shared memory, and the CTA adds the partials of a row in
-// a fixed order: the result does not depend on timing.
+// Work split.  A CTA owns whole 16-row tiles [t0, t1) of one K slice.  Its
+// (tile, super-chunk) items, tile by tile, are cut into sixteen contiguous runs,
+// one per warp, so that a warp changes tile (and flushes its partial sums to
+// shared memory) only a few times; the CTA adds the partials of a row in warp
+// order: the result does not depend on timing.
 //
 // x is converted to f16 once per CTA, as x * 2^-sigma with one power of two
 // for the whole slice (its largest |x'| in [2^14, 2^15)), exact whenever every
 // nonzero |x'| >= 2^-17, and permuted per 128-k super-chunk to the MMA operand
 // order.  A CTA whose x does not convert exactly (range above 2^31, Inf/NaN)
 // computes in binary32 on the CUDA cores from the bf16 x in global memory.  A
-// warp's partial sum is scaled to acc * g * 2^sigma in binary64 (scale_out)
-// before the partials are added.
+// warp's partial sum is scaled to acc * g * 2^sigma in binary64 (the factor
+// g * 2^sigma is exact there; one rounding to binary32) before the partials are
+// added.
 //
 // The kernel waits on nothing but its own loads and CTA barriers.
 #pragma once
@@ -147,30 +147,40 @@ __device__ __forceinline__ void m1_convert_x(const uint16_t *xg, uint16_t *xs, i
     }
 }
 
-// Super-chunks [b, e) of tile j for warp w: the share of warp (w + j) mod 16.
-__device__ __forceinline__ void m1_share(int w, int j, int SC, int &b, int &e) {
-    const int wr = (w + j) % kM1Warps;
-    b = wr * SC / kM1Warps;
-    e = (wr + 1) * SC / kM1Warps;
+// The CTA's items in order: item i is super-chunk i % SC of tile i / SC.  Warp
+// w takes the contiguous run [w n / 16, (w + 1) n / 16) of the n = nt * SC
+// items, so it crosses few tile boundaries (each one costs a flush of its
+// partial sums).
+__device__ __forceinline__ void m1_range(int w, int nt, int SC, int &lo, int &hi) {
+    const int n = nt * SC;
+    lo = w * n / kM1Warps;
+    hi = (w + 1) * n / kM1Warps;
 }
 
-// Walks warp w's (tile, super-chunk) items of tiles [0, nt) in order.
+// Whether warp w has items of tile j (and so partial sums of it).
+__device__ __forceinline__ bool m1_has(int w, int j, int nt, int SC) {
+    int lo, hi;
+    m1_range(w, nt, SC, lo, hi);
+    return lo < hi && lo < (j + 1) * SC && hi > j * SC;
+}
+
+// Walks warp w's items: tile j (nt once done), super-chunk s.
 struct M1Items {
-    int j, s, e;
+    int j, s, left;
     __device__ __forceinline__ void first(int w, int nt, int SC) {
-        j = 0;
-        m1_share(w, 0, SC, s, e);
-        skip_empty(w, nt, SC);
+        int lo, hi;
+        m1_range(w, nt, SC, lo, hi);
+        left = hi - lo;
+        j = left > 0 ? lo / SC : nt;
+        s = lo - (lo / SC) * SC;
     }
-    __device__ __forceinline__ void skip_empty(int w, int nt, int SC) {
-        while (j < nt && s >= e) {
+    __device__ __forceinline__ void next(int, int nt, int SC) {
+        if (--left == 0) {
+            j = nt;
+        } else if (++s == SC) {
+            s = 0;
             j++;
-            if (j < nt) m1_share(w, j, SC, s, e);
         }
-    }
-    __device__ __forceinline__ void next(int w, int nt, int SC) {
-        s++;
-        skip_empty(w, nt, SC);
     }
 };
 
@@ -264,6 +274,7 @@ __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, 
     // binary32 path: partial sums in units of x * 2^fold
     const int fold = fast ? 0 : fallback_fold(gs, mx >= ((127u + 100u) << 7));   // largest |x| >= 2^100
     const int sref = fast ? sigma : -fold;
+    const double osc = out_factor(gs, sref);   // partial sums -> units of y
 
     // MMA operands.  Lane (g, t) holds rows g, g+8 of the codes of k = 32t .. 32t+31
     // (blocks 2t, 2t+1) and B column g.  Column g is block g: it is nonzero only for
@@ -288,12 +299,12 @@ __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, 
             accB += __shfl_xor_sync(0xFFFFFFFFu, accB, 1);
             accB += __shfl_xor_sync(0xFFFFFFFFu, accB, 2);
             if (t4 == 0) {
-                rb[g] = scale_out(accA, gs, sref);
-                rb[g + 8] = scale_out(accB, gs, sref);
+                rb[g] = scale_by(accA, osc);
+                rb[g + 8] = scale_by(accB, osc);
             }
         } else {
             accA += __shfl_xor_sync(0xFFFFFFFFu, accA, 1);
-            if ((lane & 1) == 0) rb[lane >> 1] = scale_out(accA, gs, sref);
+            if ((lane & 1) == 0) rb[lane >> 1] = scale_by(accA, osc);
         }
         accA = 0.0f;
         accB = 0.0f;
@@ -390,11 +401,8 @@ __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, 
         for (int w = 0; w < kM1Warps; w++) v[w] = red[((size_t)j * kM1Warps + w) * kTcRows + r];
         float s = 0.0f;
 #pragma unroll
-        for (int w = 0; w < kM1Warps; w++) {
-            int b, e;
-            m1_share(w, j, SC, b, e);
-            if (b < e) s += v[w];
-        }
+        for (int w = 0; w < kM1Warps; w++)
+            if (m1_has(w, j, nt, SC)) s += v[w];
         if (nslices == 1)
             a.y[n] = s;
         else

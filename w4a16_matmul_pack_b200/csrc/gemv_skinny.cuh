@@ -127,6 +127,7 @@ template <int M>
 __device__ __noinline__ void skinny_fallback(const GemvTcArgs &a, float *red, int warp, int lane, int nt, int SC,
                                              int t0, int k0, float gs, int fold, int sref) {
     const int K = a.K, N = a.N;
+    const double osc = out_factor(gs, sref);
     const size_t RB = (size_t)K / 2, SB = (size_t)K / 16;
     const int row = lane >> 1, half = lane & 1;
     float facc[M];
@@ -138,7 +139,7 @@ __device__ __noinline__ void skinny_fallback(const GemvTcArgs &a, float *red, in
 #pragma unroll
         for (int m = 0; m < M; m++) {
             facc[m] += __shfl_xor_sync(0xFFFFFFFFu, facc[m], 1);
-            if ((lane & 1) == 0) rb[(lane >> 1) * skinny_pad(M) + m] = scale_out(facc[m], gs, sref);
+            if ((lane & 1) == 0) rb[(lane >> 1) * skinny_pad(M) + m] = scale_by(facc[m], osc);
             facc[m] = 0.0f;
         }
     };
@@ -209,6 +210,7 @@ __global__ void __launch_bounds__(kM1Threads, 1) gemv_nvfp4_skinny_kernel(const 
     __syncthreads();
     const int fold = fast ? 0 : fallback_fold(gs, mx >= ((127u + 100u) << 7));   // largest |x| >= 2^100
     const int sref = fast ? sigma : -fold;
+    const double osc = out_factor(gs, sref);   // partial sums -> units of y
 
     int cur = -1;                       // tile being accumulated
     float acc[NT][4];                   // MMA C fragments (rows g, g+8 x tokens 8nt + 2t, +1)
@@ -222,7 +224,7 @@ __global__ void __launch_bounds__(kM1Threads, 1) gemv_nvfp4_skinny_kernel(const 
 #pragma unroll
             for (int e = 0; e < 4; e++) {
                 const int row = g + 8 * (e >> 1), m = 8 * q + 2 * t4 + (e & 1);
-                if (m < M) rb[row * MP + m] = scale_out(acc[q][e], gs, sref);
+                if (m < M) rb[row * MP + m] = scale_by(acc[q][e], osc);
                 acc[q][e] = 0.0f;
             }
         }
@@ -284,11 +286,8 @@ __global__ void __launch_bounds__(kM1Threads, 1) gemv_nvfp4_skinny_kernel(const 
         for (int w = 0; w < kM1Warps; w++) v[w] = src[(size_t)w * kTcRows * M4];
         float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
 #pragma unroll
-        for (int w = 0; w < kM1Warps; w++) {
-            int b, e;
-            m1_share(w, j, SC, b, e);
-            if (b < e) s0 += v[w].x, s1 += v[w].y, s2 += v[w].z, s3 += v[w].w;
-        }
+        for (int w = 0; w < kM1Warps; w++)
+            if (m1_has(w, j, nt, SC)) s0 += v[w].x, s1 += v[w].y, s2 += v[w].z, s3 += v[w].w;
         const float o[4] = {s0, s1, s2, s3};
 #pragma unroll
         for (int e = 0; e < 4; e++) {

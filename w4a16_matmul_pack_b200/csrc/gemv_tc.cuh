@@ -83,6 +83,14 @@ __device__ __forceinline__ float scale_out(float v, float g, int e) {
     return (float)((double)v * (double)g * p2);
 }
 
+// g * 2^e in binary64 (exact for |e| <= 400).  (double)v times it, rounded once
+// (scale_by), is the exact v * g * 2^e rounded once: scale_out bit for bit, with
+// the factor computed once per CTA.
+__device__ __forceinline__ double out_factor(float g, int e) {
+    return (double)g * __longlong_as_double((long long)(1023 + e) << 52);
+}
+__device__ __forceinline__ float scale_by(float v, double f) { return (float)((double)v * f); }
+
 // Power of two folded into the decoded weights of the binary32 fallback paths:
 // the exponent of g, clamped to [-100, 0], when x reaches 2^100 (else 0).  Sums
 // of x * e2m1 * 2^fold (and their products with the block scale) then stay near
