@@ -279,72 +279,80 @@ __device__ __forceinline__ float epilogue_factor(float g, int e) {
 
 // Row m of x -> f16 as x * 2^-sigma_m, sigma_m chosen so that the row's largest
 // |x * 2^-sigma_m| lies in [2^14, 2^15); bad[m] = 1 when some nonzero value
-// lands below 2^-17 (then it may be inexact in f16) or the row holds Inf / NaN.
-// One warp per row, eight rows per block; every launch rewrites sigma and bad of
-// every row.  Rows of up to kXRowVec * 32 * 8 values are read once (kept in
-// registers); longer rows are read twice.
-constexpr int kXRowVec = 16;
+// lies below 2^(sigma_m - 17) (then x * 2^-sigma_m may be inexact in f16) or
+// the row holds Inf / NaN.  One CTA of four warps per row, so that enough rows
+// are in flight to hide the load latency; every launch rewrites sigma and bad
+// of every row.  Rows of up to kXcVec * kXcThreads * 8 values are read once
+// (kept in registers); longer rows are read twice.
+constexpr int kXcThreads = 128;
+constexpr int kXcWarps = kXcThreads / 32;
+constexpr int kXcVec = 8;
 
-__device__ __forceinline__ uint4 x_row_to_f16(uint4 v, int sg, bool &b) {
-    const float tiny = 7.62939453125e-06f;   // 2^-17
+// Per 16-bit lane: the largest magnitude, and the smallest of (|x| - 1) over
+// |x| != 0 (0 -> 0xFFFF), of eight BF16 values.
+__device__ __forceinline__ void x_stats8(uint4 v, uint32_t &mx2, uint32_t &mn2) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t o[4];
 #pragma unroll
     for (int j = 0; j < 4; j++) {
-        const float a0 = mul_pow2(__uint_as_float(w[j] << 16), -sg), a1 = mul_pow2(__uint_as_float(w[j] & 0xFFFF0000u), -sg);
-        b |= (a0 != 0.0f && fabsf(a0) < tiny) | (a1 != 0.0f && fabsf(a1) < tiny);
-        const __half2 hv = __floats2half2_rn(a0, a1);
-        o[j] = *reinterpret_cast<const uint32_t *>(&hv);
+        const uint32_t mag = w[j] & 0x7FFF7FFFu;
+        mx2 = __vmaxu2(mx2, mag);
+        mn2 = __vminu2(mn2, (mag + 0x7FFF7FFFu) ^ 0x80008000u);
     }
-    return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-__device__ __forceinline__ uint32_t absmax_bf16x8(uint32_t mx, uint4 v) {
-    mx = __vmaxu2(mx, v.x & 0x7FFF7FFFu);
-    mx = __vmaxu2(mx, v.y & 0x7FFF7FFFu);
-    mx = __vmaxu2(mx, v.z & 0x7FFF7FFFu);
-    return __vmaxu2(mx, v.w & 0x7FFF7FFFu);
+__device__ __forceinline__ uint4 x_row_to_f16(uint4 v, const XScale &xs) {
+    if (xs.one)
+        return make_uint4(x_pair_f16_scaled(v.x, xs.p), x_pair_f16_scaled(v.y, xs.p), x_pair_f16_scaled(v.z, xs.p),
+                          x_pair_f16_scaled(v.w, xs.p));
+    bool unused = false;
+    return make_uint4(x_pair_f16(v.x, xs, unused), x_pair_f16(v.y, xs, unused), x_pair_f16(v.z, xs, unused),
+                      x_pair_f16(v.w, xs, unused));
 }
 
-__global__ void __launch_bounds__(256) x_to_f16_kernel(const uint16_t *x, uint16_t *xh, int *sigma, int *bad, int M,
-                                                       int K) {
+__global__ void __launch_bounds__(kXcThreads) x_to_f16_kernel(const uint16_t *x, uint16_t *xh, int *sigma, int *bad,
+                                                              int M, int K) {
+    __shared__ uint32_t red[2][kXcWarps];
     pdl_allow_dependents();   // the GEMM may start its prologue; it waits for this grid before reading x
-    const int m = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-    if (m >= M) return;   // whole warps
+    const int m = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)m * K);
     uint4 *dst = reinterpret_cast<uint4 *>(xh + (size_t)m * K);
     const int nv = K / 8;
-    const bool in_regs = nv <= kXRowVec * 32;
-    uint4 keep[kXRowVec];
-    uint32_t mx = 0;
+    const bool in_regs = nv <= kXcVec * kXcThreads;
+    uint4 keep[kXcVec];
+    uint32_t mx2 = 0u, mn2 = 0xFFFFFFFFu;
     if (in_regs) {
 #pragma unroll
-        for (int r = 0; r < kXRowVec; r++) {
-            const int i = lane + r * 32;
-            keep[r] = i < nv ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
-            mx = absmax_bf16x8(mx, keep[r]);
+        for (int r = 0; r < kXcVec; r++) {
+            const int i = threadIdx.x + r * kXcThreads;
+            if (i < nv) keep[r] = __ldg(src + i);
         }
-    } else {
-        for (int i = lane; i < nv; i += 32) mx = absmax_bf16x8(mx, __ldg(src + i));
-    }
-    mx = max(mx & 0xFFFFu, mx >> 16);
 #pragma unroll
-    for (int o = 16; o; o >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+        for (int r = 0; r < kXcVec; r++)
+            if (threadIdx.x + r * kXcThreads < nv) x_stats8(keep[r], mx2, mn2);
+    } else {
+        for (int i = threadIdx.x; i < nv; i += kXcThreads) x_stats8(__ldg(src + i), mx2, mn2);
+    }
+    uint32_t mx = __reduce_max_sync(0xFFFFFFFFu, max(mx2 & 0xFFFFu, mx2 >> 16));
+    uint32_t mn = __reduce_min_sync(0xFFFFFFFFu, min(mn2 & 0xFFFFu, mn2 >> 16));
+    if (lane == 0) red[0][warp] = mx, red[1][warp] = mn;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < kXcWarps; w++) mx = max(mx, red[0][w]), mn = min(mn, red[1][w]);
     const int sg = (mx == 0) ? 0 : max((int)(mx >> 7), 1) - 127 - 14;
-    bool b = mx >= 0x7F80u;
+    const XScale xs = make_xscale(sg);
     if (in_regs) {
 #pragma unroll
-        for (int r = 0; r < kXRowVec; r++) {
-            const int i = lane + r * 32;
-            if (i < nv) dst[i] = x_row_to_f16(keep[r], sg, b);
+        for (int r = 0; r < kXcVec; r++) {
+            const int i = threadIdx.x + r * kXcThreads;
+            if (i < nv) dst[i] = x_row_to_f16(keep[r], xs);
         }
     } else {
-        for (int i = lane; i < nv; i += 32) dst[i] = x_row_to_f16(__ldg(src + i), sg, b);
+        for (int i = threadIdx.x; i < nv; i += kXcThreads) dst[i] = x_row_to_f16(__ldg(src + i), xs);
     }
-    const bool any = __any_sync(0xFFFFFFFFu, b);
-    if (lane == 0) {
+    if (threadIdx.x == 0) {
         sigma[m] = sg;
-        bad[m] = any ? 1 : 0;
+        // Inf / NaN, or a nonzero |x| below 2^(sigma - 17) (mn + 1: the smallest nonzero magnitude)
+        bad[m] = (mx >= 0x7F80u || mn + 1u < xs.thr) ? 1 : 0;
     }
 }
 
@@ -755,7 +763,7 @@ inline w4_status gemm_launch_fmt(const w4_weights *w, const void *x, int M, floa
     p.bad = bad;
     p.sigma = sigma;
     if (f16)
-        x_to_f16_kernel<<<(M + 7) / 8, 256, 0, st>>>(reinterpret_cast<const uint16_t *>(x), xh, sigma, bad, M, K);
+        x_to_f16_kernel<<<M, kXcThreads, 0, st>>>(reinterpret_cast<const uint16_t *>(x), xh, sigma, bad, M, K);
     const int ntiles = p.tiles_m * p.tiles_n;
     const int grid = std::max(1, std::min(ntiles, sms));   // persistent, one CTA per SM
     cudaLaunchConfig_t cfg = {};
