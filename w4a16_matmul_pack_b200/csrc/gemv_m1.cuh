@@ -87,22 +87,25 @@ constexpr int kM1ScStride = 136;   // halves per super-chunk
 // is written (otherwise the CTA computes in binary32 from global memory).
 constexpr int kM1MaxSlice = 32768;   // longest K slice of one CTA
 constexpr int kM1XPieces = kM1MaxSlice / 8 / kM1Threads;
+constexpr int kM1XRegs = 3;   // pieces a thread keeps in registers (slices up to 12288 k); later ones are read twice
 
 __device__ __forceinline__ void m1_convert_x(const uint16_t *xg, uint16_t *xs, int kcs, int warp, int lane,
                                              int *flags, int &sigma, bool &exact, uint32_t &mx) {
     const uint4 *src = reinterpret_cast<const uint4 *>(xg);
     const int nvec = kcs / 8;
-    uint4 val[kM1XPieces];
+    uint4 val[kM1XRegs];
     uint32_t mx2 = 0u, mn2 = 0xFFFFFFFFu;   // per 16-bit lane: max |x|, min (|x| - 1) over |x| != 0
 #pragma unroll
-    for (int u = 0; u < kM1XPieces; u++) {
+    for (int u = 0; u < kM1XRegs; u++) {
         const int i = threadIdx.x + u * kM1Threads;
         if (i < nvec) val[u] = __ldg(src + i);
     }
 #pragma unroll
     for (int u = 0; u < kM1XPieces; u++) {
-        if (threadIdx.x + u * kM1Threads < nvec) {
-            const uint32_t w4v[4] = {val[u].x, val[u].y, val[u].z, val[u].w};
+        const int i = threadIdx.x + u * kM1Threads;
+        if (i < nvec) {
+            const uint4 v = u < kM1XRegs ? val[u] : __ldg(src + i);
+            const uint32_t w4v[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int j = 0; j < 4; j++) {
                 const uint32_t mag = w4v[j] & 0x7FFF7FFFu;
@@ -132,13 +135,14 @@ __device__ __forceinline__ void m1_convert_x(const uint16_t *xg, uint16_t *xs, i
         const int i = threadIdx.x + u * kM1Threads;
         if (i < nvec) {
             const int sc = i >> 4, q = i & 15;
+            const uint4 v = u < kM1XRegs ? val[u] : __ldg(src + i);
             uint4 out;
             if (xsc.one) {
-                out = make_uint4(x_pair_f16_scaled(val[u].x, xsc.p), x_pair_f16_scaled(val[u].y, xsc.p),
-                                 x_pair_f16_scaled(val[u].z, xsc.p), x_pair_f16_scaled(val[u].w, xsc.p));
+                out = make_uint4(x_pair_f16_scaled(v.x, xsc.p), x_pair_f16_scaled(v.y, xsc.p),
+                                 x_pair_f16_scaled(v.z, xsc.p), x_pair_f16_scaled(v.w, xsc.p));
             } else {
-                out = make_uint4(x_pair_f16(val[u].x, xsc, unused), x_pair_f16(val[u].y, xsc, unused),
-                                 x_pair_f16(val[u].z, xsc, unused), x_pair_f16(val[u].w, xsc, unused));
+                out = make_uint4(x_pair_f16(v.x, xsc, unused), x_pair_f16(v.y, xsc, unused),
+                                 x_pair_f16(v.z, xsc, unused), x_pair_f16(v.w, xsc, unused));
             }
             uint16_t *row = xs + (size_t)sc * kM1ScStride;
             *reinterpret_cast<uint4 *>(row + ((q & 3) * 4 + (q >> 2)) * 8) = out;
@@ -214,6 +218,17 @@ __device__ __forceinline__ M1Rows m1_rows(const GemvTcArgs &a, int t0, int k0, i
     return w;
 }
 
+// 16 code bytes, read once (evict-first).  The 256-byte L2 fetch size brings
+// the row's next three super-chunks into L2 with this one: a warp's run walks
+// a tile's super-chunks in order, so its later loads of the row hit L2.
+__device__ __forceinline__ uint4 ld_codes16(const uint8_t *p) {
+    uint4 v;
+    asm volatile("ld.global.cs.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
 // Issue the loads of the warp's next D items (streaming: read once).
 template <int D>
 __device__ __forceinline__ void m1_load(M1Batch<D> &b, M1Items &it, const M1Rows &w, int warp, int nt, int SC,
@@ -226,8 +241,8 @@ __device__ __forceinline__ void m1_load(M1Batch<D> &b, M1Items &it, const M1Rows
             const uint32_t r0 = (uint32_t)min(b.jt[d] * kTcRows + g, w.rmax);
             const uint32_t r1 = (uint32_t)min(b.jt[d] * kTcRows + g + 8, w.rmax);
             const uint32_t kc = (uint32_t)b.st[d] * 64u, ks = (uint32_t)b.st[d] * 8u;
-            b.c0[d] = __ldcs(reinterpret_cast<const uint4 *>(w.c + ((uint64_t)r0 * w.RB + kc)));
-            b.c1[d] = __ldcs(reinterpret_cast<const uint4 *>(w.c + ((uint64_t)r1 * w.RB + kc)));
+            b.c0[d] = ld_codes16(w.c + ((uint64_t)r0 * w.RB + kc));
+            b.c1[d] = ld_codes16(w.c + ((uint64_t)r1 * w.RB + kc));
             b.s0[d] = __ldcs(reinterpret_cast<const unsigned short *>(w.s + ((uint64_t)r0 * w.SB + ks)));
             b.s1[d] = __ldcs(reinterpret_cast<const unsigned short *>(w.s + ((uint64_t)r1 * w.SB + ks)));
             it.next(warp, nt, SC);
@@ -255,13 +270,14 @@ __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, 
     const int g = lane >> 2, t4 = lane & 3;
 
     pdl_allow_dependents();
-    // The weights do not depend on the previous kernel: the first batch of this
-    // warp's items is loaded before waiting for it (and before x is ready).
+    // The weights do not depend on the previous kernel: the first two batches of
+    // this warp's items are loaded before waiting for it (and before x is ready).
     M1Items it;
     it.first(warp, nt, SC);
     M1Batch<> bA, bB;
     const M1Rows wrows = m1_rows(a, t0, k0, t4);
     m1_load(bA, it, wrows, warp, nt, SC, g);
+    m1_load(bB, it, wrows, warp, nt, SC, g);
     const float gs = __ldg(a.gscale);
     pdl_wait_prior_grid();   // x (and y, which the previous kernel may read) belong to it
 
@@ -348,14 +364,15 @@ __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, 
         }
     };
     if (fast) {
-        // software pipeline: the next batch's loads are in flight while this one is multiplied
+        // software pipeline: one batch's loads are in flight while the other is
+        // multiplied (both were issued before the wait for the previous kernel)
         for (;;) {
             if (bA.jt[0] < 0) break;
-            m1_load(bB, it, wrows, warp, nt, SC, g);
             compute(bA);
-            if (bB.jt[0] < 0) break;
             m1_load(bA, it, wrows, warp, nt, SC, g);
+            if (bB.jt[0] < 0) break;
             compute(bB);
+            m1_load(bB, it, wrows, warp, nt, SC, g);
         }
     } else {
         // binary32 on the CUDA cores: lane l takes row l/2 of the tile, 64 k of each super-chunk
