@@ -32,10 +32,11 @@
 // shared memory) only a few times; the CTA adds the partials of a row in warp
 // order: the result does not depend on timing.
 //
-// x is converted to f16 once per CTA, as x * 2^-sigma with one power of two
-// for the whole slice (its largest |x'| in [2^14, 2^15)), exact whenever every
-// nonzero |x'| >= 2^-17, and permuted per 128-k super-chunk to the MMA operand
-// order.  A CTA whose x does not convert exactly (range above 2^31, Inf/NaN)
+// x is converted to f16 once per CTA, as x itself when every nonzero |x| lies
+// in [2^-17, 65280] (decided with one barrier), else as x * 2^-sigma with one
+// power of two for the whole slice (its largest |x'| in [2^14, 2^15)), exact
+// whenever every nonzero |x'| >= 2^-17; either way permuted per 128-k
+// super-chunk to the MMA operand order.  A CTA whose x does not convert exactly (range above 2^31, Inf/NaN)
 // computes in binary32 on the CUDA cores from the bf16 x in global memory.  A
 // warp's partial sum is scaled to acc * g * 2^sigma in binary64 (the factor
 // g * 2^sigma is exact there; one rounding to binary32) before the partials are
@@ -81,10 +82,12 @@ __device__ __forceinline__ void decode_codes32(uint4 c, uint32_t (&h)[16]) {
 constexpr int kM1ScStride = 136;   // halves per super-chunk
 
 // x slice (BF16, global) -> x' (f16, x * 2^-sigma) in the zero-padded B
-// layout.  Each thread keeps its pieces in registers between the two passes:
-// the largest magnitude and the smallest nonzero one (two 16-bit lanes at a
-// time) decide sigma and whether the f16 copy is exact, and only an exact copy
-// is written (otherwise the CTA computes in binary32 from global memory).
+// layout, ending with a CTA barrier.  x is first written with sigma = 0 and
+// kept when every value converts exactly (one barrier decides).  Otherwise
+// each thread keeps its pieces in registers between two more passes: the
+// largest magnitude and the smallest nonzero one (two 16-bit lanes at a time)
+// decide sigma and whether the f16 copy is exact, and only an exact copy is
+// written (otherwise the CTA computes in binary32 from global memory).
 constexpr int kM1MaxSlice = 32768;   // longest K slice of one CTA
 constexpr int kM1XPieces = kM1MaxSlice / 8 / kM1Threads;
 constexpr int kM1XRegs = 3;   // pieces a thread keeps in registers (slices up to 12288 k); later ones are read twice
@@ -99,6 +102,40 @@ __device__ __forceinline__ void m1_convert_x(const uint16_t *xg, uint16_t *xs, i
     for (int u = 0; u < kM1XRegs; u++) {
         const int i = threadIdx.x + u * kM1Threads;
         if (i < nvec) val[u] = __ldg(src + i);
+    }
+    // First try sigma = 0 (x as it is), decided with a single barrier: every
+    // nonzero |x| in [2^-17, 65280] (BF16 bits 0x3700 .. 0x477F) converts
+    // exactly.  The partial sums do not depend on sigma (powers of two scale
+    // every product and sum exactly), so this only saves the statistics pass
+    // when x is in that range -- as activations normally are.
+    bool ok = true;
+#pragma unroll
+    for (int u = 0; u < kM1XPieces; u++) {
+        const int i = threadIdx.x + u * kM1Threads;
+        if (i < nvec) {
+            const uint4 v = u < kM1XRegs ? val[u] : __ldg(src + i);
+            const uint32_t w4v[4] = {v.x, v.y, v.z, v.w};
+            uint32_t hi2 = 0u, lo2 = 0xFFFFFFFFu;
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const uint32_t mag = w4v[j] & 0x7FFF7FFFu;
+                hi2 = __vmaxu2(hi2, mag);
+                lo2 = __vminu2(lo2, (mag + 0x7FFF7FFFu) ^ 0x80008000u);   // 0 -> 0xFFFF, else |x| - 1
+            }
+            ok &= max(hi2 & 0xFFFFu, hi2 >> 16) <= 0x477Fu && min(lo2 & 0xFFFFu, lo2 >> 16) + 1u >= 0x3700u;
+            const int sc = i >> 4, q = i & 15;
+            uint16_t *row = xs + (size_t)sc * kM1ScStride;
+            *reinterpret_cast<uint4 *>(row + ((q & 3) * 4 + (q >> 2)) * 8) =
+                make_uint4(x_pair_f16_scaled(v.x, 1.0f), x_pair_f16_scaled(v.y, 1.0f), x_pair_f16_scaled(v.z, 1.0f),
+                           x_pair_f16_scaled(v.w, 1.0f));
+            if (q == 0) *reinterpret_cast<uint4 *>(row + 128) = make_uint4(0, 0, 0, 0);
+        }
+    }
+    if (__syncthreads_and(ok)) {   // also the barrier after the x' writes
+        sigma = 0;
+        exact = true;
+        mx = 0u;
+        return;
     }
 #pragma unroll
     for (int u = 0; u < kM1XPieces; u++) {
@@ -128,7 +165,7 @@ __device__ __forceinline__ void m1_convert_x(const uint16_t *xg, uint16_t *xs, i
     const XScale xsc = make_xscale(sigma);
     // exact: no NaN / Inf, and every nonzero |x| >= 2^(sigma - 17)
     exact = mx < 0x7F80u && mn + 1u >= xsc.thr;
-    if (!exact) return;
+    if (!exact) return;   // (uniform: the caller's binary32 path reads no x')
     bool unused = false;
 #pragma unroll
     for (int u = 0; u < kM1XPieces; u++) {
@@ -149,6 +186,7 @@ __device__ __forceinline__ void m1_convert_x(const uint16_t *xg, uint16_t *xs, i
             if (q == 0) *reinterpret_cast<uint4 *>(row + 128) = make_uint4(0, 0, 0, 0);
         }
     }
+    __syncthreads();
 }
 
 // The CTA's items in order: item i is super-chunk i % SC of tile i / SC.  Warp
@@ -285,8 +323,7 @@ __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, 
     int sigma;
     uint32_t mx;
     bool fast;
-    m1_convert_x(a.x + k0, xs, kcs, warp, lane, flags, sigma, fast, mx);
-    __syncthreads();
+    m1_convert_x(a.x + k0, xs, kcs, warp, lane, flags, sigma, fast, mx);   // ends with a barrier
     // binary32 path: partial sums in units of x * 2^fold
     const int fold = fast ? 0 : fallback_fold(gs, mx >= ((127u + 100u) << 7));   // largest |x| >= 2^100
     const int sref = fast ? sigma : -fold;
