@@ -51,10 +51,12 @@ __host__ __device__ __forceinline__ M1Layout skinny_layout(int M, int xstride, i
 }
 
 // x[M][K] slice (BF16, global; SC super-chunks of 128 k from k0) -> x' rows
-// (f16, x * 2^-sigma).  Each thread holds its pieces in registers between the
-// two passes: the largest magnitude and the smallest nonzero one (two 16-bit
-// lanes at a time) decide sigma and whether the f16 copy is exact; only then
-// is it written.  Token rows M .. 8*NT-1 are left as they are: they only feed
+// (f16, x * 2^-sigma), ending with a CTA barrier.  x is first written with
+// sigma = 0 and kept when every value converts exactly (one barrier decides).
+// Otherwise each thread holds its pieces in registers between two more
+// passes: the largest magnitude and the smallest nonzero one (two 16-bit lanes
+// at a time) decide sigma and whether the f16 copy is exact; only then is it
+// written.  Token rows M .. 8*NT-1 are left as they are: they only feed
 // MMA columns whose sums are never read.
 template <int M>
 __device__ __forceinline__ void skinny_convert_x(const uint16_t *x, int K, int k0, int SC, uint16_t *xs, int XS,
@@ -70,6 +72,39 @@ __device__ __forceinline__ void skinny_convert_x(const uint16_t *x, int K, int k
         if (i < total) {
             const int q = i & 15, r = i >> 4, m = r % M, sc = r / M;
             val[u] = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)m * K + k0 + sc * 128) + q);
+        }
+    }
+    // First try sigma = 0 (x as it is), decided with one barrier: every nonzero
+    // |x| in [2^-17, 65280] (BF16 bits 0x3700 .. 0x477F) converts exactly, and
+    // the partial sums do not depend on sigma (powers of two scale every product
+    // and sum exactly).  Up to 8 tokens only: above that the extra pass costs
+    // the fast path registers (measured slower at 16 tokens).
+    if constexpr (M <= 8) {
+        bool ok = true;
+#pragma unroll
+        for (int u = 0; u < V; u++) {
+            const int i = threadIdx.x + u * kM1Threads;
+            if (i < total) {
+                const int q = i & 15, r = i >> 4, m = r % M, sc = r / M;
+                const uint32_t w4v[4] = {val[u].x, val[u].y, val[u].z, val[u].w};
+                uint32_t hi2 = 0u, lo2 = 0xFFFFFFFFu;
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    const uint32_t mag = w4v[j] & 0x7FFF7FFFu;
+                    hi2 = __vmaxu2(hi2, mag);
+                    lo2 = __vminu2(lo2, (mag + 0x7FFF7FFFu) ^ 0x80008000u);
+                }
+                ok &= max(hi2 & 0xFFFFu, hi2 >> 16) <= 0x477Fu && min(lo2 & 0xFFFFu, lo2 >> 16) + 1u >= 0x3700u;
+                *reinterpret_cast<uint4 *>(xs + (size_t)m * XS + sc * 128 + ((q & 3) * 4 + (q >> 2)) * 8) =
+                    make_uint4(x_pair_f16_scaled(val[u].x, 1.0f), x_pair_f16_scaled(val[u].y, 1.0f),
+                               x_pair_f16_scaled(val[u].z, 1.0f), x_pair_f16_scaled(val[u].w, 1.0f));
+            }
+        }
+        if (__syncthreads_and(ok)) {   // also the barrier after the x' writes
+            sigma = 0;
+            exact = true;
+            mx = 0u;
+            return;
         }
     }
 #pragma unroll
@@ -117,6 +152,7 @@ __device__ __forceinline__ void skinny_convert_x(const uint16_t *x, int K, int k
             *reinterpret_cast<uint4 *>(xs + (size_t)m * XS + sc * 128 + ((q & 3) * 4 + (q >> 2)) * 8) = out;
         }
     }
+    __syncthreads();
 }
 
 // The binary32 path of one CTA (x that could not be rescaled exactly into
@@ -206,8 +242,7 @@ __global__ void __launch_bounds__(kM1Threads, 1) gemv_nvfp4_skinny_kernel(const 
     int sigma;
     uint32_t mx;
     bool fast;
-    skinny_convert_x<M>(a.x, K, k0, SC, xs, XS, warp, lane, flags, sigma, fast, mx);
-    __syncthreads();
+    skinny_convert_x<M>(a.x, K, k0, SC, xs, XS, warp, lane, flags, sigma, fast, mx);   // ends with a barrier
     const int fold = fast ? 0 : fallback_fold(gs, mx >= ((127u + 100u) << 7));   // largest |x| >= 2^100
     const int sref = fast ? sigma : -fold;
     const double osc = out_factor(gs, sref);   // partial sums -> units of y
