@@ -150,6 +150,8 @@ __global__ void __launch_bounds__(256) gemv_any_kernel(const uint8_t *__restrict
 // y[m][n] = g * sum_s partial[s][m][n], slices in order.
 __global__ void gemv_finalize_kernel(const float *__restrict__ partial, int S, int MN,
                                      const float *__restrict__ gscale, float *__restrict__ y) {
+    pdl_allow_dependents();
+    pdl_wait_prior_grid();   // the slices' partials (a no-op without programmatic dependent launch)
     const float g = gscale ? __ldg(gscale) : 1.0f;
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < MN; i += gridDim.x * blockDim.x) {
         float s = 0.0f;

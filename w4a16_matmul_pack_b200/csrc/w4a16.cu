@@ -311,8 +311,17 @@ w4_status launch_gemv_tc_m(const w4_weights *w, const void *x, float *y, void *w
     if (e != cudaSuccess) return W4_ERR_CUDA;
     if (p.S > 1) {
         const int MN = M * N;
-        // the slice partials already carry the global scale (scale_out)
-        gemv_finalize_kernel<<<std::min((MN + 255) / 256, 1024), 256, 0, st>>>(a.partial, p.S, MN, nullptr, y);
+        // the slice partials already carry the global scale (scale_out); with
+        // PDL the adds launch early and wait for the slices in the kernel
+        cudaLaunchConfig_t fc = {};
+        fc.gridDim = dim3(std::min((MN + 255) / 256, 1024), 1, 1);
+        fc.blockDim = dim3(256, 1, 1);
+        fc.stream = st;
+        fc.attrs = attr;
+        fc.numAttrs = pdl ? 1 : 0;
+        if (cudaLaunchKernelEx(&fc, gemv_finalize_kernel, (const float *)a.partial, p.S, MN, (const float *)nullptr,
+                               y) != cudaSuccess)
+            return W4_ERR_CUDA;
     }
     return launch_status();
 }
