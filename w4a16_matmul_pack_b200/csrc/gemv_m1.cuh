@@ -267,29 +267,41 @@ __device__ __forceinline__ uint4 ld_codes16(const uint8_t *p) {
     return v;
 }
 
-// Issue the loads of the warp's next D items (streaming: read once).
+// Issue the loads of the warp's next item into slot d of a batch (streaming:
+// read once); the slot's tile becomes -1 once the warp's items run out.
+template <int D>
+__device__ __forceinline__ void m1_load_one(M1Batch<D> &b, int d, M1Items &it, const M1Rows &w, int warp, int nt,
+                                            int SC, int g) {
+    b.jt[d] = it.j < nt ? it.j : -1;
+    b.st[d] = it.s;
+    if (b.jt[d] >= 0) {
+        const uint32_t r0 = (uint32_t)min(b.jt[d] * kTcRows + g, w.rmax);
+        const uint32_t r1 = (uint32_t)min(b.jt[d] * kTcRows + g + 8, w.rmax);
+        const uint32_t kc = (uint32_t)b.st[d] * 64u, ks = (uint32_t)b.st[d] * 8u;
+        b.c0[d] = ld_codes16(w.c + ((uint64_t)r0 * w.RB + kc));
+        b.c1[d] = ld_codes16(w.c + ((uint64_t)r1 * w.RB + kc));
+        b.s0[d] = __ldcs(reinterpret_cast<const unsigned short *>(w.s + ((uint64_t)r0 * w.SB + ks)));
+        b.s1[d] = __ldcs(reinterpret_cast<const unsigned short *>(w.s + ((uint64_t)r1 * w.SB + ks)));
+        it.next(warp, nt, SC);
+    }
+}
+
+// Issue the loads of the warp's next D items.
 template <int D>
 __device__ __forceinline__ void m1_load(M1Batch<D> &b, M1Items &it, const M1Rows &w, int warp, int nt, int SC,
                                         int g) {
 #pragma unroll
-    for (int d = 0; d < D; d++) {
-        b.jt[d] = it.j < nt ? it.j : -1;
-        b.st[d] = it.s;
-        if (b.jt[d] >= 0) {
-            const uint32_t r0 = (uint32_t)min(b.jt[d] * kTcRows + g, w.rmax);
-            const uint32_t r1 = (uint32_t)min(b.jt[d] * kTcRows + g + 8, w.rmax);
-            const uint32_t kc = (uint32_t)b.st[d] * 64u, ks = (uint32_t)b.st[d] * 8u;
-            b.c0[d] = ld_codes16(w.c + ((uint64_t)r0 * w.RB + kc));
-            b.c1[d] = ld_codes16(w.c + ((uint64_t)r1 * w.RB + kc));
-            b.s0[d] = __ldcs(reinterpret_cast<const unsigned short *>(w.s + ((uint64_t)r0 * w.SB + ks)));
-            b.s1[d] = __ldcs(reinterpret_cast<const unsigned short *>(w.s + ((uint64_t)r1 * w.SB + ks)));
-            it.next(warp, nt, SC);
-        }
-    }
+    for (int d = 0; d < D; d++) m1_load_one(b, d, it, w, warp, nt, SC, g);
 }
 
 // The kernel body for one CTA: CTA `cta` of `ncta` working on tiles of one
 // problem, K-slice `slice` of `nslices` (split-K partials when nslices > 1).
+//
+// REFILL: each item's registers get the warp's next item as soon as the item is
+// decoded (loads in flight earlier; the grouped launch, measured faster there),
+// else a batch's slots are refilled after the whole batch (fewer registers: the
+// single-problem kernel, whose split-K bookkeeping leaves no room for REFILL).
+template <bool REFILL>
 __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, int slice, int nslices) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int K = a.K, N = a.N, kc = a.kc;
@@ -362,8 +374,10 @@ __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, 
         accA = 0.0f;
         accB = 0.0f;
     };
-    // the math of one batch (fast path)
-    auto compute = [&](const M1Batch<> &b) {
+    // the math of one batch (fast path); with REFILL each item's slot takes the
+    // warp's next item as soon as its codes and scales are decoded, so that
+    // load is in flight while the item's MMAs and the rest of the batch run
+    auto compute = [&](M1Batch<> &b) {
 #pragma unroll
         for (int d = 0; d < kM1Depth; d++) {
             if (b.jt[d] < 0) break;
@@ -380,6 +394,9 @@ __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, 
             uint32_t h0[16], h1[16];
             decode_codes32(b.c0[d], h0);
             decode_codes32(b.c1[d], h1);
+            // the two scales of each row, exact in f16 and then in binary32
+            const uint32_t sa = e4m3x2_to_f16x2(b.s0[d]), sb = e4m3x2_to_f16x2(b.s1[d]);
+            if constexpr (REFILL) m1_load_one(b, d, it, wrows, warp, nt, SC, g);
             // two chains of four MMAs: block 2t in column 2t of d0, block 2t+1 in column 2t+1 of d1
             float d0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, d1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
             mma_f16_16816(d0, h0[0], h1[0], h0[1], h1[1], b0.x, b0.y);
@@ -390,8 +407,6 @@ __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, 
             mma_f16_16816(d1, h0[12], h1[12], h0[13], h1[13], b3.x, b3.y);
             mma_f16_16816(d0, h0[6], h1[6], h0[7], h1[7], b1.z, b1.w);
             mma_f16_16816(d1, h0[14], h1[14], h0[15], h1[15], b3.z, b3.w);
-            // the two scales of each row, exact in f16 and then in binary32
-            const uint32_t sa = e4m3x2_to_f16x2(b.s0[d]), sb = e4m3x2_to_f16x2(b.s1[d]);
             const float2 fa = __half22float2(*reinterpret_cast<const __half2 *>(&sa));
             const float2 fb = __half22float2(*reinterpret_cast<const __half2 *>(&sb));
             accA = __fmaf_rn(fa.x, d0[0], accA);
@@ -406,10 +421,10 @@ __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, 
         for (;;) {
             if (bA.jt[0] < 0) break;
             compute(bA);
-            m1_load(bA, it, wrows, warp, nt, SC, g);
+            if constexpr (!REFILL) m1_load(bA, it, wrows, warp, nt, SC, g);
             if (bB.jt[0] < 0) break;
             compute(bB);
-            m1_load(bB, it, wrows, warp, nt, SC, g);
+            if constexpr (!REFILL) m1_load(bB, it, wrows, warp, nt, SC, g);
         }
     } else {
         // binary32 on the CUDA cores: lane l takes row l/2 of the tile, 64 k of each super-chunk
@@ -465,7 +480,7 @@ __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, 
 }
 
 __global__ void __launch_bounds__(kM1Threads, 1) gemv_nvfp4_m1_kernel(const GemvTcArgs a) {
-    m1_body(a, blockIdx.x, gridDim.x, blockIdx.y, gridDim.y);
+    m1_body<false>(a, blockIdx.x, gridDim.x, blockIdx.y, gridDim.y);
 }
 
 // Several independent one-token problems in one launch (e.g. the q, k and v
@@ -483,7 +498,7 @@ struct GroupArgs {
 __global__ void __launch_bounds__(kM1Threads, 1) gemv_nvfp4_m1_grouped_kernel(const __grid_constant__ GroupArgs g) {
     int p = 0;
     while (p + 1 < g.G && (int)blockIdx.x >= g.cta0[p + 1]) p++;
-    m1_body(g.a[p], (int)blockIdx.x - g.cta0[p], g.cta0[p + 1] - g.cta0[p], 0, 1);
+    m1_body<true>(g.a[p], (int)blockIdx.x - g.cta0[p], g.cta0[p + 1] - g.cta0[p], 0, 1);
 }
 
 }  // namespace w4
