@@ -82,12 +82,14 @@ __device__ __forceinline__ void decode_codes32(uint4 c, uint32_t (&h)[16]) {
 constexpr int kM1ScStride = 136;   // halves per super-chunk
 
 // x slice (BF16, global) -> x' (f16, x * 2^-sigma) in the zero-padded B
-// layout, ending with a CTA barrier.  x is first written with sigma = 0 and
-// kept when every value converts exactly (one barrier decides).  Otherwise
-// each thread keeps its pieces in registers between two more passes: the
-// largest magnitude and the smallest nonzero one (two 16-bit lanes at a time)
-// decide sigma and whether the f16 copy is exact, and only an exact copy is
-// written (otherwise the CTA computes in binary32 from global memory).
+// layout, ending with a CTA barrier whenever x' is used (a CTA whose x does not
+// convert exactly returns without one: its binary32 path reads no x').  x is
+// first written with sigma = 0 and kept when every value converts exactly (one
+// barrier decides).  Otherwise each thread keeps its pieces in registers
+// between two more passes: the largest magnitude and the smallest nonzero one
+// (two 16-bit lanes at a time) decide sigma and whether the f16 copy is exact,
+// and only an exact copy is written (otherwise the CTA computes in binary32
+// from global memory).
 constexpr int kM1MaxSlice = 32768;   // longest K slice of one CTA
 constexpr int kM1XPieces = kM1MaxSlice / 8 / kM1Threads;
 constexpr int kM1XRegs = 3;   // pieces a thread keeps in registers (slices up to 12288 k); later ones are read twice
@@ -335,7 +337,7 @@ __device__ __forceinline__ void m1_body(const GemvTcArgs &a, int cta, int ncta, 
     int sigma;
     uint32_t mx;
     bool fast;
-    m1_convert_x(a.x + k0, xs, kcs, warp, lane, flags, sigma, fast, mx);   // ends with a barrier
+    m1_convert_x(a.x + k0, xs, kcs, warp, lane, flags, sigma, fast, mx);   // barrier when x' is used
     // binary32 path: partial sums in units of x * 2^fold
     const int fold = fast ? 0 : fallback_fold(gs, mx >= ((127u + 100u) << 7));   // largest |x| >= 2^100
     const int sref = fast ? sigma : -fold;

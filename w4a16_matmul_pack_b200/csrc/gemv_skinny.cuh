@@ -51,7 +51,8 @@ __host__ __device__ __forceinline__ M1Layout skinny_layout(int M, int xstride, i
 }
 
 // x[M][K] slice (BF16, global; SC super-chunks of 128 k from k0) -> x' rows
-// (f16, x * 2^-sigma), ending with a CTA barrier.  x is first written with
+// (f16, x * 2^-sigma), ending with a CTA barrier whenever x' is used (the
+// binary32 path of an inexact x reads no x').  x is first written with
 // sigma = 0 and kept when every value converts exactly (one barrier decides).
 // Otherwise each thread holds its pieces in registers between two more
 // passes: the largest magnitude and the smallest nonzero one (two 16-bit lanes
@@ -242,7 +243,7 @@ __global__ void __launch_bounds__(kM1Threads, 1) gemv_nvfp4_skinny_kernel(const 
     int sigma;
     uint32_t mx;
     bool fast;
-    skinny_convert_x<M>(a.x, K, k0, SC, xs, XS, warp, lane, flags, sigma, fast, mx);   // ends with a barrier
+    skinny_convert_x<M>(a.x, K, k0, SC, xs, XS, warp, lane, flags, sigma, fast, mx);   // barrier when x' is used
     const int fold = fast ? 0 : fallback_fold(gs, mx >= ((127u + 100u) << 7));   // largest |x| >= 2^100
     const int sref = fast ? sigma : -fold;
     const double osc = out_factor(gs, sref);   // partial sums -> units of y
