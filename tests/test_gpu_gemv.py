@@ -321,3 +321,36 @@ def test_huge_range_grouped(case):
         pw, wh = nvfp4_packed(W.contiguous())
         pws.append(pw); whs.append(wh); xs.append(x)
     check_group(pws, whs, xs)
+
+
+@pytest.mark.parametrize("M", [1, 4, 9])
+def test_x_conversion_paths_agree(M):
+    """x whose every value converts to f16 as it is takes the one-barrier
+    conversion with no power of two (up to 8 tokens); the same x times 2^20
+    exceeds f16 and takes the conversion with a power of two.  A power of two
+    scales every product and partial sum exactly, so the two outputs must differ
+    by exactly 2^20, and both meet the oracle's bound.  x holding the edges of
+    the unscaled range (2^-17, 65280), or values just outside it (2^-18, 65536),
+    must meet it too."""
+    K, N = 2560, 512
+    pw, wh = nvfp4_packed(I.sweep_weights(K, N, 4)[:N].contiguous())
+    x = I.activations(M, K, 41 + M)
+    y = run_and_check(pw, wh, x)
+    y_big = run_and_check(pw, wh, I.bf16_rne(x.double() * 2.0 ** 20))
+    assert torch.equal(y_big, y * 2.0 ** 20)
+    for lo, hi in ((2.0 ** -17, 65280.0), (2.0 ** -18, 65536.0)):
+        xe = x.double().clone()
+        xe[:, 7], xe[:, 8], xe[:, 9], xe[:, 10] = lo, -lo, hi, -hi
+        run_and_check(pw, wh, I.bf16_rne(xe))
+
+
+def test_grouped_x_conversion_paths_agree():
+    """The grouped one-token launch: the same two conversions, the same exact 2^20."""
+    K, N = 2560, 512
+    pw, wh = nvfp4_packed(I.sweep_weights(K, N, 5)[:N].contiguous())
+    x = I.activations(1, K, 43)
+    xb = I.bf16_rne(x.double() * 2.0 ** 20)
+    y, y_big = W4.w4a16_gemv_grouped([pw, pw], [x.cuda(), xb.cuda()])
+    yr, ar = O.matmul(x, wh)
+    assert_within_tolerance(np_of(y), yr, ar)
+    assert torch.equal(y_big, y * 2.0 ** 20)
